@@ -1,0 +1,329 @@
+// C ABI of the library: argument checks, the geometry plan, workspace
+// layout, and the launch sequence K1 -> K2 -> K3 on the caller's stream.
+//
+// Argument rules follow lite_boost.ops.sparse_attention (input_layout must be
+// BSND or BNSD; scale defaults to head_dim ** -0.5; sparsity in [0, 1];
+// output shaped like q) and vllm-omni "RainFusion Attention" (sparsity finite
+// in [0, 1]; 128-token blocks; fewer than 32 video blocks or no geometry is
+// dense attention).
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <mutex>
+#include <string>
+
+#include "rf_geometry.h"
+#include "rf_kernels.h"
+#include "rfsa.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+rf_status_t fail(rf_status_t code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+rf_status_t ok() {
+  g_last_error.clear();
+  return RF_OK;
+}
+
+rf_status_t cuda_fail(cudaError_t e, const char* what) {
+  return fail(RF_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct Dims {
+  int B, S, N, D;
+};
+
+rf_status_t check_common(rf_layout_t layout, int B, int S, int N, int D) {
+  if (layout != RF_BSND && layout != RF_BNSD) return fail(RF_ERR_LAYOUT, "input layout must be BSND (0) or BNSD (1)");
+  if (B <= 0 || S <= 0 || N <= 0) return fail(RF_ERR_ARG, "B, S and N must be positive");
+  if (B > 65535 || (int64_t)B * N > 65535) return fail(RF_ERR_UNSUPPORTED, "B * N above 65535");
+  if (D != RF_HEAD_DIM) return fail(RF_ERR_UNSUPPORTED, "head dim must be 128 (got %d)", D);
+  return RF_OK;
+}
+
+rf_status_t check_ws(void* ws, size_t ws_bytes, const rf_ws_layout_t& lay) {
+  if (!ws) return fail(RF_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(RF_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < lay.total)
+    return fail(RF_ERR_WORKSPACE, "workspace has %zu bytes, needs %zu", ws_bytes, lay.total);
+  return RF_OK;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+float resolve_scale(float scale, int D) { return (scale > 0.f && std::isfinite(scale)) ? scale : 1.0f / std::sqrt((float)D); }
+
+// Library-owned workspace, one per device, grown on demand.
+struct WsCache {
+  std::mutex mu;
+  void* ptr[64] = {};
+  size_t bytes[64] = {};
+};
+WsCache g_ws, g_io;
+
+rf_status_t cached_buffer(WsCache& c, size_t need, void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(RF_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(c.mu);
+  if (c.bytes[dev] < need) {
+    if (c.ptr[dev]) {
+      e = cudaFree(c.ptr[dev]);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFree (workspace growth)");
+      c.ptr[dev] = nullptr;
+      c.bytes[dev] = 0;
+    }
+    e = cudaMalloc(&c.ptr[dev], need);
+    if (e != cudaSuccess) {
+      c.ptr[dev] = nullptr;
+      return cuda_fail(e, "cudaMalloc (workspace)");
+    }
+    c.bytes[dev] = need;
+  }
+  *out = c.ptr[dev];
+  return RF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rf_status_t rf_plan(int S, int txt_len, int T, int H, int W, int block_size, float sparsity, rf_plan_t* g) {
+  if (!g) return fail(RF_ERR_ARG, "plan pointer is NULL");
+  if (block_size != RF_BLOCK) return fail(RF_ERR_UNSUPPORTED, "block_size must be 128 (got %d)", block_size);
+  if (!(sparsity >= 0.f && sparsity <= 1.f)) return fail(RF_ERR_ARG, "sparsity must be finite and in [0, 1]");
+  if (S <= 0 || txt_len < 0 || T < 0 || H < 0 || W < 0) return fail(RF_ERR_ARG, "negative or empty size");
+  if (txt_len > S) return fail(RF_ERR_ARG, "txt_len %d exceeds S %d", txt_len, S);
+  const int64_t video = (int64_t)T * H * W;
+  if (video != 0 && (int64_t)S != txt_len + video)
+    return fail(RF_ERR_ARG, "S (%d) must equal txt_len + t*h*w (%lld)", S, (long long)(txt_len + video));
+  rf_plan_t p{};
+  p.S = S;
+  p.txt_len = txt_len;
+  p.T = T;
+  p.H = H;
+  p.W = W;
+  p.Ha = 8 * (H / 8);
+  p.Wa = 8 * (W / 8);
+  int nb = 0;
+  if (video != 0) {
+    const int64_t aligned = (int64_t)T * p.Ha * p.Wa;
+    nb = (int)(aligned / RF_BLOCK);
+    p.n_tail = (int)(aligned - (int64_t)nb * RF_BLOCK);
+    p.n_promoted = (int)(video - aligned);
+  }
+  if (video == 0 || nb < 32) {
+    p.dense = 1;
+    p.P = S;
+    p.nb = 0;
+  } else {
+    if (nb > RF_MAX_BLOCKS) return fail(RF_ERR_UNSUPPORTED, "%d sparse blocks exceed the limit %d", nb, RF_MAX_BLOCKS);
+    p.dense = 0;
+    p.nb = nb;
+    p.P = txt_len + p.n_promoted + p.n_tail;
+    p.ff = std::min(nb, (p.Ha * p.Wa + RF_BLOCK - 1) / RF_BLOCK);
+    const int drop = (int)std::floor((double)sparsity * nb + 1e-6);
+    p.k = std::max(0, std::min(nb, nb - drop));
+  }
+  p.P_pad = (p.P + RF_BLOCK - 1) / RF_BLOCK * RF_BLOCK;
+  if ((int64_t)p.P_pad + (int64_t)RF_BLOCK * p.nb > (int64_t)0x7FFFFF00)
+    return fail(RF_ERR_UNSUPPORTED, "sequence too long");
+  p.S_int = p.P_pad + RF_BLOCK * p.nb;
+  p.n_tiles = p.S_int / RF_BLOCK;
+  p.mask_words = (p.nb + 31) / 32;
+  *g = p;
+  return ok();
+}
+
+rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* g, rf_ws_layout_t* lay) {
+  if (!g || !lay) return fail(RF_ERR_ARG, "NULL plan or layout");
+  if (B <= 0 || N <= 0) return fail(RF_ERR_ARG, "B and N must be positive");
+  if (D != RF_HEAD_DIM) return fail(RF_ERR_UNSUPPORTED, "head dim must be 128 (got %d)", D);
+  const size_t heads = (size_t)B * N;
+  const size_t tensor = heads * g->S_int * RF_HEAD_DIM * 2;
+  const size_t pooled = heads * g->nb * RF_HEAD_DIM * 4;
+  const size_t rows = heads * g->nb;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at_off = off;
+    off = align256(off + bytes);
+    return at_off;
+  };
+  rf_ws_layout_t L{};
+  L.q_int = take(tensor);
+  L.k_int = take(tensor);
+  L.v_int = take(tensor);
+  L.pooled_q = take(pooled);
+  L.pooled_k = take(pooled);
+  L.mask = take(rows * g->mask_words * 4);
+  L.kept = take(rows * 4);
+  L.margin = take(rows * 4);
+  L.counter = take(4);
+  L.status = take(4);
+  L.total = off;
+  *lay = L;
+  return ok();
+}
+
+size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int T, int H, int W) {
+  rf_plan_t g;
+  rf_ws_layout_t L;
+  if (rf_plan(S, txt_len, T, H, W, RF_BLOCK, 0.f, &g) != RF_OK) return 0;
+  if (rf_workspace_layout(B, N, D, &g, &L) != RF_OK) return 0;
+  return L.total;
+}
+
+rf_status_t rf_prepare(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N, int D,
+                       int txt_len, int T, int H, int W, int block_size, float sparsity, void* ws, size_t ws_bytes,
+                       void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if (!q || !k || !v) return fail(RF_ERR_ARG, "q, k and v must be device pointers");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_ws_layout_t L;
+  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = rf::launch_permute_pool(q, k, v, layout, B, S, N, g, at<void>(ws, L.q_int), at<void>(ws, L.k_int),
+                                          at<void>(ws, L.v_int), at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k),
+                                          s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
+  e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, at<uint32_t>(ws, L.mask),
+                      at<int>(ws, L.kept), at<float>(ws, L.margin), s);
+  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
+  return ok();
+}
+
+rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W,
+                      int block_size, float sparsity, float scale, void* out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if (!out) return fail(RF_ERR_ARG, "out must be a device pointer");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_ws_layout_t L;
+  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
+                                       at<uint32_t>(ws, L.mask), layout, B, S, N, g, resolve_scale(scale, D), out,
+                                       at<int>(ws, L.counter), at<int>(ws, L.status),
+                                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return ok();
+}
+
+rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
+                                   int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
+                                   float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
+  if (out && (out == q || out == k || out == v)) return fail(RF_ERR_ARG, "out must not alias q, k or v");
+  rf_status_t st = rf_prepare(q, k, v, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, ws, ws_bytes,
+                              stream);
+  if (st != RF_OK) return st;
+  return rf_attend(layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws, ws_bytes, stream);
+}
+
+rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
+                                int D, int txt_len, int T, int H, int W, int block_size, float sparsity, float scale,
+                                void* out, void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_ws_layout_t L;
+  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
+  if (!q || !k || !v || !out) return fail(RF_ERR_ARG, "q, k, v and out must be device pointers");
+  void* ws = nullptr;
+  if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
+  return rf_sparse_attention_ws(q, k, v, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws,
+                                L.total, stream);
+}
+
+rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H,
+                         int W, void* out, void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if (!o_int || !out) return fail(RF_ERR_ARG, "o_int and out must be device pointers");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, RF_BLOCK, 0.f, &g)) != RF_OK) return st;
+  cudaError_t e = rf::launch_unpermute(o_int, layout, B, S, N, g, out, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "unpermute launch");
+  return ok();
+}
+
+rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void* vh, rf_layout_t layout, int B, int S,
+                                     int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
+                                     float scale, void* out_h, void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if (!qh || !kh || !vh || !out_h) return fail(RF_ERR_ARG, "host buffers must not be NULL");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_ws_layout_t L;
+  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
+  const size_t tensor = (size_t)B * S * N * D * 2;
+  const size_t t_al = align256(tensor);
+  void* io = nullptr;
+  void* ws = nullptr;
+  if ((st = cached_buffer(g_io, 4 * t_al, &io)) != RF_OK) return st;
+  if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
+  char* d = static_cast<char*>(io);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  const void* srcs[3] = {qh, kh, vh};
+  for (int i = 0; i < 3; ++i) {
+    e = cudaMemcpyAsync(d + i * t_al, srcs[i], tensor, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+  }
+  st = rf_sparse_attention_ws(d, d + t_al, d + 2 * t_al, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity,
+                              scale, d + 3 * t_al, ws, L.total, stream);
+  if (st != RF_OK) return st;
+  e = cudaMemcpyAsync(out_h, d + 3 * t_al, tensor, cudaMemcpyDeviceToHost, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
+  e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  return ok();
+}
+
+rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const rf_plan_t* g, int* status,
+                           void* stream) {
+  if (!status) return fail(RF_ERR_ARG, "status pointer is NULL");
+  rf_ws_layout_t L;
+  rf_status_t st = rf_workspace_layout(B, N, D, g, &L);
+  if (st != RF_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, at<int>(ws, L.status), sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
+  *status = h;
+  return ok();
+}
+
+const char* rf_last_error_string(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// Launchers of the library's kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "rfsa.h"
+
+namespace rf {
+
+// K1: token reorder into [B, N, S_int, 128] bf16 for q, k, v (pad rows
+// zeroed), with the fp32 block means of q and k for the sparse blocks.
+cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int layout, int B, int S, int N,
+                                const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
+                                float* pooled_k, cudaStream_t stream);
+
+// K4: inverse reorder of an internal-order tensor into the caller's layout.
+cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N, const rf_plan_t& g, void* out,
+                             cudaStream_t stream);
+
+// K2: block scores + top-k + forced first-frame blocks -> bit mask rows,
+// kept counts and k-th-score margins.
+cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g, uint32_t* mask,
+                        int* kept, float* margin, cudaStream_t stream);
+
+// K3: block-sparse flash attention over the internal layout, output written
+// straight to the caller's layout (inverse reorder fused in the epilogue).
+cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
+                             int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
+                             int* counter, int* status, cudaStream_t stream);
+
+}  // namespace rf

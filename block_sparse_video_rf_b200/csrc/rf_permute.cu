@@ -1,0 +1,131 @@
+// Token reorder with block pooling fused in (K1), and the inverse reorder
+// (K4).  Both are HBM-bound row gathers/scatters of 256-byte rows.
+//
+// lite_boost.ops.sparse_attention, rf_v2 pipeline: token reorder, then block
+// pooling; inverse reorder at the end.  vllm-omni "RainFusion Attention":
+// 128-token key blocks are pooled (intro); the reorder groups video tokens
+// into 8x8 tiles and promotes the non-aligned rest ("Geometry handling").
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rf_geometry.h"
+#include "rf_kernels.h"
+
+namespace rf {
+
+namespace {
+
+constexpr int kPermThreads = 256;   // 16 rows x 16 chunks of 16 bytes per pass
+constexpr int kRowsPerPass = kPermThreads / 16;
+constexpr int kPasses = RF_BLOCK / kRowsPerPass;
+
+__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& u) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc[2 * i] += __uint_as_float(w[i] << 16);
+    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// One CTA = one 128-row internal tile of one (b, head), for q, k and v.
+// Sparse tiles also write the fp32 block means of q and k.  The column sums
+// run in a fixed order (per thread over its 8 rows, then over the 16 row
+// groups), so results are deterministic.
+__global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
+    int layout, int B, int S, int N, rf_plan_t g, __nv_bfloat16* __restrict__ q_int, __nv_bfloat16* __restrict__ k_int,
+    __nv_bfloat16* __restrict__ v_int, float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+  __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
+  const int tile = blockIdx.x;
+  const int bn = blockIdx.y;
+  const int b = bn / N, n = bn - b * N;
+  const int chunk = threadIdx.x & 15;     // 16-byte column chunk
+  const int rsub = threadIdx.x >> 4;      // row within the pass
+  const bool sparse = (tile * RF_BLOCK >= g.P_pad) && !g.dense;
+
+  int64_t src_off[kPasses];
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const int r = tile * RF_BLOCK + p * kRowsPerPass + rsub;
+    const int s = rf_src_of_row(g, r);
+    src_off[p] = s < 0 ? -1 : rf_token_offset(layout, B, S, N, b, n, s) + chunk * 8;
+  }
+  const int64_t dst_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM + chunk * 8;
+
+  const __nv_bfloat16* srcs[3] = {q, k, v};
+  __nv_bfloat16* dsts[3] = {q_int, k_int, v_int};
+#pragma unroll
+  for (int t = 0; t < 3; ++t) {
+    uint4 buf[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      buf[p] = src_off[p] < 0 ? make_uint4(0, 0, 0, 0)
+                              : __ldcs(reinterpret_cast<const uint4*>(srcs[t] + src_off[p]));
+    }
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      *reinterpret_cast<uint4*>(dsts[t] + dst_base + (int64_t)(p * kRowsPerPass + rsub) * RF_HEAD_DIM) = buf[p];
+    }
+    if (t < 2 && sparse) {
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p) acc_bf16x8(acc, buf[p]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) red[t][rsub][chunk * 8 + i] = acc[i];
+    }
+  }
+  if (!sparse) return;
+  __syncthreads();
+  // 256 threads: 2 tensors x 128 columns.
+  const int t = threadIdx.x >> 7, c = threadIdx.x & 127;
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowsPerPass; ++i) s += red[t][i][c];
+  const int blk = tile - g.P_pad / RF_BLOCK;
+  float* dst = (t == 0 ? pooled_q : pooled_k) + ((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c;
+  *dst = s * (1.0f / RF_BLOCK);
+}
+
+__global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __nv_bfloat16* __restrict__ o_int, int layout,
+                                                                 int B, int S, int N, rf_plan_t g,
+                                                                 __nv_bfloat16* __restrict__ out) {
+  const int tile = blockIdx.x;
+  const int bn = blockIdx.y;
+  const int b = bn / N, n = bn - b * N;
+  const int chunk = threadIdx.x & 15;
+  const int rsub = threadIdx.x >> 4;
+  const int64_t src_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM + chunk * 8;
+  uint4 buf[kPasses];
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p)
+    buf[p] = __ldcs(reinterpret_cast<const uint4*>(o_int + src_base + (int64_t)(p * kRowsPerPass + rsub) * RF_HEAD_DIM));
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) {
+    const int s = rf_src_of_row(g, tile * RF_BLOCK + p * kRowsPerPass + rsub);
+    if (s >= 0) *reinterpret_cast<uint4*>(out + rf_token_offset(layout, B, S, N, b, n, s) + chunk * 8) = buf[p];
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int layout, int B, int S, int N,
+                                const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
+                                float* pooled_k, cudaStream_t stream) {
+  dim3 grid(g.n_tiles, B * N);
+  permute_pool_kernel<<<grid, kPermThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+      static_cast<const __nv_bfloat16*>(v), layout, B, S, N, g, static_cast<__nv_bfloat16*>(q_int),
+      static_cast<__nv_bfloat16*>(k_int), static_cast<__nv_bfloat16*>(v_int), pooled_q, pooled_k);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N, const rf_plan_t& g, void* out,
+                             cudaStream_t stream) {
+  dim3 grid(g.n_tiles, B * N);
+  unpermute_kernel<<<grid, kPermThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(o_int), layout, B, S, N, g,
+                                                      static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace rf

@@ -1,0 +1,243 @@
+"""ctypes binding of ``librfsa.so`` (see include/rfsa.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  Importing this module fails loudly when the library has not been
+built (``python -m block_sparse_video_rf_b200.build``); there is no fallback.
+Tensors are torch CUDA tensors; the stream defaults to torch's current
+stream on the tensor's device.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "librfsa.so")
+
+RF_BSND, RF_BNSD = 0, 1
+LAYOUTS = {"BSND": RF_BSND, "BNSD": RF_BNSD}
+STATUS = {0: "RF_OK", 1: "RF_ERR_LAYOUT", 2: "RF_ERR_ARG", 3: "RF_ERR_UNSUPPORTED", 4: "RF_ERR_CUDA",
+          5: "RF_ERR_WORKSPACE", 6: "RF_ERR_TIMEOUT"}
+
+PLAN_FIELDS = ["S", "txt_len", "T", "H", "W", "Ha", "Wa", "n_promoted", "n_tail", "P", "P_pad", "nb", "ff", "k",
+               "dense", "S_int", "n_tiles", "mask_words"]
+WS_FIELDS = ["q_int", "k_int", "v_int", "pooled_q", "pooled_k", "mask", "kept", "margin", "counter", "status",
+             "total"]
+
+# Every symbol include/rfsa.h declares.
+EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
+           "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
+           "rf_last_error_string"]
+
+
+class RfPlan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in PLAN_FIELDS]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n in PLAN_FIELDS}
+
+
+class RfWsLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_size_t) for n in WS_FIELDS]
+
+
+class RfError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"{STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m block_sparse_video_rf_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    I, F, P, Z = ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t
+    geo = [I, I, I, I, I, I, I, I]  # layout, B, S, N, D, txt_len, t, h ... (w appended below)
+    sig = {
+        "rf_plan": (I, [I, I, I, I, I, I, F, ctypes.POINTER(RfPlan)]),
+        "rf_workspace_layout": (I, [I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfWsLayout)]),
+        "rf_workspace_size": (Z, [I, I, I, I, I, I, I, I]),
+        "rf_sparse_attention": (I, [P, P, P] + geo + [I, I, F, F, P, P]),
+        "rf_sparse_attention_ws": (I, [P, P, P] + geo + [I, I, F, F, P, P, Z, P]),
+        "rf_prepare": (I, [P, P, P] + geo + [I, I, F, P, Z, P]),
+        "rf_attend": (I, geo + [I, I, F, F, P, P, Z, P]),
+        "rf_unpermute": (I, [P] + geo + [I, P, P]),
+        "rf_sparse_attention_host": (I, [P, P, P] + geo + [I, I, F, F, P, P]),
+        "rf_read_status": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(I), P]),
+        "rf_last_error_string": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+LIB = _load()
+
+
+def _check(code: int):
+    if code != 0:
+        raise RfError(code, LIB.rf_last_error_string().decode())
+
+
+def _dims(x, layout: str):
+    if layout == "BSND":
+        B, S, N, D = x.shape
+    elif layout == "BNSD":
+        B, N, S, D = x.shape
+    else:
+        raise RfError(1, "input layout must be BSND or BNSD")
+    return B, S, N, D
+
+
+def _stream(x, stream):
+    if stream is not None:
+        return ctypes.c_void_p(stream)
+    import torch
+    return ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream)
+
+
+def _ptr(x):
+    return ctypes.c_void_p(x.data_ptr()) if x is not None else None
+
+
+def _scale(scale):
+    return float("nan") if scale is None else float(scale)
+
+
+def rf_plan(S: int, txt_len: int, latent, sparsity: float, block_size: int = 128) -> RfPlan:
+    p = RfPlan()
+    _check(LIB.rf_plan(S, txt_len, *latent, block_size, float(sparsity), ctypes.byref(p)))
+    return p
+
+
+def rf_workspace_layout(B: int, N: int, D: int, plan: RfPlan) -> RfWsLayout:
+    lay = RfWsLayout()
+    _check(LIB.rf_workspace_layout(B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
+    return lay
+
+
+def rf_workspace_size(B, S, N, D, txt_len, latent) -> int:
+    return int(LIB.rf_workspace_size(B, S, N, D, txt_len, *latent))
+
+
+def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: float, scale=None, out=None,
+                        block_size: int = 128, stream=None):
+    """The whole rf_v2 call on device tensors; returns ``out`` (shape and layout of q)."""
+    import torch
+    B, S, N, D = _dims(q, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(LIB.rf_sparse_attention(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
+                                   *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
+                                   _stream(q, stream)))
+    return out
+
+
+def rf_sparse_attention_ws(q, k, v, layout, txt_len, latent, sparsity, workspace, scale=None, out=None,
+                           block_size=128, stream=None):
+    import torch
+    B, S, N, D = _dims(q, layout)
+    if out is None:
+        out = torch.empty_like(q)
+    _check(LIB.rf_sparse_attention_ws(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
+                                      *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(q, stream)))
+    return out
+
+
+def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size=128, stream=None):
+    B, S, N, D = _dims(q, layout)
+    _check(LIB.rf_prepare(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
+                          block_size, float(sparsity), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                          _stream(q, stream)))
+
+
+def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, block_size=128, stream=None):
+    B, S, N, D = _dims(out, layout)
+    _check(LIB.rf_attend(LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent, block_size, float(sparsity),
+                         _scale(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                         _stream(out, stream)))
+    return out
+
+
+def rf_unpermute(o_int, out, layout, txt_len, latent, stream=None):
+    B, S, N, D = _dims(out, layout)
+    _check(LIB.rf_unpermute(_ptr(o_int), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent, _ptr(out),
+                            _stream(out, stream)))
+    return out
+
+
+def rf_sparse_attention_host(q, k, v, layout, txt_len, latent, sparsity, out, scale=None, block_size=128,
+                             stream=None):
+    """q, k, v, out: CPU (ideally pinned) bf16 tensors; copies happen inside the library."""
+    import torch
+    B, S, N, D = _dims(q, layout)
+    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
+    _check(LIB.rf_sparse_attention_host(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
+                                        *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
+                                        ctypes.c_void_p(st)))
+    return out
+
+
+def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(LIB.rf_read_status(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
+                              ctypes.byref(plan), ctypes.byref(st), _stream(workspace, stream)))
+    return st.value
+
+
+def workspace_views(workspace, B, N, plan):
+    """Typed torch views of the workspace regions (for inspection and tests)."""
+    import torch
+    lay = rf_workspace_layout(B, N, 128, plan)
+    raw = workspace.view(torch.uint8)
+    heads = B * N
+
+    def view(off, count, dtype, shape):
+        nbytes = count * torch.empty((), dtype=dtype).element_size()
+        return raw[off:off + nbytes].view(dtype).view(shape)
+
+    nb, words = plan.nb, plan.mask_words
+    return {
+        "q_int": view(lay.q_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
+        "k_int": view(lay.k_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
+        "v_int": view(lay.v_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
+        "pooled_q": view(lay.pooled_q, heads * nb * 128, torch.float32, (B, N, nb, 128)),
+        "pooled_k": view(lay.pooled_k, heads * nb * 128, torch.float32, (B, N, nb, 128)),
+        "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),
+        "kept": view(lay.kept, heads * nb, torch.int32, (B, N, nb)),
+        "margin": view(lay.margin, heads * nb, torch.float32, (B, N, nb)),
+    }
+
+
+def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda"):
+    import torch
+    n = rf_workspace_size(B, S, N, D, txt_len, latent)
+    if n == 0:
+        raise RfError(2, "bad arguments for the workspace size")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def kept_block_flops(plan: RfPlan, kept, B: int, N: int, D: int = 128) -> float:
+    """Algorithmic FLOPs of one call: 4 * D * sum over query rows of |key set|.
+
+    Dense rows (prefix, first-frame blocks, or everything in the dense
+    fallback) read all S keys; a sparse block's 128 rows read the P prefix
+    keys plus 128 per kept block.  ``kept`` is the per-row kept-count tensor
+    (B, N, nb) from the workspace.
+    """
+    S = plan.S
+    if plan.dense:
+        return 4.0 * D * B * N * S * S
+    dense_rows = plan.P + 128 * plan.ff
+    sparse_keys = kept[..., plan.ff:].double().sum().item() * 128.0 + (plan.nb - plan.ff) * B * N * plan.P
+    return 4.0 * D * (B * N * dense_rows * S + 128.0 * sparse_keys)
+
+
+def default_scale(D: int = 128) -> float:
+    return 1.0 / math.sqrt(D)

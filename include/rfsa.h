@@ -1,0 +1,155 @@
+/*
+ * rfsa.h -- C ABI of the RainFusion rf_v2 block-sparse video attention
+ * library for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the rf_v2 mode of MindSpore Lite's
+ * "lite_boost.ops.sparse_attention" (pipeline: token reorder -> block
+ * pooling -> top-k sparse mask -> rain_fusion_attention -> inverse reorder),
+ * with the geometry and dense-fallback rules of the vllm-omni user guide
+ * page "RainFusion Attention" (intro; "Configuration"; "Geometry handling").
+ *
+ * Conventions for every entry point:
+ *  - q, k, v, out: DEVICE pointers to bf16, caller-owned, contiguous, in the
+ *    layout given (RF_BSND = [B, S, N, D], RF_BNSD = [B, N, S, D]); out has
+ *    the shape and layout of q and must not alias q, k or v.
+ *  - D and block_size must be 128.
+ *  - S = txt_len + latent_t * latent_h * latent_w.  latent (0, 0, 0) means
+ *    "no video geometry": the call is dense softmax attention over S.
+ *  - sparsity must be finite and in [0, 1]; it is the nominal fraction of
+ *    key blocks dropped per query block (0 = dense).
+ *  - scale <= 0 or NaN selects head_dim ** -0.5.
+ *  - Argument errors are returned before anything is enqueued.  Work is
+ *    enqueued on `stream` (NULL = legacy default stream) and is asynchronous;
+ *    launch failures return RF_ERR_CUDA.  Nothing here synchronises the
+ *    device except rf_read_status and rf_sparse_attention_host.
+ *  - A device-side wait that runs past its time limit makes the kernel
+ *    record RF_ERR_TIMEOUT in the workspace status word and return early;
+ *    rf_read_status reports it.
+ *  - The library never frees caller memory.
+ *  - On error, rf_last_error_string() (thread-local) says why.
+ */
+#ifndef RFSA_H
+#define RFSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { RF_BSND = 0, RF_BNSD = 1 } rf_layout_t;
+
+typedef enum {
+  RF_OK = 0,
+  RF_ERR_LAYOUT = 1,      /* layout not BSND/BNSD (the page's ValueError on input_layout) */
+  RF_ERR_ARG = 2,         /* bad sizes, sparsity outside [0, 1], S != txt_len + t*h*w, NULL pointer */
+  RF_ERR_UNSUPPORTED = 3, /* D != 128, block_size != 128, or more sparse blocks than RF_MAX_BLOCKS */
+  RF_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  RF_ERR_WORKSPACE = 5,   /* workspace too small or misaligned */
+  RF_ERR_TIMEOUT = 6      /* a device-side wait ran past its limit (read via rf_read_status) */
+} rf_status_t;
+
+#define RF_HEAD_DIM 128
+#define RF_BLOCK 128
+#define RF_MAX_BLOCKS 4096
+
+/* Geometry of one clip, shared by every (batch, head).
+ * Internal row order per (b, head): [prefix: text, promoted video tokens in
+ * natural (t, h, w) order, aligned tokens past the last whole block]
+ * [zero pad to a multiple of 128] [nb sparse blocks of 128 rows, each two
+ * 8x8 tiles: frames in order, tiles row-major, raster inside a tile]. */
+typedef struct {
+  int S, txt_len, T, H, W;
+  int Ha, Wa;        /* 8 * floor(H / 8), 8 * floor(W / 8) */
+  int n_promoted;    /* video tokens outside the Ha x Wa grid */
+  int n_tail;        /* aligned tokens past the last whole 128-block */
+  int P;             /* dense prefix rows (S when dense) */
+  int P_pad;         /* P rounded up to 128 */
+  int nb;            /* sparse 128-blocks (0 when dense) */
+  int ff;            /* first-frame blocks: ceil(Ha * Wa / 128), at most nb */
+  int k;             /* top-k kept per sparse query block: nb - floor(sparsity * nb + 1e-6) */
+  int dense;         /* 1: every row attends to every key (no geometry, or nb < 32) */
+  int S_int;         /* internal rows per (b, head) = P_pad + 128 * nb */
+  int n_tiles;       /* S_int / 128 */
+  int mask_words;    /* 32-bit words per mask row = ceil(nb / 32) */
+} rf_plan_t;
+
+/* Byte offsets of the regions of a workspace (all 256-byte aligned).
+ * q_int/k_int/v_int: bf16 [B, N, S_int, 128]; pooled_q/pooled_k: fp32
+ * [B, N, nb, 128] (block means); mask: uint32 [B, N, nb, mask_words], bit j
+ * of row i set when query block i reads key block j; kept: int32 [B, N, nb]
+ * (bits set per row); margin: fp32 [B, N, nb] (relative gap between the
+ * k-th and (k+1)-th block score of the row, +inf when not defined);
+ * counter: int32 work counter; status: int32 device status word. */
+typedef struct {
+  size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status, total;
+} rf_ws_layout_t;
+
+/* Host-only: validate a geometry and fill *plan.  No CUDA call. */
+rf_status_t rf_plan(int S, int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
+                    rf_plan_t* plan);
+
+/* Host-only: workspace regions for B x N heads of head dim D under `plan`. */
+rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* plan, rf_ws_layout_t* layout);
+
+/* Host-only: bytes of workspace rf_sparse_attention_ws needs (0 on bad arguments). */
+size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int latent_t, int latent_h, int latent_w);
+
+/* The whole rf_v2 call, with a workspace cached by the library per device
+ * (grown with cudaMalloc on first use of a larger shape; never shrunk). */
+rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
+                                int D, int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
+                                float sparsity, float scale, void* out, void* stream);
+
+/* The whole call with a caller-owned device workspace of ws_bytes
+ * (>= rf_workspace_size, 256-byte aligned).  Calls that share a workspace
+ * must be ordered on one stream. */
+rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
+                                   int N, int D, int txt_len, int latent_t, int latent_h, int latent_w,
+                                   int block_size, float sparsity, float scale, void* out, void* workspace,
+                                   size_t ws_bytes, void* stream);
+
+/* Stage 1 (token reorder + block pooling, then block scores + top-k mask):
+ * fills q_int/k_int/v_int, pooled_q/pooled_k, mask, kept and margin of the
+ * workspace. */
+rf_status_t rf_prepare(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N, int D,
+                       int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/* Stage 2 (rain_fusion_attention + inverse reorder): attention of every
+ * query over its key set as given by the workspace mask, written to out in
+ * the caller's token order and layout.  The mask region may be overwritten
+ * between the stages (e.g. to run under another mask). */
+rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
+                      int latent_w, int block_size, float sparsity, float scale, void* out, void* workspace,
+                      size_t ws_bytes, void* stream);
+
+/* Inverse reorder alone: o_int bf16 [B, N, S_int, 128] (internal order) ->
+ * out in the caller's layout.  Pad rows are skipped. */
+rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len,
+                         int latent_t, int latent_h, int latent_w, void* out, void* stream);
+
+/* End-to-end through HOST buffers (bf16, caller layout): copies q, k, v to
+ * the device, runs the call with the cached workspace, copies the result
+ * back to out_host and synchronises `stream`.  Host buffers should be pinned
+ * for full copy bandwidth. */
+rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, const void* v_host, rf_layout_t layout,
+                                     int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
+                                     int latent_w, int block_size, float sparsity, float scale, void* out_host,
+                                     void* stream);
+
+/* Synchronises `stream`, reads the workspace status word into *status
+ * (0 = fine, otherwise an rf_status_t code recorded by a kernel) and clears
+ * it.  Returns RF_OK or RF_ERR_CUDA. */
+rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
+                           int* status, void* stream);
+
+/* Thread-local text of the last error returned on this thread. */
+const char* rf_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RFSA_H */
