@@ -1,0 +1,337 @@
+"""Benchmark of the rf_v2 block-sparse attention call on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload minimax] [--impl reference]
+
+One step = one full call (token reorder + pooling, block scores + top-k mask,
+block-sparse attention with the inverse reorder fused) on one batch of seeded
+synthetic bf16 Q/K/V resident in HBM.  The metric is the effective
+throughput over the kept blocks: FLOPs = 4 * D * sum over query rows of the
+number of keys the row attends to (dense prefix and first-frame rows count
+all S keys), divided by the device time of the step.  Under torchrun each rank
+runs its own replica (the call shards by independent problems; no collective
+on the data path), so the aggregate is the sum over ranks divided by the
+slowest rank's time.
+
+``--impl reference`` times the plain CPU oracle on the host cores instead, on
+a bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "rf_v2 sparse-attn ms/call & effective TFLOPS (kept blocks) at MiniMax-H3 shape"
+UNIT = "TFLOP/s"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _k3_traffic(heads: int):
+    """DRAM bytes per attention launch from the committed ncu summary, scaled to
+    ``heads``; None when the kernel source changed since the capture."""
+    import hashlib
+    src = os.path.join(ROOT, "block_sparse_video_rf_b200", "csrc", "rf_attn.cu")
+    path = os.path.join(ROOT, "profiles", "k3_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == "attn_kernel" and parts[1] == digest:
+            return int(parts[2]) * heads / 56.0
+    return None
+
+
+def _describe(w) -> str:
+    t, h, wd = w.latent
+    return (f"{w.name}: B={w.B}, {w.N} heads, D={w.D}, txt_len={w.txt_len}, latent ({t},{h},{wd}) -> S={w.S}, "
+            f"sparsity {w.sparsity}, {w.layout}, bf16 synthetic ({w.kind})")
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.device_index = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- multi-rank aggregation
+def reduce_max(values, dist=None, device="cpu"):
+    """Element-wise max over ranks (the slowest rank decides every time)."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate(flops_per_rank_step: float, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput in TFLOP/s: every rank runs the same replica."""
+    return world * flops_per_rank_step / (ms_per_step_max * 1e-3) / 1e12
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(q, k, v, w, budget_s: float = 15.0, heads_total=None):
+    """Times the CPU oracle on head 0: its own mask, then attention for evenly
+    spaced query tiles until about ``budget_s`` of CPU work.  Returns
+    (TFLOP/s, threads, description)."""
+    import oracle
+    from threadpoolctl import threadpool_info
+    qh = q[0, :, 0].float().cpu().numpy() if w.layout == "BSND" else q[0, 0].float().cpu().numpy()
+    kh = k[0, :, 0].float().cpu().numpy() if w.layout == "BSND" else k[0, 0].float().cpu().numpy()
+    vh = v[0, :, 0].float().cpu().numpy() if w.layout == "BSND" else v[0, 0].float().cpu().numpy()
+    t0 = time.perf_counter()
+    g = oracle.geometry(w.S, w.txt_len, *w.latent)
+    mask, _ = oracle.build_mask(qh[None, None], kh[None, None], g, float(np.float32(w.sparsity)))
+    mask = mask[0, 0]
+    # query tiles in the oracle's own terms: prefix rows in chunks of 128, then sparse blocks
+    tiles = [("prefix", g.prefix[i:i + 128]) for i in range(0, len(g.prefix), 128)]
+    tiles += [("block", g.blocks[i]) for i in range(g.nb)] if not g.dense else []
+    order = list(range(0, len(tiles), 7)) + [i for i in range(len(tiles)) if i % 7]
+    flops, done = 0.0, 0
+    scale = w.D ** -0.5
+    for idx in order:
+        kind, rows = tiles[idx]
+        out = oracle.attention_rows(qh, kh, vh, g, None if g.dense else mask, scale, rows=rows)
+        blk = None if kind == "prefix" else idx - (len(tiles) - g.nb)
+        nkeys = len(oracle.key_set(g, mask, blk)) if not g.dense else g.S
+        flops += 4.0 * w.D * len(rows) * nkeys
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    desc = (f"head 0 of {heads_total or w.N}: mask of all {g.nb} blocks + attention of {done} of {len(tiles)} query tiles "
+            f"(every 7th first), {flops / 1e12:.3f} TFLOP in {dt:.1f} s")
+    return flops / dt / 1e12, threads, desc
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_sparse_video_rf_b200 import synth
+    q, k, v = synth.make_inputs(synth.workload(w.name, N=1, seed=w.seed), device="cpu")
+    vals, walls = [], []
+    desc = threads = None
+    w1 = synth.workload(w.name, N=1, **({} if args.sparsity is None else {"sparsity": args.sparsity}))
+    for i in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        val, threads, desc = oracle_sample(q, k, v, w1, budget_s=args.ref_budget, heads_total=w.N)
+        if i >= args.warmup:
+            vals.append(val)
+            walls.append(time.perf_counter() - t0)
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(walls),
+        "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": _describe(w), "sample": "one head per step, bounded CPU time"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- CUDA arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="minimax")
+    ap.add_argument("--sparsity", type=float, default=None)
+    ap.add_argument("--heads", type=int, default=None, help="override the head count (small profiling cases)")
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=6.0, help="seconds of oracle work per reference step")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    args = ap.parse_args()
+
+    from block_sparse_video_rf_b200 import synth
+    over = {} if args.sparsity is None else {"sparsity": args.sparsity}
+    if args.heads is not None:
+        over["N"] = args.heads
+    w = synth.workload(args.workload, **over)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    from block_sparse_video_rf_b200 import rfsa
+    dev = torch.device("cuda", local)
+    q, k, v = synth.make_inputs(w, device=dev)
+    out = torch.empty_like(q)
+    sp = np.float32(w.sparsity)
+    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent, device=dev)
+    plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, sp)
+    views = rfsa.workspace_views(ws, w.B, w.N, plan)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws)
+        if ev is not None:
+            ev[1].record(stream)
+        rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize(dev)
+    status = rfsa.rf_read_status(ws, w.B, w.N, w.D, plan)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after warm-up")
+    flops = rfsa.kept_block_flops(plan, views["kept"], w.B, w.N, w.D)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    k1k2 = [e[0].elapsed_time(e[1]) for e in evs]
+    k3 = [e[1].elapsed_time(e[2]) for e in evs]
+    status = rfsa.rf_read_status(ws, w.B, w.N, w.D, plan)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed steps")
+
+    # end to end through host buffers: H2D of q, k, v and D2H of the output inside the timed region
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else min(args.steps, 10)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    rfsa.rf_sparse_attention_host(qh, kh, vh, w.layout, w.txt_len, w.latent, sp, oh)   # warm the caches
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        rfsa.rf_sparse_attention_host(qh, kh, vh, w.layout, w.txt_len, w.latent, sp, oh)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / max(e2e_steps, 1)
+
+    # slowest rank decides
+    ms_total, e2e_ms, k3_ms = reduce_max([ms_total, e2e_ms, statistics.mean(k3)], dist, dev)
+    ms_step = ms_total / args.steps
+    value = aggregate(flops, world, ms_step)
+    e2e_value = aggregate(flops, world, e2e_ms)
+
+    if rank == 0:
+        peaks, src = _peaks()
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        k3_tflops = flops / (k3_ms * 1e-3) / 1e12
+        tensor_bytes = q.numel() * q.element_size()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": _describe(w), "l2": "inputs larger than L2 (no flush)",
+                       "kept_block_tflop_per_call": flops / 1e12, "k": plan.k, "nb": plan.nb, "ff": plan.ff,
+                       "P": plan.P, "ms_prepare": statistics.mean(k1k2), "ms_attention": k3_ms},
+            "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
+            "roofline": {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": k3_tflops / peak, "traffic": _k3_traffic(w.N),
+                         "peak_source": f"{src} bf16_tflops_sustained"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            val, threads, desc = oracle_sample(q, k, v, w)
+            line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
