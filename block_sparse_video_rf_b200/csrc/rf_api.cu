@@ -324,6 +324,27 @@ rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const
   return ok();
 }
 
+rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layout, int B, int S, int N, int D,
+                                  int txt_len, int T, int H, int W, int block_size, float sparsity, uint32_t* mask,
+                                  int32_t* kept, float* margin, void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if (!q || !k) return fail(RF_ERR_ARG, "q and k must be device pointers");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  if (g.nb == 0) return ok();
+  if (!mask || !kept || !margin) return fail(RF_ERR_ARG, "mask, kept and margin must be device pointers");
+  const size_t need = (size_t)B * N * g.nb * RF_HEAD_DIM * sizeof(float) * 2;
+  if (need > RF_NOALLOC_SCRATCH_BYTES)
+    return fail(RF_ERR_UNSUPPORTED,
+                "B*N*nb = %zu block rows need %zu bytes of pooled scratch, above the static %u-byte array",
+                (size_t)B * N * g.nb, need, (unsigned)RF_NOALLOC_SCRATCH_BYTES);
+  cudaError_t e = rf::launch_block_mask_noalloc(q, k, layout, B, S, N, g, mask, kept, margin,
+                                                static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "no-allocation mask launch");
+  return ok();
+}
+
 const char* rf_last_error_string(void) { return g_last_error.c_str(); }
 
 }  // extern "C"

@@ -29,4 +29,10 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
                              int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
                              int* counter, int* status, cudaStream_t stream);
 
+// Block mask with the pooled means in the library's static scratch array
+// (no device allocation); see rf_block_mask_noalloc.
+cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int layout, int B, int S, int N,
+                                      const rf_plan_t& g, uint32_t* mask, int* kept, float* margin,
+                                      cudaStream_t stream);
+
 }  // namespace rf

@@ -29,7 +29,7 @@ WS_FIELDS = ["q_int", "k_int", "v_int", "pooled_q", "pooled_k", "mask", "kept", 
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_last_error_string"]
+           "rf_block_mask_noalloc", "rf_last_error_string"]
 
 
 class RfPlan(ctypes.Structure):
@@ -66,6 +66,7 @@ def _load():
         "rf_unpermute": (I, [P] + geo + [I, P, P]),
         "rf_sparse_attention_host": (I, [P, P, P] + geo + [I, I, F, F, P, P]),
         "rf_read_status": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(I), P]),
+        "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_last_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -182,6 +183,15 @@ def rf_sparse_attention_host(q, k, v, layout, txt_len, latent, sparsity, out, sc
                                         *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
                                         ctypes.c_void_p(st)))
     return out
+
+
+def rf_block_mask_noalloc(q, k, layout, txt_len, latent, sparsity, mask, kept, margin, block_size=128,
+                          stream=None):
+    """Block mask into caller buffers, with no device allocation (see include/rfsa.h)."""
+    B, S, N, D = _dims(q, layout)
+    _check(LIB.rf_block_mask_noalloc(_ptr(q), _ptr(k), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
+                                     block_size, float(sparsity), _ptr(mask), _ptr(kept), _ptr(margin),
+                                     _stream(q, stream)))
 
 
 def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:

@@ -145,6 +145,38 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
 rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                            int* status, void* stream);
 
+/* Size of the library-owned static scratch array of rf_block_mask_noalloc,
+ * per device (32 MiB): enough for B * N * nb <= 32768 block rows of pooled Q and K
+ * (the 56-head MiniMax-H3 shape needs 26,040). */
+#define RF_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* Block mask without any device allocation.  The pages have no counterpart:
+ * this is a library convenience for callers that cannot allocate device
+ * memory themselves.  Examples are a plugin in a process whose device memory
+ * belongs entirely to one allocator that forbids side allocations, or a
+ * latency-critical loop that cannot afford the implicit synchronisation of
+ * cudaMalloc/cudaFree.
+ * It computes what rf_prepare puts in the mask, kept and margin regions
+ * (block pooling of q and k over the reordered sparse blocks, block scores,
+ * top-k plus the forced first-frame blocks) and writes them to the caller's
+ * device buffers: mask uint32 [B, N, nb, ceil(nb / 32)], kept int32
+ * [B, N, nb], margin fp32 [B, N, nb] (nb and the geometry as in rf_plan).
+ * Its only scratch, the fp32 block means of q and k, lives in a file-scope
+ * static device array of RF_NOALLOC_SCRATCH_BYTES that every device loading
+ * the library holds until the process exits.  It calls no cudaMalloc,
+ * cudaFree or allocating routine.
+ * - B * N * nb * 128 * 8 bytes above RF_NOALLOC_SCRATCH_BYTES returns
+ *   RF_ERR_UNSUPPORTED with a message; a dense plan (nb = 0) writes nothing.
+ * - The first call on a device looks up the device address of the array
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ * - All calls share the array: calls whose work overlaps on the GPU race
+ *   and must be ordered by the caller.  Each call rewrites all the scratch
+ *   it reads, so nothing needs clearing between calls. */
+rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layout, int B, int S, int N, int D,
+                                  int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
+                                  float sparsity, uint32_t* mask, int32_t* kept, float* margin, void* stream);
+
 /* Thread-local text of the last error returned on this thread. */
 const char* rf_last_error_string(void);
 
