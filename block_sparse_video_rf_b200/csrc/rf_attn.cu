@@ -9,21 +9,30 @@
 //
 // Work unit: one 128-row query tile of one (b, head).  Its KV list is every
 // prefix tile, then either every sparse block (dense tile) or the blocks set
-// in its mask row, in ascending order.  Persistent CTAs (two per SM) take
+// in its mask row, in ascending order.  Persistent CTAs (one per SM) take
 // units from a global counter in (head, tile) order, dense tiles of a head
 // first, so the heads in flight keep their K/V in L2.
 //
-// CTA = 6 warps:
-//   warps 0-3  softmax: thread t owns query row t (TMEM lane t); online
-//              softmax in exp2 with a lazily updated running max, P written
-//              back to TMEM as bf16, epilogue O / l -> bf16 -> global.
-//   warp 4     TMA producer (one thread): Q tile, then K and V tiles of the
-//              KV list, 128-byte swizzled boxes of 128 rows x 64 columns.
-//   warp 5     MMA issuer (one thread) and TMEM owner:
+// CTA = 10 warps, software-pipelined over the KV list:
+//   warps 0-7  softmax: warps w and w + 4 share query rows 32 (w % 4) ..
+//              32 (w % 4) + 31 (TMEM lanes) and split the 128 key columns in
+//              halves; the row max and the row sum are combined through
+//              shared memory.  Online softmax in exp2 with a lazily updated
+//              running max.  Most exponentials run on the MUFU unit, one
+//              pair in four on the FMA pipe (polynomial).  At the end of a
+//              unit the same threads write O / l -> bf16 -> the caller's
+//              layout while the tensor pipe starts the next unit.
+//   warp 8     TMA producer (one thread): Q tile, K and V tiles of the KV
+//              list through 3- and 2-stage rings of 128-byte swizzled boxes
+//              (128 rows x 64 columns), K two tiles ahead of V.
+//   warp 9     MMA issuer (one thread) and TMEM owner:
 //              S = Q K^T   (tcgen05 kind::f16, A/B from shared memory)
 //              O += P V    (A = P from tensor memory, B = V MN-major)
-// Tensor memory (256 columns): S fp32 in [0, 128), aliased by P bf16 in
-// [0, 64); O fp32 in [128, 256).
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256) double-buffer the
+// score tile; O [256,384) is the accumulator; P0 [384,448), P1 [448,512)
+// double-buffer P as bf16.  The QK of tile j+2 only waits for the softmax to
+// have read S of tile j, so the tensor pipe runs S = Q K^T of later tiles
+// while the softmax of tile j is still computing.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -39,12 +48,16 @@ namespace rf {
 
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 320;
+constexpr int kSoftmaxThreads = 256;
+constexpr int kKStages = 3;                              // K ring depth
+constexpr int kVStages = 2;                              // V ring depth
+constexpr int kKAhead = 2;                               // K tiles issued ahead of V
 constexpr int kTileBytes = RF_BLOCK * RF_HEAD_DIM * 2;   // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;               // 64 columns x 128 rows
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0, kColO = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;  // S b at 128 b; P b at 384 + 64 b
+constexpr int kPolyEvery = 4;                            // pair i uses the polynomial when i % 4 == 3
 constexpr float kRescaleThreshold = 8.0f;                // log2 units
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -54,12 +67,17 @@ struct Item {
 
 struct __align__(1024) Smem {
   uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
-  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
-  uint64_t s_full, p_full, pv_done, o_empty;
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kTileBytes];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_read[2], p_full[2], p_free[2];
+  uint64_t o_full, o_empty;
+  uint64_t xbar[4];             // per row quadrant: rendezvous of its two softmax warps
   uint64_t item_full[2], item_empty[2];
   Item items[2];
+  float xmax[2][2][RF_BLOCK];   // [tile parity][column half][row] partial row maxima
+  float xsum[2][RF_BLOCK];      // [column half][row] partial row sums at the end of a unit
   uint32_t tmem_base;
   int abort;
 };
@@ -81,46 +99,104 @@ __device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
   return p.g.dense || qt < p.n_ptiles || (qt - p.n_ptiles) < p.g.ff;
 }
 
+// Bounded wait by one thread.
+__device__ __forceinline__ bool wait1(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
+  return rf_wait(bar, parity, &sm.abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs);
+}
+// Bounded wait by a whole warp, with a warp-uniform outcome (the warp then
+// runs .sync.aligned tcgen05 instructions together or leaves together).
+__device__ __forceinline__ bool waitw(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xFFFFFFFFu, wait1(sm, p, bar, parity));
+}
+// Parity of completion number n (0-based) of a barrier phase.
+__device__ __forceinline__ uint32_t ph(uint32_t n) { return n & 1u; }
+
+// Rendezvous of the two softmax warps that share a row quadrant, on an
+// mbarrier (bounded wait, so a warp that leaves on an abort cannot strand its
+// partner).  Orders each thread's earlier shared-memory writes before the
+// partner's later reads.
+__device__ __forceinline__ bool pair_sync(Smem& sm, const AttnParams& p, int quad, uint32_t& phase) {
+  mbar_arrive(&sm.xbar[quad]);
+  return waitw(sm, p, &sm.xbar[quad], ph(phase++));
+}
+
 // ---------------------------------------------------------------- producer
+// Visits the KV tile rows of one unit in order: every prefix tile, then every
+// sparse block (dense unit) or the set bits of its mask row.
+struct KvIter {
+  int base, n_ptiles, nb, words;
+  const uint32_t* mrow;   // nullptr for a dense unit
+  int t, wd;
+  uint32_t bits;
+  __device__ void init(int base_, const AttnParams& p, const uint32_t* mrow_) {
+    base = base_;
+    n_ptiles = p.n_ptiles;
+    nb = p.g.nb;
+    words = p.g.mask_words;
+    mrow = mrow_;
+    t = 0;
+    wd = 0;
+    bits = 0;
+  }
+  // Row of the next KV tile, or -1 at the end.
+  __device__ int next() {
+    if (t < n_ptiles) return base + (t++) * RF_BLOCK;
+    if (!mrow) {
+      const int j = t - n_ptiles;
+      if (j >= nb) return -1;
+      ++t;
+      return base + (n_ptiles + j) * RF_BLOCK;
+    }
+    while (bits == 0) {
+      if (wd >= words) return -1;
+      bits = mrow[wd++];
+    }
+    const int j = 32 * (wd - 1) + __ffs(bits) - 1;
+    bits &= bits - 1;
+    return base + (n_ptiles + j) * RF_BLOCK;
+  }
+};
+
 __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv) {
-  volatile int* abort = &sm.abort;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  uint32_t it = 0, nq = 0, nk = 0, nv = 0;
+  uint32_t c = 0, gk = 0, gv = 0;   // units, K tiles and V tiles issued
   const int S_int = p.g.S_int;
   bool ok = true;
 
-  auto load_kv = [&](int row) -> bool {
-    if (nk > 0 && !rf_wait(&sm.k_empty, (nk - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return false;
-    mbar_arrive_expect_tx(&sm.k_full, kTileBytes);
-    tma_load_2d(sm.k, tk, &sm.k_full, 0, row, pol_kv);
-    tma_load_2d(sm.k + kHalfBytes, tk, &sm.k_full, 64, row, pol_kv);
-    ++nk;
-    if (nv > 0 && !rf_wait(&sm.v_empty, (nv - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return false;
-    mbar_arrive_expect_tx(&sm.v_full, kTileBytes);
-    tma_load_2d(sm.v, tv, &sm.v_full, 0, row, pol_kv);
-    tma_load_2d(sm.v + kHalfBytes, tv, &sm.v_full, 64, row, pol_kv);
-    ++nv;
+  auto load_k = [&](int row) -> bool {
+    const uint32_t st = gk % kKStages, use = gk / kKStages;
+    if (use > 0 && !wait1(sm, p, &sm.k_empty[st], ph(use - 1))) return false;
+    mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
+    tma_load_2d(sm.k[st], tk, &sm.k_full[st], 0, row, pol_kv);
+    tma_load_2d(sm.k[st] + kHalfBytes, tk, &sm.k_full[st], 64, row, pol_kv);
+    ++gk;
+    return true;
+  };
+  auto load_v = [&](int row) -> bool {
+    const uint32_t st = gv % kVStages, use = gv / kVStages;
+    if (use > 0 && !wait1(sm, p, &sm.v_empty[st], ph(use - 1))) return false;
+    mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
+    tma_load_2d(sm.v[st], tv, &sm.v_full[st], 0, row, pol_kv);
+    tma_load_2d(sm.v[st] + kHalfBytes, tv, &sm.v_full[st], 64, row, pol_kv);
+    ++gv;
     return true;
   };
 
   while (ok) {
     const int w = atomicAdd(p.counter, 1);
-    const int slot = it & 1;
-    if (it >= 2 && !rf_wait(&sm.item_empty[slot], ((it >> 1) - 1) & 1, abort, p.status, RF_ERR_TIMEOUT,
-                            kWaitLimitNs)) {
+    const uint32_t slot = c & 1;
+    if (c >= 2 && !wait1(sm, p, &sm.item_empty[slot], ph((c >> 1) - 1))) {
       ok = false;
       break;
     }
     Item itm{-1, 0, 0, 0};
     const uint32_t* mrow = nullptr;
-    bool dense = true;
     if (w < p.total_items) {
       itm.bn = w / p.g.n_tiles;
       itm.qt = w - itm.bn * p.g.n_tiles;
-      dense = is_dense_tile(p, itm.qt);
-      if (dense) {
+      if (is_dense_tile(p, itm.qt)) {
         itm.ntiles = p.g.n_tiles;
       } else {
         mrow = p.mask + ((size_t)itm.bn * p.g.nb + (itm.qt - p.n_ptiles)) * p.g.mask_words;
@@ -131,135 +207,170 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
     }
     sm.items[slot] = itm;
     mbar_arrive(&sm.item_full[slot]);
-    ++it;
     if (itm.bn < 0) break;
 
     const int base = itm.bn * S_int;
-    if (nq > 0 && !rf_wait(&sm.q_empty, (nq - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) {
+    if (c >= 1 && !wait1(sm, p, &sm.q_empty, ph(c - 1))) {
       ok = false;
       break;
     }
     mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
     tma_load_2d(sm.q, tq, &sm.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
     tma_load_2d(sm.q + kHalfBytes, tq, &sm.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
-    ++nq;
+    ++c;
 
-    for (int t = 0; t < p.n_ptiles && ok; ++t) ok = load_kv(base + t * RF_BLOCK);
-    if (dense) {
-      for (int j = 0; j < p.g.nb && ok; ++j) ok = load_kv(base + (p.n_ptiles + j) * RF_BLOCK);
-    } else {
-      for (int wd = 0; wd < p.g.mask_words && ok; ++wd) {
-        uint32_t bits = mrow[wd];
-        while (bits && ok) {
-          const int j = 32 * wd + __ffs(bits) - 1;
-          bits &= bits - 1;
-          ok = load_kv(base + (p.n_ptiles + j) * RF_BLOCK);
-        }
-      }
+    // K runs kKAhead tiles ahead of V: K0, K1, K2, V0, K3, V1, ..., V(n-1).
+    KvIter kit, vit;
+    kit.init(base, p, mrow);
+    vit.init(base, p, mrow);
+    for (int i = 0; i < kKAhead && ok; ++i) {
+      const int rk = kit.next();
+      if (rk < 0) break;
+      ok = load_k(rk);
+    }
+    while (ok) {
+      const int rk = kit.next();
+      if (rk >= 0) ok = load_k(rk);
+      if (!ok) break;
+      const int rv = vit.next();
+      if (rv < 0) break;
+      ok = load_v(rv);
     }
   }
   if (!ok) {
-    // Let the copies already issued land before the CTA may exit.
-    if (nq > 0) rf_wait(&sm.q_full, (nq - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs / 4);
-    if (nk > 0) rf_wait(&sm.k_full, (nk - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs / 4);
-    if (nv > 0) rf_wait(&sm.v_full, (nv - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs / 4);
+    // Let the copies already issued land before the CTA may exit (bounded).
+    const uint64_t lim = kWaitLimitNs / 4;
+    if (c) rf_wait(&sm.q_full, ph(c - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+    for (uint32_t st = 0; st < kKStages; ++st) {
+      const uint32_t nk = (gk > st) ? (gk - st + kKStages - 1) / kKStages : 0;
+      if (nk) rf_wait(&sm.k_full[st], ph(nk - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+    }
+    for (uint32_t st = 0; st < kVStages; ++st) {
+      const uint32_t nv = (gv > st) ? (gv - st + kVStages - 1) / kVStages : 0;
+      if (nv) rf_wait(&sm.v_full[st], ph(nv - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+    }
   }
 }
 
 // ---------------------------------------------------------------- MMA issuer
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_addr, uint32_t k_addr) {
+  constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
+    mma_ss(s_tmem, make_sdesc_sw128(q_addr + off, 16, 1024), make_sdesc_sw128(k_addr + off, 16, 1024), idesc,
+           kk > 0);
+  }
+}
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
+  constexpr uint32_t idesc = make_idesc_bf16(128, 128, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    mma_ts(o_tmem, p_tmem + kk * 8, make_sdesc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
 __device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
-  volatile int* abort = &sm.abort;
-  constexpr uint32_t idesc_qk = make_idesc_bf16(128, 128, false);
-  constexpr uint32_t idesc_pv = make_idesc_bf16(128, 128, true);
-  const uint32_t q_addr = smem_u32(sm.q), k_addr = smem_u32(sm.k), v_addr = smem_u32(sm.v);
-  uint32_t it = 0, nq = 0, nk = 0, nv = 0, np = 0, npv = 0, items_done = 0;
+  uint32_t c = 0, g = 0;   // units and KV tiles consumed
+  // S of tile t into buffer t % 2: needs K tile t and S of tile t-2 read by the softmax.
+  auto qk = [&](uint32_t t) -> bool {
+    const uint32_t st = t % kKStages, sb = t & 1;
+    if (!wait1(sm, p, &sm.k_full[st], ph(t / kKStages))) return false;
+    if (t >= 2 && !wait1(sm, p, &sm.s_read[sb], ph((t >> 1) - 1))) return false;
+    tc_fence_after();
+    issue_qk(tmem + kColS + 128 * sb, smem_u32(sm.q), smem_u32(sm.k[st]));
+    mma_commit(&sm.s_full[sb]);
+    mma_commit(&sm.k_empty[st]);
+    return true;
+  };
   for (;;) {
-    const int slot = it & 1;
-    if (!rf_wait(&sm.item_full[slot], (it >> 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
+    const uint32_t slot = c & 1;
+    if (!wait1(sm, p, &sm.item_full[slot], ph(c >> 1))) return;
     const Item itm = sm.items[slot];
     mbar_arrive(&sm.item_empty[slot]);
-    ++it;
     if (itm.bn < 0) return;
-    if (!rf_wait(&sm.q_full, nq & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-    ++nq;
-    for (int j = 0; j < itm.ntiles; ++j) {
-      if (!rf_wait(&sm.k_full, nk & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-      ++nk;
-      // P of the previous tile lives in the S columns: its P*V must be done.
-      if (npv > 0 && !rf_wait(&sm.pv_done, (npv - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tmem + kColS, make_sdesc_sw128(q_addr + off, 16, 1024), make_sdesc_sw128(k_addr + off, 16, 1024),
-               idesc_qk, kk > 0);
+    const uint32_t n = itm.ntiles;
+    if (!wait1(sm, p, &sm.q_full, ph(c))) return;
+    if (!qk(g)) return;
+    if (n == 1) mma_commit(&sm.q_empty);
+    for (uint32_t j = 0; j < n; ++j) {
+      const uint32_t t = g + j, pb = t & 1, vs = t % kVStages;
+      if (j + 1 < n) {
+        if (!qk(t + 1)) return;
+        if (j + 2 == n) mma_commit(&sm.q_empty);
       }
-      mma_commit(&sm.s_full);
-      mma_commit(&sm.k_empty);
-      if (j == itm.ntiles - 1) mma_commit(&sm.q_empty);
-
-      if (!rf_wait(&sm.p_full, np & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-      ++np;
-      if (!rf_wait(&sm.v_full, nv & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-      ++nv;
-      if (j == 0 && items_done > 0 &&
-          !rf_wait(&sm.o_empty, (items_done - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs))
-        return;
+      if (!wait1(sm, p, &sm.p_full[pb], ph(t >> 1))) return;
+      if (!wait1(sm, p, &sm.v_full[vs], ph(t / kVStages))) return;
+      // the epilogue of the previous unit must have read O
+      if (j == 0 && c >= 1 && !wait1(sm, p, &sm.o_empty, ph(c - 1))) return;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        mma_ts(tmem + kColO, tmem + kColS + kk * 8, make_sdesc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), idesc_pv,
-               (j > 0 || kk > 0) ? 1u : 0u);
-      }
-      mma_commit(&sm.pv_done);
-      mma_commit(&sm.v_empty);
-      ++npv;
+      issue_pv(tmem + kColO, tmem + kColP + 64 * pb, smem_u32(sm.v[vs]), j > 0);
+      mma_commit(&sm.p_free[pb]);
+      mma_commit(&sm.v_empty[vs]);
+      if (j + 1 == n) mma_commit(&sm.o_full);
     }
-    ++items_done;
+    g += n;
+    ++c;
   }
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
 __device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
-  volatile int* abort = &sm.abort;
-  const int row = threadIdx.x;                 // 0..127 == TMEM lane
-  const int warp = row >> 5;
-  const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
-  const uint32_t tS = lane_base + kColS, tO = lane_base + kColO;
+  const int warp = threadIdx.x >> 5;           // 0..7
+  const int quad = warp & 3, half = warp >> 2;
+  const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
+  const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tO = lane_base + kColO + 64 * half;
+  const int col0 = 64 * half;                  // first key column of this thread
   const float sl2 = p.scale_log2;
-  uint32_t it = 0, ns = 0, npv = 0;
+  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+  uint32_t c = 0, g = 0, xph = 0;
   for (;;) {
-    const int slot = it & 1;
-    if (!rf_wait(&sm.item_full[slot], (it >> 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
+    const uint32_t slot = c & 1;
+    if (!waitw(sm, p, &sm.item_full[slot], ph(c >> 1))) return;
     const Item itm = sm.items[slot];
     mbar_arrive(&sm.item_empty[slot]);
-    ++it;
     if (itm.bn < 0) return;
 
     float m_use = -CUDART_INF_F, l = 0.f;
     for (int j = 0; j < itm.ntiles; ++j) {
-      if (!rf_wait(&sm.s_full, ns & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
-      ++ns;
+      const uint32_t t = g + j, sb = t & 1;
+      const uint32_t tS = lane_base + kColS + 128 * sb + col0;
+      const uint32_t tP = lane_base + kColP + 64 * sb + 32 * half;
+      if (!waitw(sm, p, &sm.s_full[sb], ph(t >> 1))) return;
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+      uint32_t s[2][32];
+      tmem_ld32(tS, s[0]);
+      tmem_ld32(tS + 32, s[1]);
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence32(s[c]);
+      reg_fence32(s[0]);
+      reg_fence32(s[1]);
+      // S is in registers: the tensor pipe may overwrite this buffer.
+      tc_fence_before();
+      mbar_arrive(&sm.s_read[sb]);
 
-      if (p.p_rem != 0 && j == p.n_ptiles - 1) {
+      const bool partial = (p.p_rem != 0 && j == p.n_ptiles - 1);
+      if (partial) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (32 * c + e >= p.p_rem) s[c][e] = __float_as_uint(-CUDART_INF_F);
+            if (col0 + 32 * q2 + e >= p.p_rem) s[q2][e] = __float_as_uint(-CUDART_INF_F);
       }
-      float mx = -CUDART_INF_F;
+      // row max over this half: 8 independent chains of 3-input max
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(s[c][e]));
+      for (int q2 = 0; q2 < 2; ++q2)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q2][e]), __uint_as_float(s[q2][e + 1]));
+      const float mxh = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+      // combine with the other half of the row
+      sm.xmax[sb][half][row] = mxh;
+      if (!pair_sync(sm, p, quad, xph)) return;
+      const float mx = fmaxf(mxh, sm.xmax[sb][half ^ 1][row]);
       const float mx_s = mx * sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -270,70 +381,100 @@ __device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
         m_use = mx_s;
         rescale = true;
       }
-      // exponentials, packed to bf16 pairs in place (s[c][0..15] of each chunk)
-      float sum = 0.f;
-      uint32_t pk[64];
+      // p = 2^(s * scale * log2 e - m): pairs, packed fp32 arithmetic
+      const uint64_t negm = f2_pack(-m_use, -m_use);
+      uint64_t sum2[4] = {0, 0, 0, 0};
+      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int q2 = 0; q2 < 2; ++q2)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[c][e]), sl2, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[c][e + 1]), sl2, -m_use));
-          sum += p0 + p1;
-          pk[16 * c + e / 2] = pack_bf16x2(p0, p1);
+          const int i = 16 * q2 + (e >> 1);     // pair index 0..31 within this half
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q2][e]), __uint_as_float(s[q2][e + 1])), sl2x2, negm);
+          uint64_t p2;
+          if ((i % kPolyEvery) == kPolyEvery - 1) {
+            p2 = exp2_poly_x2(x2);
+          } else {
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+          }
+          if (partial) {
+            float a0, a1;
+            f2_unpack(p2, a0, a1);
+            const int k0 = col0 + 2 * i;
+            p2 = f2_pack(k0 < p.p_rem ? a0 : 0.f, k0 + 1 < p.p_rem ? a1 : 0.f);
+          }
+          sum2[i & 3] = f2_add(sum2[i & 3], p2);
+          float a0, a1;
+          f2_unpack(p2, a0, a1);
+          pk[i] = pack_bf16x2(a0, a1);
         }
-      l = l * alpha + sum;
+      float s0, s1, s2, s3;
+      f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
+      f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
+      l = l * alpha + ((s0 + s1) + (s2 + s3));
       if (__any_sync(0xFFFFFFFFu, rescale)) {
-        // O holds the sum over the tiles before j (their P*V completed before
-        // this tile's S was computed).
+        // O holds the tiles before j once the P*V of tile j-1 is done.
+        if (!waitw(sm, p, &sm.p_free[(t - 1) & 1], ph((t - 1) >> 1))) return;
+        tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int q2 = 0; q2 < 2; ++q2) {
           uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
+          tmem_ld32(tO + 32 * q2, o);
           tmem_wait_ld();
           reg_fence32(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+          tmem_st32(tO + 32 * q2, o);
         }
       }
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      // P buffer sb is free once the P*V of tile t-2 is done
+      if (t >= 2 && !waitw(sm, p, &sm.p_free[sb], ph((t >> 1) - 1))) return;
+      tc_fence_after();
+      tmem_st32(tP, pk);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full);
-      ++npv;
+      mbar_arrive(&sm.p_full[sb]);
     }
-
-    // epilogue: wait for the last P*V of this tile
-    if (!rf_wait(&sm.pv_done, (npv - 1) & 1, abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs)) return;
+    // epilogue: O / l of this unit once its last P*V is done
+    if (!waitw(sm, p, &sm.o_full, ph(c))) return;
     tc_fence_after();
-    const float rl = 1.f / l;
+    uint32_t o[2][32];
+    tmem_ld32(tO, o[0]);
+    tmem_ld32(tO + 32, o[1]);
+    tmem_wait_ld();
+    reg_fence32(o[0]);
+    reg_fence32(o[1]);
+    // O is in registers: the next unit may start accumulating.
+    tc_fence_before();
+    mbar_arrive(&sm.o_empty);
+    // xsum is rewritten only at the end of the next unit, after at least one
+    // more rendezvous, so one rendezvous here is enough.
+    sm.xsum[half][row] = l;
+    if (!pair_sync(sm, p, quad, xph)) return;
+    const float rl = 1.f / (sm.xsum[0][row] + sm.xsum[1][row]);
     const int b = itm.bn / p.N, n = itm.bn - b * p.N;
     const int src = rf_src_of_row(p.g, itm.qt * RF_BLOCK + row);
-    __nv_bfloat16* dst = src >= 0 ? p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, n, src) : nullptr;
-#pragma unroll 1
-    for (int c = 0; c < 4; ++c) {
-      uint32_t o[32];
-      tmem_ld32(tO + 32 * c, o);
-      tmem_wait_ld();
-      reg_fence32(o);
-      uint32_t w[16];
+    if (src >= 0) {
+      __nv_bfloat16* dst = p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, n, src) + col0;
 #pragma unroll
-      for (int e = 0; e < 16; ++e)
-        w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
-      if (dst) {
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * c);
+      for (int q2 = 0; q2 < 2; ++q2) {
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(o[q2][2 * e]) * rl, __uint_as_float(o[q2][2 * e + 1]) * rl);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q2);
 #pragma unroll
         for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
-    tc_fence_before();
-    mbar_arrive(&sm.o_empty);
+    g += itm.ntiles;
+    ++c;
   }
 }
 
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -343,27 +484,34 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    mbar_init(&sm.k_full, 1);
-    mbar_init(&sm.k_empty, 1);
-    mbar_init(&sm.v_full, 1);
-    mbar_init(&sm.v_empty, 1);
-    mbar_init(&sm.s_full, 1);
-    mbar_init(&sm.p_full, kSoftmaxThreads);
-    mbar_init(&sm.pv_done, 1);
-    mbar_init(&sm.o_empty, kSoftmaxThreads);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_read[i], kSoftmaxThreads);
+      mbar_init(&sm.p_full[i], kSoftmaxThreads);
+      mbar_init(&sm.p_free[i], 1);
       mbar_init(&sm.item_full[i], 1);
       mbar_init(&sm.item_empty[i], kSoftmaxThreads + 1);
     }
+    for (int i = 0; i < kKStages; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.v_empty[i], 1);
+    }
+    mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.o_empty, kSoftmaxThreads);
+    for (int i = 0; i < 4; ++i) mbar_init(&sm.xbar[i], 64);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -372,9 +520,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp < 4) {
+  if (warp < 8) {
     softmax_loop(sm, p, tmem);
-  } else if (warp == 4) {
+  } else if (warp == 8) {
     if (lane == 0) producer_loop(sm, p, &tm_q, &tm_k, &tm_v);
   } else {
     if (lane == 0) mma_loop(sm, p, tmem);
@@ -383,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------- host side
@@ -450,7 +598,7 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
-  const int grid = std::min(2 * sms, p.total_items);
+  const int grid = std::min(sms, p.total_items);
   attn_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }

@@ -195,6 +195,61 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------- packed fp32 (sm_100)
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^x for a pair on the FMA pipe instead of the MUFU unit.
+// x = n + f with n = round(x) (the 1.5 * 2^23 rounding trick, exact) and
+// f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted here for minimum
+// relative error on [-0.5, 0.5] (max relative error 7.5e-5, far below the
+// bf16 rounding of P); 2^n by adding n to the exponent field.  Inputs are
+// clamped at -125 so the exponent field stays normal: anything below gives
+// 2^-125 (about 2.4e-38) instead of a smaller number; callers that need an
+// exact 0 (masked keys) zero those lanes themselves.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+  float a, b;
+  f2_unpack(x2, a, b);
+  const uint64_t xc = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
+  const uint64_t minus1 = f2_pack(-1.f, -1.f);
+  const uint64_t t = f2_add(xc, magic);            // n in the low mantissa bits
+  const uint64_t nf = f2_add(t, neg_magic);        // n as a float
+  const uint64_t f = f2_fma(nf, minus1, xc);       // x - n, exact
+  uint64_t p = f2_fma(f, f2_pack(0.0551716685295105f, 0.0551716685295105f),
+                      f2_pack(0.2426111400127411f, 0.2426111400127411f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float pl, ph, tl, th;
+  f2_unpack(p, pl, ph);
+  f2_unpack(t, tl, th);
+  const int rl = __float_as_int(pl) + (__float_as_int(tl) << 23);
+  const int rh = __float_as_int(ph) + (__float_as_int(th) << 23);
+  return f2_pack(__int_as_float(rl), __int_as_float(rh));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
