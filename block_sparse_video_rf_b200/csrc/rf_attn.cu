@@ -253,32 +253,40 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
 }
 
 // ---------------------------------------------------------------- MMA issuer
-__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_addr, uint32_t k_addr) {
+// Descriptor low words of the 128-byte swizzled operands; every descriptor
+// used here shares one high word (stride 1024 B, sm_100 version, swizzle).
+// A K step of 16 elements advances a K-major operand by 32 B (2 in the
+// descriptor's 16-byte units), and the second 64-column half by 16 KB.
+__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
   constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-    mma_ss(s_tmem, make_sdesc_sw128(q_addr + off, 16, 1024), make_sdesc_sw128(k_addr + off, 16, 1024), idesc,
-           kk > 0);
+    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
+    mma_ss_lo(s_tmem, q_lo + off, k_lo + off, hi, idesc, kk > 0);
   }
 }
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_addr, bool accumulate) {
+// V is MN-major: a K step of 16 keys advances it by 16 rows of 128 B.
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
+                                         bool accumulate) {
   constexpr uint32_t idesc = make_idesc_bf16(128, 128, true);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_ts(o_tmem, p_tmem + kk * 8, make_sdesc_sw128(v_addr + kk * 2048, kHalfBytes, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
   uint32_t c = 0, g = 0;   // units and KV tiles consumed
+  const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
+  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sm.q), 16, 1024);
+  const uint32_t k_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
+  const uint32_t v_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.v[0]), kHalfBytes, 1024);
   // S of tile t into buffer t % 2: needs K tile t and S of tile t-2 read by the softmax.
   auto qk = [&](uint32_t t) -> bool {
     const uint32_t st = t % kKStages, sb = t & 1;
     if (!wait1(sm, p, &sm.k_full[st], ph(t / kKStages))) return false;
     if (t >= 2 && !wait1(sm, p, &sm.s_read[sb], ph((t >> 1) - 1))) return false;
     tc_fence_after();
-    issue_qk(tmem + kColS + 128 * sb, smem_u32(sm.q), smem_u32(sm.k[st]));
+    issue_qk(tmem + kColS + 128 * sb, q_lo, k_lo0 + st * (kTileBytes >> 4), hi);
     mma_commit(&sm.s_full[sb]);
     mma_commit(&sm.k_empty[st]);
     return true;
@@ -304,7 +312,7 @@ __device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
       // the epilogue of the previous unit must have read O
       if (j == 0 && c >= 1 && !wait1(sm, p, &sm.o_empty, ph(c - 1))) return;
       tc_fence_after();
-      issue_pv(tmem + kColO, tmem + kColP + 64 * pb, smem_u32(sm.v[vs]), j > 0);
+      issue_pv(tmem + kColO, tmem + kColP + 64 * pb, v_lo0 + vs * (kTileBytes >> 4), hi, j > 0);
       mma_commit(&sm.p_free[pb]);
       mma_commit(&sm.v_empty[vs]);
       if (j + 1 == n) mma_commit(&sm.o_full);
