@@ -23,6 +23,15 @@ namespace {
 
 thread_local std::string g_last_error;
 
+// Process-wide test controls of the attention kernel (rf_debug_set_wait).
+std::mutex g_debug_mu;
+rf::AttnDebug g_debug;
+
+rf::AttnDebug debug_settings() {
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  return g_debug;
+}
+
 rf_status_t fail(rf_status_t code, const char* fmt, ...) {
   char buf[512];
   va_list ap;
@@ -229,7 +238,7 @@ rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_le
   if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
   e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
                                        at<uint32_t>(ws, L.mask), layout, B, S, N, g, resolve_scale(scale, D), out,
-                                       at<int>(ws, L.counter), at<int>(ws, L.status),
+                                       at<int>(ws, L.counter), at<int>(ws, L.status), debug_settings(),
                                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
@@ -342,6 +351,15 @@ rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layo
   cudaError_t e = rf::launch_block_mask_noalloc(q, k, layout, B, S, N, g, mask, kept, margin,
                                                 static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "no-allocation mask launch");
+  return ok();
+}
+
+rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q) {
+  if (wait_limit_ns < 0 || (skip_first_q != 0 && skip_first_q != 1))
+    return fail(RF_ERR_ARG, "wait limit must be >= 0 and skip_first_q 0 or 1");
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  g_debug.wait_limit_ns = wait_limit_ns;
+  g_debug.skip_first_q = skip_first_q;
   return ok();
 }
 

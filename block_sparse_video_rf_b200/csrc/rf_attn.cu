@@ -73,6 +73,7 @@ struct __align__(1024) Smem {
   uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_read[2], p_full[2], p_free[2];
   uint64_t o_full, o_empty;
+  uint64_t drain;               // MMA issuer's last commit when it leaves early
   uint64_t xbar[4];             // per row quadrant: rendezvous of its two softmax warps
   uint64_t item_full[2], item_empty[2];
   Item items[2];
@@ -93,6 +94,8 @@ struct AttnParams {
   int* counter;
   int* status;
   __nv_bfloat16* out;
+  uint64_t wait_limit_ns;   // limit of every device-side wait
+  int skip_first_q;         // test control: the first unit's Q load is never issued
 };
 
 __device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
@@ -101,7 +104,7 @@ __device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
 
 // Bounded wait by one thread.
 __device__ __forceinline__ bool wait1(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
-  return rf_wait(bar, parity, &sm.abort, p.status, RF_ERR_TIMEOUT, kWaitLimitNs);
+  return rf_wait(bar, parity, &sm.abort, p.status, RF_ERR_TIMEOUT, p.wait_limit_ns);
 }
 // Bounded wait by a whole warp, with a warp-uniform outcome (the warp then
 // runs .sync.aligned tcgen05 instructions together or leaves together).
@@ -214,9 +217,11 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
       ok = false;
       break;
     }
-    mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-    tma_load_2d(sm.q, tq, &sm.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
-    tma_load_2d(sm.q + kHalfBytes, tq, &sm.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
+    if (!(p.skip_first_q && c == 0)) {
+      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
+      tma_load_2d(sm.q, tq, &sm.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
+      tma_load_2d(sm.q + kHalfBytes, tq, &sm.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
+    }
     ++c;
 
     // K runs kKAhead tiles ahead of V: K0, K1, K2, V0, K3, V1, ..., V(n-1).
@@ -238,16 +243,17 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
     }
   }
   if (!ok) {
-    // Let the copies already issued land before the CTA may exit (bounded).
-    const uint64_t lim = kWaitLimitNs / 4;
-    if (c) rf_wait(&sm.q_full, ph(c - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+    // Let the copies already issued land before the CTA may exit (bounded by
+    // time, not cut short by the abort flag).
+    const uint64_t lim = p.wait_limit_ns / 4;
+    if (c) rf_wait_time(&sm.q_full, ph(c - 1), lim);
     for (uint32_t st = 0; st < kKStages; ++st) {
       const uint32_t nk = (gk > st) ? (gk - st + kKStages - 1) / kKStages : 0;
-      if (nk) rf_wait(&sm.k_full[st], ph(nk - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+      if (nk) rf_wait_time(&sm.k_full[st], ph(nk - 1), lim);
     }
     for (uint32_t st = 0; st < kVStages; ++st) {
       const uint32_t nv = (gv > st) ? (gv - st + kVStages - 1) / kVStages : 0;
-      if (nv) rf_wait(&sm.v_full[st], ph(nv - 1), &sm.abort, p.status, RF_ERR_TIMEOUT, lim);
+      if (nv) rf_wait_time(&sm.v_full[st], ph(nv - 1), lim);
     }
   }
 }
@@ -274,7 +280,7 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
     mma_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-__device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
+__device__ bool mma_loop_body(Smem& sm, const AttnParams& p, uint32_t tmem) {
   uint32_t c = 0, g = 0;   // units and KV tiles consumed
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
   const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sm.q), 16, 1024);
@@ -293,24 +299,24 @@ __device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
   };
   for (;;) {
     const uint32_t slot = c & 1;
-    if (!wait1(sm, p, &sm.item_full[slot], ph(c >> 1))) return;
+    if (!wait1(sm, p, &sm.item_full[slot], ph(c >> 1))) return false;
     const Item itm = sm.items[slot];
     mbar_arrive(&sm.item_empty[slot]);
-    if (itm.bn < 0) return;
+    if (itm.bn < 0) return true;
     const uint32_t n = itm.ntiles;
-    if (!wait1(sm, p, &sm.q_full, ph(c))) return;
-    if (!qk(g)) return;
+    if (!wait1(sm, p, &sm.q_full, ph(c))) return false;
+    if (!qk(g)) return false;
     if (n == 1) mma_commit(&sm.q_empty);
     for (uint32_t j = 0; j < n; ++j) {
       const uint32_t t = g + j, pb = t & 1, vs = t % kVStages;
       if (j + 1 < n) {
-        if (!qk(t + 1)) return;
+        if (!qk(t + 1)) return false;
         if (j + 2 == n) mma_commit(&sm.q_empty);
       }
-      if (!wait1(sm, p, &sm.p_full[pb], ph(t >> 1))) return;
-      if (!wait1(sm, p, &sm.v_full[vs], ph(t / kVStages))) return;
+      if (!wait1(sm, p, &sm.p_full[pb], ph(t >> 1))) return false;
+      if (!wait1(sm, p, &sm.v_full[vs], ph(t / kVStages))) return false;
       // the epilogue of the previous unit must have read O
-      if (j == 0 && c >= 1 && !wait1(sm, p, &sm.o_empty, ph(c - 1))) return;
+      if (j == 0 && c >= 1 && !wait1(sm, p, &sm.o_empty, ph(c - 1))) return false;
       tc_fence_after();
       issue_pv(tmem + kColO, tmem + kColP + 64 * pb, v_lo0 + vs * (kTileBytes >> 4), hi, j > 0);
       mma_commit(&sm.p_free[pb]);
@@ -319,6 +325,15 @@ __device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
     }
     g += n;
     ++c;
+  }
+}
+
+// Leaves after the last unit, or early on an abort; in the latter case the
+// MMAs already issued must finish before tensor memory is freed.
+__device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
+  if (!mma_loop_body(sm, p, tmem)) {
+    mma_commit(&sm.drain);
+    rf_wait_time(&sm.drain, 0, p.wait_limit_ns / 4);
   }
 }
 
@@ -509,6 +524,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sm.v_empty[i], 1);
     }
     mbar_init(&sm.o_full, 1);
+    mbar_init(&sm.drain, 1);
     mbar_init(&sm.o_empty, kSoftmaxThreads);
     for (int i = 0; i < 4; ++i) mbar_init(&sm.xbar[i], 64);
     sm.abort = 0;
@@ -576,7 +592,7 @@ bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) {
 
 cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
                              int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
-                             int* counter, int* status, cudaStream_t stream) {
+                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream) {
   const uint64_t rows = (uint64_t)B * N * g.S_int;
   CUtensorMap tq, tk, tv;
   if (!make_tile_map(&tq, q_int, rows) || !make_tile_map(&tk, k_int, rows) || !make_tile_map(&tv, v_int, rows))
@@ -595,6 +611,8 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
   p.counter = counter;
   p.status = status;
   p.out = static_cast<__nv_bfloat16*>(out);
+  p.wait_limit_ns = dbg.wait_limit_ns > 0 ? (uint64_t)dbg.wait_limit_ns : kWaitLimitNs;
+  p.skip_first_q = dbg.skip_first_q;
 
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);

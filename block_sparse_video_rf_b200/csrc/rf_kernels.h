@@ -23,11 +23,17 @@ cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N,
 cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g, uint32_t* mask,
                         int* kept, float* margin, cudaStream_t stream);
 
+// Test controls of the attention kernel's bounded waits (see rf_debug_set_wait).
+struct AttnDebug {
+  long long wait_limit_ns = 0;   // 0: the default limit (2 s)
+  int skip_first_q = 0;          // 1: the first unit of every CTA never gets its Q tile
+};
+
 // K3: block-sparse flash attention over the internal layout, output written
 // straight to the caller's layout (inverse reorder fused in the epilogue).
 cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
                              int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
-                             int* counter, int* status, cudaStream_t stream);
+                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream);
 
 // Block mask with the pooled means in the library's static scratch array
 // (no device allocation); see rf_block_mask_noalloc.

@@ -64,6 +64,17 @@ __device__ __forceinline__ bool rf_wait(uint64_t* bar, uint32_t parity, volatile
   }
 }
 
+// Wait bounded by time only (the abort flag is ignored): used to let a
+// thread's own asynchronous copies or MMAs finish before the CTA may exit.
+__device__ __forceinline__ bool rf_wait_time(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

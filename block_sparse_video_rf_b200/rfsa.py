@@ -29,7 +29,7 @@ WS_FIELDS = ["q_int", "k_int", "v_int", "pooled_q", "pooled_k", "mask", "kept", 
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_block_mask_noalloc", "rf_last_error_string"]
+           "rf_debug_set_wait", "rf_block_mask_noalloc", "rf_last_error_string"]
 
 
 class RfPlan(ctypes.Structure):
@@ -67,6 +67,7 @@ def _load():
         "rf_sparse_attention_host": (I, [P, P, P] + geo + [I, I, F, F, P, P]),
         "rf_read_status": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(I), P]),
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
+        "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "rf_last_error_string": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -192,6 +193,11 @@ def rf_block_mask_noalloc(q, k, layout, txt_len, latent, sparsity, mask, kept, m
     _check(LIB.rf_block_mask_noalloc(_ptr(q), _ptr(k), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
                                      block_size, float(sparsity), _ptr(mask), _ptr(kept), _ptr(margin),
                                      _stream(q, stream)))
+
+
+def rf_debug_set_wait(wait_limit_ns: int = 0, skip_first_q: int = 0):
+    """Test control of the attention kernel's bounded waits (see include/rfsa.h)."""
+    _check(LIB.rf_debug_set_wait(int(wait_limit_ns), int(skip_first_q)))
 
 
 def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:

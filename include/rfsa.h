@@ -145,6 +145,16 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
 rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                            int* status, void* stream);
 
+/* Test control of the device-side waits of the attention kernel, process-wide,
+ * read at each launch.  wait_limit_ns: limit of every wait (0 = the default,
+ * 2 s).  skip_first_q = 1: every CTA's first query tile never gets its Q
+ * copy, so the first wait on it runs out; the kernel then records
+ * RF_ERR_TIMEOUT in the workspace status word (read with rf_read_status),
+ * lets its issued copies land, frees its tensor memory and returns, and the
+ * output is not valid.  Used by the tests to exercise the timeout path
+ * without any fault; call with (0, 0) to restore normal operation. */
+rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q);
+
 /* Size of the library-owned static scratch array of rf_block_mask_noalloc,
  * per device (32 MiB): enough for B * N * nb <= 32768 block rows of pooled Q and K
  * (the 56-head MiniMax-H3 shape needs 26,040). */
