@@ -13,26 +13,29 @@
 // units from a global counter in (head, tile) order, dense tiles of a head
 // first, so the heads in flight keep their K/V in L2.
 //
-// CTA = 10 warps, software-pipelined over the KV list:
-//   warps 0-7  softmax: warps w and w + 4 share query rows 32 (w % 4) ..
-//              32 (w % 4) + 31 (TMEM lanes) and split the 128 key columns in
-//              halves; the row max and the row sum are combined through
-//              shared memory.  Online softmax in exp2 with a lazily updated
-//              running max.  Most exponentials run on the MUFU unit, one
-//              pair in four on the FMA pipe (polynomial).  At the end of a
-//              unit the same threads write O / l -> bf16 -> the caller's
-//              layout while the tensor pipe starts the next unit.
-//   warp 8     TMA producer (one thread): Q tile, K and V tiles of the KV
-//              list through 3- and 2-stage rings of 128-byte swizzled boxes
-//              (128 rows x 64 columns), K two tiles ahead of V.
-//   warp 9     MMA issuer (one thread) and TMEM owner:
-//              S = Q K^T   (tcgen05 kind::f16, A/B from shared memory)
-//              O += P V    (A = P from tensor memory, B = V MN-major)
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256) double-buffer the
-// score tile; O [256,384) is the accumulator; P0 [384,448), P1 [448,512)
-// double-buffer P as bf16.  The QK of tile j+2 only waits for the softmax to
-// have read S of tile j, so the tensor pipe runs S = Q K^T of later tiles
-// while the softmax of tile j is still computing.
+// A CTA runs two units at once in two independent slots, each with its own
+// Q/K/V shared-memory buffers, its own S and O in tensor memory and its own
+// warps, so that while the softmax of one slot runs the tensor pipe works on
+// the other slot's MMAs:
+//   warps 0-3   softmax of slot 0, warps 4-7 of slot 1: thread = query row
+//               (TMEM lane); online softmax in exp2 with a lazily updated
+//               running max; most exponentials on the MUFU unit, one pair in
+//               four on the FMA pipe (polynomial); P (bf16) is written over
+//               the first 64 columns of the slot's S; at the end of a unit
+//               the same threads write O / l -> bf16 -> the caller's layout.
+//   warps 8, 9  TMA producers of slot 0 and slot 1 (one thread each): Q, then
+//               the K and V tiles of the KV list, 128-byte swizzled boxes of
+//               128 rows x 64 columns.
+//   warps 10, 11 MMA issuers of slot 0 and slot 1 (one elected lane issues);
+//               warp 10 also owns the tensor memory.
+//               S = Q K^T: tcgen05 kind::f16, A and B from shared memory;
+//               O += P V:  A = P from tensor memory, B = V MN-major.
+// Tensor memory (512 columns): slot z has S at [256 z, 256 z + 128) (P in
+// its first 64 columns) and O at [256 z + 128, 256 z + 256).  Since P
+// overwrites S, the QK of a slot's next tile is issued once its P V is done.
+// Registers: the control warpgroup (warps 8-11) gives registers to the two
+// softmax warpgroups (setmaxnreg 64 / 216: 8 x 32 x 216 + 4 x 32 x 64 =
+// 63,488 <= 384 threads x 168 at launch).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -48,15 +51,13 @@ namespace rf {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kSoftmaxThreads = 256;
-constexpr int kKStages = 3;                              // K ring depth
-constexpr int kVStages = 2;                              // V ring depth
-constexpr int kKAhead = 2;                               // K tiles issued ahead of V
+constexpr int kThreads = 384;
+constexpr int kSlots = 2;
+constexpr int kSlotWarps = 4;                            // softmax warps per slot
+constexpr uint32_t kRegsSoftmax = 216, kRegsControl = 64;
 constexpr int kTileBytes = RF_BLOCK * RF_HEAD_DIM * 2;   // 32 KB
 constexpr int kHalfBytes = kTileBytes / 2;               // 64 columns x 128 rows
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;  // S b at 128 b; P b at 384 + 64 b
 constexpr int kPolyEvery = 4;                            // pair i uses the polynomial when i % 4 == 3
 constexpr float kRescaleThreshold = 8.0f;                // log2 units
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -65,20 +66,20 @@ struct Item {
   int bn, qt, ntiles, pad;
 };
 
-struct __align__(1024) Smem {
+// One slot: buffers and barriers of one unit in flight.
+struct __align__(1024) Slot {
   uint8_t q[kTileBytes];
-  uint8_t k[kKStages][kTileBytes];
-  uint8_t v[kVStages][kTileBytes];
-  uint64_t q_full, q_empty;
-  uint64_t k_full[kKStages], k_empty[kKStages], v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_read[2], p_full[2], p_free[2];
-  uint64_t o_full, o_empty;
-  uint64_t drain;               // MMA issuer's last commit when it leaves early
-  uint64_t xbar[4];             // per row quadrant: rendezvous of its two softmax warps
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
+  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
+  uint64_t s_full, p_full, pv_done, o_full, o_empty;
+  uint64_t drain;               // the issuer's last commit when it leaves early
   uint64_t item_full[2], item_empty[2];
   Item items[2];
-  float xmax[2][2][RF_BLOCK];   // [tile parity][column half][row] partial row maxima
-  float xsum[2][RF_BLOCK];      // [column half][row] partial row sums at the end of a unit
+};
+
+struct Smem {
+  Slot slot[kSlots];
   uint32_t tmem_base;
   int abort;
 };
@@ -111,16 +112,21 @@ __device__ __forceinline__ bool wait1(Smem& sm, const AttnParams& p, uint64_t* b
 __device__ __forceinline__ bool waitw(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
   return __all_sync(0xFFFFFFFFu, wait1(sm, p, bar, parity));
 }
+// One arrival per warp, after every lane's preceding work (callers fence first).
+__device__ __forceinline__ void arrive_w(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
 // Parity of completion number n (0-based) of a barrier phase.
 __device__ __forceinline__ uint32_t ph(uint32_t n) { return n & 1u; }
 
-// Rendezvous of the two softmax warps that share a row quadrant, on an
-// mbarrier (bounded wait, so a warp that leaves on an abort cannot strand its
-// partner).  Orders each thread's earlier shared-memory writes before the
-// partner's later reads.
-__device__ __forceinline__ bool pair_sync(Smem& sm, const AttnParams& p, int quad, uint32_t& phase) {
-  mbar_arrive(&sm.xbar[quad]);
-  return waitw(sm, p, &sm.xbar[quad], ph(phase++));
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ---------------------------------------------------------------- producer
@@ -160,37 +166,20 @@ struct KvIter {
   }
 };
 
-__device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
+// Producer of one slot: takes units from the global counter, loads Q and then
+// the K and V tiles of the KV list (one buffer each; K of the next tile as
+// soon as the previous S = Q K^T is done, V as soon as the previous P V is).
+__device__ void producer_loop(Smem& sm, Slot& sl, const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                               const CUtensorMap* tv) {
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
-  uint32_t c = 0, gk = 0, gv = 0;   // units, K tiles and V tiles issued
+  uint32_t c = 0, nk = 0, nv = 0;   // units, K tiles and V tiles issued
   const int S_int = p.g.S_int;
   bool ok = true;
-
-  auto load_k = [&](int row) -> bool {
-    const uint32_t st = gk % kKStages, use = gk / kKStages;
-    if (use > 0 && !wait1(sm, p, &sm.k_empty[st], ph(use - 1))) return false;
-    mbar_arrive_expect_tx(&sm.k_full[st], kTileBytes);
-    tma_load_2d(sm.k[st], tk, &sm.k_full[st], 0, row, pol_kv);
-    tma_load_2d(sm.k[st] + kHalfBytes, tk, &sm.k_full[st], 64, row, pol_kv);
-    ++gk;
-    return true;
-  };
-  auto load_v = [&](int row) -> bool {
-    const uint32_t st = gv % kVStages, use = gv / kVStages;
-    if (use > 0 && !wait1(sm, p, &sm.v_empty[st], ph(use - 1))) return false;
-    mbar_arrive_expect_tx(&sm.v_full[st], kTileBytes);
-    tma_load_2d(sm.v[st], tv, &sm.v_full[st], 0, row, pol_kv);
-    tma_load_2d(sm.v[st] + kHalfBytes, tv, &sm.v_full[st], 64, row, pol_kv);
-    ++gv;
-    return true;
-  };
-
   while (ok) {
     const int w = atomicAdd(p.counter, 1);
-    const uint32_t slot = c & 1;
-    if (c >= 2 && !wait1(sm, p, &sm.item_empty[slot], ph((c >> 1) - 1))) {
+    const uint32_t it = c & 1;
+    if (c >= 2 && !wait1(sm, p, &sl.item_empty[it], ph((c >> 1) - 1))) {
       ok = false;
       break;
     }
@@ -208,53 +197,49 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
         itm.ntiles = p.n_ptiles + cnt;
       }
     }
-    sm.items[slot] = itm;
-    mbar_arrive(&sm.item_full[slot]);
+    sl.items[it] = itm;
+    mbar_arrive(&sl.item_full[it]);
     if (itm.bn < 0) break;
 
     const int base = itm.bn * S_int;
-    if (c >= 1 && !wait1(sm, p, &sm.q_empty, ph(c - 1))) {
+    if (c >= 1 && !wait1(sm, p, &sl.q_empty, ph(c - 1))) {
       ok = false;
       break;
     }
     if (!(p.skip_first_q && c == 0)) {
-      mbar_arrive_expect_tx(&sm.q_full, kTileBytes);
-      tma_load_2d(sm.q, tq, &sm.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
-      tma_load_2d(sm.q + kHalfBytes, tq, &sm.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
+      mbar_arrive_expect_tx(&sl.q_full, kTileBytes);
+      tma_load_2d(sl.q, tq, &sl.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
+      tma_load_2d(sl.q + kHalfBytes, tq, &sl.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
     }
     ++c;
-
-    // K runs kKAhead tiles ahead of V: K0, K1, K2, V0, K3, V1, ..., V(n-1).
-    KvIter kit, vit;
+    KvIter kit;
     kit.init(base, p, mrow);
-    vit.init(base, p, mrow);
-    for (int i = 0; i < kKAhead && ok; ++i) {
-      const int rk = kit.next();
-      if (rk < 0) break;
-      ok = load_k(rk);
-    }
-    while (ok) {
-      const int rk = kit.next();
-      if (rk >= 0) ok = load_k(rk);
-      if (!ok) break;
-      const int rv = vit.next();
-      if (rv < 0) break;
-      ok = load_v(rv);
+    for (int row = kit.next(); row >= 0 && ok; row = kit.next()) {
+      if (nk >= 1 && !wait1(sm, p, &sl.k_empty, ph(nk - 1))) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&sl.k_full, kTileBytes);
+      tma_load_2d(sl.k, tk, &sl.k_full, 0, row, pol_kv);
+      tma_load_2d(sl.k + kHalfBytes, tk, &sl.k_full, 64, row, pol_kv);
+      ++nk;
+      if (nv >= 1 && !wait1(sm, p, &sl.v_empty, ph(nv - 1))) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&sl.v_full, kTileBytes);
+      tma_load_2d(sl.v, tv, &sl.v_full, 0, row, pol_kv);
+      tma_load_2d(sl.v + kHalfBytes, tv, &sl.v_full, 64, row, pol_kv);
+      ++nv;
     }
   }
   if (!ok) {
     // Let the copies already issued land before the CTA may exit (bounded by
     // time, not cut short by the abort flag).
     const uint64_t lim = p.wait_limit_ns / 4;
-    if (c) rf_wait_time(&sm.q_full, ph(c - 1), lim);
-    for (uint32_t st = 0; st < kKStages; ++st) {
-      const uint32_t nk = (gk > st) ? (gk - st + kKStages - 1) / kKStages : 0;
-      if (nk) rf_wait_time(&sm.k_full[st], ph(nk - 1), lim);
-    }
-    for (uint32_t st = 0; st < kVStages; ++st) {
-      const uint32_t nv = (gv > st) ? (gv - st + kVStages - 1) / kVStages : 0;
-      if (nv) rf_wait_time(&sm.v_full[st], ph(nv - 1), lim);
-    }
+    if (c) rf_wait_time(&sl.q_full, ph(c - 1), lim);
+    if (nk) rf_wait_time(&sl.k_full, ph(nk - 1), lim);
+    if (nv) rf_wait_time(&sl.v_full, ph(nv - 1), lim);
   }
 }
 
@@ -263,12 +248,13 @@ __device__ void producer_loop(Smem& sm, const AttnParams& p, const CUtensorMap* 
 // used here shares one high word (stride 1024 B, sm_100 version, swizzle).
 // A K step of 16 elements advances a K-major operand by 32 B (2 in the
 // descriptor's 16-byte units), and the second 64-column half by 16 KB.
+// A whole warp runs the issuer; one elected lane issues each instruction.
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
   constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    mma_ss_lo(s_tmem, q_lo + off, k_lo + off, hi, idesc, kk > 0);
+    mma_ss_lo_elect(s_tmem, q_lo + off, k_lo + off, hi, idesc, kk > 0);
   }
 }
 // V is MN-major: a K step of 16 keys advances it by 16 rows of 128 B.
@@ -277,123 +263,100 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
   constexpr uint32_t idesc = make_idesc_bf16(128, 128, true);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    mma_ts_lo(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-__device__ bool mma_loop_body(Smem& sm, const AttnParams& p, uint32_t tmem) {
-  uint32_t c = 0, g = 0;   // units and KV tiles consumed
+// Issuer of one slot: S = Q K^T of a tile once the P V of the previous tile
+// (whose P lives in the S columns) is done, then its P V once the softmax
+// has written P.
+__device__ bool mma_loop_body(Smem& sm, Slot& sl, const AttnParams& p, uint32_t s_tmem, uint32_t o_tmem) {
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
-  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sm.q), 16, 1024);
-  const uint32_t k_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
-  const uint32_t v_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.v[0]), kHalfBytes, 1024);
-  // S of tile t into buffer t % 2: needs K tile t and S of tile t-2 read by the softmax.
-  auto qk = [&](uint32_t t) -> bool {
-    const uint32_t st = t % kKStages, sb = t & 1;
-    if (!wait1(sm, p, &sm.k_full[st], ph(t / kKStages))) return false;
-    if (t >= 2 && !wait1(sm, p, &sm.s_read[sb], ph((t >> 1) - 1))) return false;
-    tc_fence_after();
-    issue_qk(tmem + kColS + 128 * sb, q_lo, k_lo0 + st * (kTileBytes >> 4), hi);
-    mma_commit(&sm.s_full[sb]);
-    mma_commit(&sm.k_empty[st]);
-    return true;
-  };
-  for (;;) {
-    const uint32_t slot = c & 1;
-    if (!wait1(sm, p, &sm.item_full[slot], ph(c >> 1))) return false;
-    const Item itm = sm.items[slot];
-    mbar_arrive(&sm.item_empty[slot]);
+  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.q), 16, 1024);
+  const uint32_t k_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.k), 16, 1024);
+  const uint32_t v_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.v), kHalfBytes, 1024);
+  uint32_t c = 0, t = 0;   // units and tiles of this slot
+  for (;; ++c) {
+    const uint32_t it = c & 1;
+    if (!waitw(sm, p, &sl.item_full[it], ph(c >> 1))) return false;
+    const Item itm = sl.items[it];
+    arrive_w(&sl.item_empty[it]);
     if (itm.bn < 0) return true;
-    const uint32_t n = itm.ntiles;
-    if (!wait1(sm, p, &sm.q_full, ph(c))) return false;
-    if (!qk(g)) return false;
-    if (n == 1) mma_commit(&sm.q_empty);
-    for (uint32_t j = 0; j < n; ++j) {
-      const uint32_t t = g + j, pb = t & 1, vs = t % kVStages;
-      if (j + 1 < n) {
-        if (!qk(t + 1)) return false;
-        if (j + 2 == n) mma_commit(&sm.q_empty);
-      }
-      if (!wait1(sm, p, &sm.p_full[pb], ph(t >> 1))) return false;
-      if (!wait1(sm, p, &sm.v_full[vs], ph(t / kVStages))) return false;
-      // the epilogue of the previous unit must have read O
-      if (j == 0 && c >= 1 && !wait1(sm, p, &sm.o_empty, ph(c - 1))) return false;
+    if (!waitw(sm, p, &sl.q_full, ph(c))) return false;
+    for (int j = 0; j < itm.ntiles; ++j, ++t) {
+      if (!waitw(sm, p, &sl.k_full, ph(t))) return false;
+      if (t >= 1 && !waitw(sm, p, &sl.pv_done, ph(t - 1))) return false;
       tc_fence_after();
-      issue_pv(tmem + kColO, tmem + kColP + 64 * pb, v_lo0 + vs * (kTileBytes >> 4), hi, j > 0);
-      mma_commit(&sm.p_free[pb]);
-      mma_commit(&sm.v_empty[vs]);
-      if (j + 1 == n) mma_commit(&sm.o_full);
+      issue_qk(s_tmem, q_lo, k_lo, hi);
+      mma_commit_elect(&sl.s_full);
+      mma_commit_elect(&sl.k_empty);
+      if (j + 1 == itm.ntiles) mma_commit_elect(&sl.q_empty);
+      if (!waitw(sm, p, &sl.p_full, ph(t))) return false;
+      if (!waitw(sm, p, &sl.v_full, ph(t))) return false;
+      // the previous unit's epilogue must have read O
+      if (j == 0 && c >= 1 && !waitw(sm, p, &sl.o_empty, ph(c - 1))) return false;
+      tc_fence_after();
+      issue_pv(o_tmem, s_tmem, v_lo, hi, j > 0);
+      mma_commit_elect(&sl.pv_done);
+      mma_commit_elect(&sl.v_empty);
+      if (j + 1 == itm.ntiles) mma_commit_elect(&sl.o_full);
     }
-    g += n;
-    ++c;
   }
 }
 
 // Leaves after the last unit, or early on an abort; in the latter case the
 // MMAs already issued must finish before tensor memory is freed.
-__device__ void mma_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
-  if (!mma_loop_body(sm, p, tmem)) {
-    mma_commit(&sm.drain);
-    rf_wait_time(&sm.drain, 0, p.wait_limit_ns / 4);
+__device__ void mma_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t s_tmem, uint32_t o_tmem) {
+  if (!mma_loop_body(sm, sl, p, s_tmem, o_tmem)) {
+    mma_commit_elect(&sl.drain);
+    rf_wait_time(&sl.drain, 0, p.wait_limit_ns / 4);
+    __syncwarp();
   }
 }
 
 // ---------------------------------------------------------------- softmax + epilogue
-__device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
-  const int warp = threadIdx.x >> 5;           // 0..7
-  const int quad = warp & 3, half = warp >> 2;
+__device__ void softmax_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem_slot) {
+  const int quad = (threadIdx.x >> 5) & 3;
   const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
-  const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-  const uint32_t tO = lane_base + kColO + 64 * half;
-  const int col0 = 64 * half;                  // first key column of this thread
+  const uint32_t lane_base = tmem_slot + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tS = lane_base, tO = lane_base + 128;
   const float sl2 = p.scale_log2;
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
-  uint32_t c = 0, g = 0, xph = 0;
+  uint32_t c = 0, t = 0;   // units and tiles of this slot
   for (;;) {
-    const uint32_t slot = c & 1;
-    if (!waitw(sm, p, &sm.item_full[slot], ph(c >> 1))) return;
-    const Item itm = sm.items[slot];
-    mbar_arrive(&sm.item_empty[slot]);
+    const uint32_t it = c & 1;
+    if (!waitw(sm, p, &sl.item_full[it], ph(c >> 1))) return;
+    const Item itm = sl.items[it];
+    arrive_w(&sl.item_empty[it]);
     if (itm.bn < 0) return;
 
     float m_use = -CUDART_INF_F, l = 0.f;
-    for (int j = 0; j < itm.ntiles; ++j) {
-      const uint32_t t = g + j, sb = t & 1;
-      const uint32_t tS = lane_base + kColS + 128 * sb + col0;
-      const uint32_t tP = lane_base + kColP + 64 * sb + 32 * half;
-      if (!waitw(sm, p, &sm.s_full[sb], ph(t >> 1))) return;
+    for (int j = 0; j < itm.ntiles; ++j, ++t) {
+      if (!waitw(sm, p, &sl.s_full, ph(t))) return;
       tc_fence_after();
-      uint32_t s[2][32];
-      tmem_ld32(tS, s[0]);
-      tmem_ld32(tS + 32, s[1]);
+      uint32_t s[4][32];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
       tmem_wait_ld();
-      reg_fence32(s[0]);
-      reg_fence32(s[1]);
-      // S is in registers: the tensor pipe may overwrite this buffer.
-      tc_fence_before();
-      mbar_arrive(&sm.s_read[sb]);
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
 
       const bool partial = (p.p_rem != 0 && j == p.n_ptiles - 1);
       if (partial) {
 #pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2)
+        for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (col0 + 32 * q2 + e >= p.p_rem) s[q2][e] = __float_as_uint(-CUDART_INF_F);
+            if (32 * q4 + e >= p.p_rem) s[q4][e] = __float_as_uint(-CUDART_INF_F);
       }
-      // row max over this half: 8 independent chains of 3-input max
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2)
+      for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
-          mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q2][e]), __uint_as_float(s[q2][e + 1]));
-      const float mxh = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-      // combine with the other half of the row
-      sm.xmax[sb][half][row] = mxh;
-      if (!pair_sync(sm, p, quad, xph)) return;
-      const float mx = fmaxf(mxh, sm.xmax[sb][half ^ 1][row]);
+          mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
+      const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
       const float mx_s = mx * sl2;
       float alpha = 1.f;
       bool rescale = false;
@@ -404,16 +367,15 @@ __device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
         m_use = mx_s;
         rescale = true;
       }
-      // p = 2^(s * scale * log2 e - m): pairs, packed fp32 arithmetic
       const uint64_t negm = f2_pack(-m_use, -m_use);
       uint64_t sum2[4] = {0, 0, 0, 0};
-      uint32_t pk[32];
+      uint32_t pk[64];
 #pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2)
+      for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const int i = 16 * q2 + (e >> 1);     // pair index 0..31 within this half
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q2][e]), __uint_as_float(s[q2][e + 1])), sl2x2, negm);
+          const int i = 16 * q4 + (e >> 1);     // pair index 0..63
+          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), sl2x2, negm);
           uint64_t p2;
           if ((i % kPolyEvery) == kPolyEvery - 1) {
             p2 = exp2_poly_x2(x2);
@@ -425,8 +387,7 @@ __device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
           if (partial) {
             float a0, a1;
             f2_unpack(p2, a0, a1);
-            const int k0 = col0 + 2 * i;
-            p2 = f2_pack(k0 < p.p_rem ? a0 : 0.f, k0 + 1 < p.p_rem ? a1 : 0.f);
+            p2 = f2_pack(2 * i < p.p_rem ? a0 : 0.f, 2 * i + 1 < p.p_rem ? a1 : 0.f);
           }
           sum2[i & 3] = f2_add(sum2[i & 3], p2);
           float a0, a1;
@@ -438,61 +399,53 @@ __device__ void softmax_loop(Smem& sm, const AttnParams& p, uint32_t tmem) {
       f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
       l = l * alpha + ((s0 + s1) + (s2 + s3));
       if (__any_sync(0xFFFFFFFFu, rescale)) {
-        // O holds the tiles before j once the P*V of tile j-1 is done.
-        if (!waitw(sm, p, &sm.p_free[(t - 1) & 1], ph((t - 1) >> 1))) return;
-        tc_fence_after();
+        // O holds the tiles before j: their P V completed before this tile's
+        // S was computed (the issuer waits for it).
 #pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {
+        for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t o[32];
-          tmem_ld32(tO + 32 * q2, o);
+          tmem_ld32(tO + 32 * q4, o);
           tmem_wait_ld();
           reg_fence32(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * q2, o);
+          tmem_st32(tO + 32 * q4, o);
         }
       }
-      // P buffer sb is free once the P*V of tile t-2 is done
-      if (t >= 2 && !waitw(sm, p, &sm.p_free[sb], ph((t >> 1) - 1))) return;
-      tc_fence_after();
-      tmem_st32(tP, pk);
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&sm.p_full[sb]);
+      arrive_w(&sl.p_full);
     }
-    // epilogue: O / l of this unit once its last P*V is done
-    if (!waitw(sm, p, &sm.o_full, ph(c))) return;
+    // epilogue: O / l of this unit once its last P V is done
+    if (!waitw(sm, p, &sl.o_full, ph(c))) return;
     tc_fence_after();
-    uint32_t o[2][32];
-    tmem_ld32(tO, o[0]);
-    tmem_ld32(tO + 32, o[1]);
-    tmem_wait_ld();
-    reg_fence32(o[0]);
-    reg_fence32(o[1]);
-    // O is in registers: the next unit may start accumulating.
-    tc_fence_before();
-    mbar_arrive(&sm.o_empty);
-    // xsum is rewritten only at the end of the next unit, after at least one
-    // more rendezvous, so one rendezvous here is enough.
-    sm.xsum[half][row] = l;
-    if (!pair_sync(sm, p, quad, xph)) return;
-    const float rl = 1.f / (sm.xsum[0][row] + sm.xsum[1][row]);
-    const int b = itm.bn / p.N, n = itm.bn - b * p.N;
+    const float rl = 1.f / l;
+    const int b = itm.bn / p.N, nh = itm.bn - b * p.N;
     const int src = rf_src_of_row(p.g, itm.qt * RF_BLOCK + row);
-    if (src >= 0) {
-      __nv_bfloat16* dst = p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, n, src) + col0;
-#pragma unroll
-      for (int q2 = 0; q2 < 2; ++q2) {
+    __nv_bfloat16* dst = src >= 0 ? p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, nh, src) : nullptr;
+#pragma unroll 1
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * q4, o);
+      tmem_wait_ld();
+      reg_fence32(o);
+      if (q4 == 3) {
+        // O is in registers: the next unit may start accumulating.
+        tc_fence_before();
+        arrive_w(&sl.o_empty);
+      }
+      if (dst) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[q2][2 * e]) * rl, __uint_as_float(o[q2][2 * e + 1]) * rl);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q2);
+          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q4);
 #pragma unroll
         for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
-    g += itm.ntiles;
     ++c;
   }
 }
@@ -505,28 +458,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_read[i], kSoftmaxThreads);
-      mbar_init(&sm.p_full[i], kSoftmaxThreads);
-      mbar_init(&sm.p_free[i], 1);
-      mbar_init(&sm.item_full[i], 1);
-      mbar_init(&sm.item_empty[i], kSoftmaxThreads + 1);
+    for (int z = 0; z < kSlots; ++z) {
+      Slot& sl = sm.slot[z];
+      mbar_init(&sl.q_full, 1);
+      mbar_init(&sl.q_empty, 1);
+      mbar_init(&sl.k_full, 1);
+      mbar_init(&sl.k_empty, 1);
+      mbar_init(&sl.v_full, 1);
+      mbar_init(&sl.v_empty, 1);
+      mbar_init(&sl.s_full, 1);
+      mbar_init(&sl.p_full, kSlotWarps);
+      mbar_init(&sl.pv_done, 1);
+      mbar_init(&sl.o_full, 1);
+      mbar_init(&sl.o_empty, kSlotWarps);
+      mbar_init(&sl.drain, 1);
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&sl.item_full[i], 1);
+        mbar_init(&sl.item_empty[i], kSlotWarps + 1);   // softmax warps + issuer warp
+      }
     }
-    for (int i = 0; i < kKStages; ++i) {
-      mbar_init(&sm.k_full[i], 1);
-      mbar_init(&sm.k_empty[i], 1);
-    }
-    for (int i = 0; i < kVStages; ++i) {
-      mbar_init(&sm.v_full[i], 1);
-      mbar_init(&sm.v_empty[i], 1);
-    }
-    mbar_init(&sm.o_full, 1);
-    mbar_init(&sm.drain, 1);
-    mbar_init(&sm.o_empty, kSoftmaxThreads);
-    for (int i = 0; i < 4; ++i) mbar_init(&sm.xbar[i], 64);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -535,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
   }
-  if (warp == 9) {
+  if (warp == 10) {
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -545,17 +495,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   if (warp < 8) {
-    softmax_loop(sm, p, tmem);
-  } else if (warp == 8) {
-    if (lane == 0) producer_loop(sm, p, &tm_q, &tm_k, &tm_v);
+    regs_increase<kRegsSoftmax>();
+    const int z = warp >> 2;
+    softmax_loop(sm, sm.slot[z], p, tmem + 256 * z);
   } else {
-    if (lane == 0) mma_loop(sm, p, tmem);
+    regs_decrease<kRegsControl>();
+    if (warp == 8 && lane == 0) producer_loop(sm, sm.slot[0], p, &tm_q, &tm_k, &tm_v);
+    if (warp == 9 && lane == 0) producer_loop(sm, sm.slot[1], p, &tm_q, &tm_k, &tm_v);
+    if (warp >= 10) {
+      const int z = warp - 10;
+      mma_loop(sm, sm.slot[z], p, tmem + 256 * z, tmem + 256 * z + 128);
+    }
   }
   __syncwarp();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 10) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------- host side
