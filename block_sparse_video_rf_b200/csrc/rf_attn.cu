@@ -17,24 +17,26 @@
 // Q/K/V shared-memory buffers, its own S and O in tensor memory and its own
 // warps, so that while the softmax of one slot runs the tensor pipe works on
 // the other slot's MMAs:
-//   warps 0-3   softmax of slot 0, warps 4-7 of slot 1: thread = query row
-//               (TMEM lane); online softmax in exp2 with a lazily updated
-//               running max; most exponentials on the MUFU unit, one pair in
-//               four on the FMA pipe (polynomial); P (bf16) is written over
-//               the first 64 columns of the slot's S; at the end of a unit
-//               the same threads write O / l -> bf16 -> the caller's layout.
+//   warps 0-3   slot 0, warps 4-7 slot 1: thread = query row (TMEM lane);
+//               online softmax in exp2 with a lazily updated running max;
+//               most exponentials on the MUFU unit, one pair in four on the
+//               FMA pipe (polynomial); P (bf16) is written over the first 64
+//               columns of the slot's S; at the end of a unit the same
+//               threads write O / l -> bf16 -> the caller's layout.  The
+//               slot's first warp also issues its MMAs (one elected lane):
+//               S = Q K^T: tcgen05 kind::f16, A and B from shared memory;
+//               O += P V:  A = P from tensor memory, B = V MN-major.
+//               The four warps meet at a named barrier after each tile, so
+//               P V follows P without an mbarrier hand-off.
 //   warps 8, 9  TMA producers of slot 0 and slot 1 (one thread each): Q, then
 //               the K and V tiles of the KV list, 128-byte swizzled boxes of
 //               128 rows x 64 columns.
-//   warps 10, 11 MMA issuers of slot 0 and slot 1 (one elected lane issues);
-//               warp 10 also owns the tensor memory.
-//               S = Q K^T: tcgen05 kind::f16, A and B from shared memory;
-//               O += P V:  A = P from tensor memory, B = V MN-major.
+//   warp 10     owns the tensor memory; warps 10 and 11 are otherwise idle.
 // Tensor memory (512 columns): slot z has S at [256 z, 256 z + 128) (P in
 // its first 64 columns) and O at [256 z + 128, 256 z + 256).  Since P
 // overwrites S, the QK of a slot's next tile is issued once its P V is done.
 // Registers: the control warpgroup (warps 8-11) gives registers to the two
-// softmax warpgroups (setmaxnreg 64 / 216: 8 x 32 x 216 + 4 x 32 x 64 =
+// slot warpgroups (setmaxnreg 64 / 216: 8 x 32 x 216 + 4 x 32 x 64 =
 // 63,488 <= 384 threads x 168 at launch).
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -72,7 +74,7 @@ struct __align__(1024) Slot {
   uint8_t k[kTileBytes];
   uint8_t v[kTileBytes];
   uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
-  uint64_t s_full, p_full, pv_done, o_full, o_empty;
+  uint64_t s_full, pv_done;
   uint64_t drain;               // the issuer's last commit when it leaves early
   uint64_t item_full[2], item_empty[2];
   Item items[2];
@@ -243,12 +245,12 @@ __device__ void producer_loop(Smem& sm, Slot& sl, const AttnParams& p, const CUt
   }
 }
 
-// ---------------------------------------------------------------- MMA issuer
+// ---------------------------------------------------------------- MMA issue
 // Descriptor low words of the 128-byte swizzled operands; every descriptor
 // used here shares one high word (stride 1024 B, sm_100 version, swizzle).
 // A K step of 16 elements advances a K-major operand by 32 B (2 in the
 // descriptor's 16-byte units), and the second 64-column half by 16 KB.
-// A whole warp runs the issuer; one elected lane issues each instruction.
+// The issuing warp runs this code together; one elected lane issues.
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
   constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
 #pragma unroll
@@ -266,187 +268,219 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint3
     mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// Issuer of one slot: S = Q K^T of a tile once the P V of the previous tile
-// (whose P lives in the S columns) is done, then its P V once the softmax
-// has written P.
-__device__ bool mma_loop_body(Smem& sm, Slot& sl, const AttnParams& p, uint32_t s_tmem, uint32_t o_tmem) {
-  const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
-  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.q), 16, 1024);
-  const uint32_t k_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.k), 16, 1024);
-  const uint32_t v_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.v), kHalfBytes, 1024);
-  uint32_t c = 0, t = 0;   // units and tiles of this slot
-  for (;; ++c) {
-    const uint32_t it = c & 1;
-    if (!waitw(sm, p, &sl.item_full[it], ph(c >> 1))) return false;
-    const Item itm = sl.items[it];
-    arrive_w(&sl.item_empty[it]);
-    if (itm.bn < 0) return true;
-    if (!waitw(sm, p, &sl.q_full, ph(c))) return false;
-    for (int j = 0; j < itm.ntiles; ++j, ++t) {
-      if (!waitw(sm, p, &sl.k_full, ph(t))) return false;
-      if (t >= 1 && !waitw(sm, p, &sl.pv_done, ph(t - 1))) return false;
-      tc_fence_after();
-      issue_qk(s_tmem, q_lo, k_lo, hi);
-      mma_commit_elect(&sl.s_full);
-      mma_commit_elect(&sl.k_empty);
-      if (j + 1 == itm.ntiles) mma_commit_elect(&sl.q_empty);
-      if (!waitw(sm, p, &sl.p_full, ph(t))) return false;
-      if (!waitw(sm, p, &sl.v_full, ph(t))) return false;
-      // the previous unit's epilogue must have read O
-      if (j == 0 && c >= 1 && !waitw(sm, p, &sl.o_empty, ph(c - 1))) return false;
-      tc_fence_after();
-      issue_pv(o_tmem, s_tmem, v_lo, hi, j > 0);
-      mma_commit_elect(&sl.pv_done);
-      mma_commit_elect(&sl.v_empty);
-      if (j + 1 == itm.ntiles) mma_commit_elect(&sl.o_full);
-    }
-  }
+// Rendezvous of a slot's four warps (named barrier `id`, 128 threads) that
+// also returns whether every thread passed `ok`: the warps of a slot leave
+// together, so none is left waiting at a later rendezvous.
+__device__ __forceinline__ bool slot_vote(int id, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred a, b;\n\tsetp.ne.u32 a, %1, 0;\n\t"
+      "bar.red.and.pred b, %2, 128, a;\n\tselp.u32 %0, 1, 0, b;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(id)
+      : "memory");
+  return r != 0;
 }
 
-// Leaves after the last unit, or early on an abort; in the latter case the
-// MMAs already issued must finish before tensor memory is freed.
-__device__ void mma_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t s_tmem, uint32_t o_tmem) {
-  if (!mma_loop_body(sm, sl, p, s_tmem, o_tmem)) {
-    mma_commit_elect(&sl.drain);
-    rf_wait_time(&sl.drain, 0, p.wait_limit_ns / 4);
-    __syncwarp();
-  }
-}
-
-// ---------------------------------------------------------------- softmax + epilogue
-__device__ void softmax_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem_slot) {
-  const int quad = (threadIdx.x >> 5) & 3;
-  const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
-  const uint32_t lane_base = tmem_slot + ((uint32_t)(quad * 32) << 16);
-  const uint32_t tS = lane_base, tO = lane_base + 128;
-  const float sl2 = p.scale_log2;
+// ---------------------------------------------------------------- softmax of one tile
+// Thread = query row.  Reads the row's 128 scores from S, updates the running
+// max m_use (log2 units, lazily: only when a score exceeds it by more than
+// the threshold, then O and l are rescaled), adds the tile's sum to l and
+// writes P = 2^(s * scale * log2 e - m_use) as bf16 over the first 64
+// columns of S.  `p_valid` < 128 masks the keys past the prefix's end.
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool first, int p_valid, float sl2,
+                                             float& m_use, float& l) {
   const uint64_t sl2x2 = f2_pack(sl2, sl2);
-  uint32_t c = 0, t = 0;   // units and tiles of this slot
-  for (;;) {
-    const uint32_t it = c & 1;
-    if (!waitw(sm, p, &sl.item_full[it], ph(c >> 1))) return;
-    const Item itm = sl.items[it];
-    arrive_w(&sl.item_empty[it]);
-    if (itm.bn < 0) return;
-
-    float m_use = -CUDART_INF_F, l = 0.f;
-    for (int j = 0; j < itm.ntiles; ++j, ++t) {
-      if (!waitw(sm, p, &sl.s_full, ph(t))) return;
-      tc_fence_after();
-      uint32_t s[4][32];
+  uint32_t s[4][32];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
-      tmem_wait_ld();
+  for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
+  tmem_wait_ld();
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
+  for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
 
-      const bool partial = (p.p_rem != 0 && j == p.n_ptiles - 1);
+  const bool partial = p_valid < RF_BLOCK;
+  if (partial) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (32 * q4 + e >= p_valid) s[q4][e] = __float_as_uint(-CUDART_INF_F);
+  }
+  float mx8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+    for (int e = 0; e < 32; e += 2)
+      mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
+  const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+  const float mx_s = mx * sl2;
+  float alpha = 1.f;
+  bool rescale = false;
+  if (first) {
+    m_use = mx_s;
+  } else if (mx_s > m_use + kRescaleThreshold) {
+    alpha = ex2_approx(m_use - mx_s);
+    m_use = mx_s;
+    rescale = true;
+  }
+  const uint64_t negm = f2_pack(-m_use, -m_use);
+  uint64_t sum2[4] = {0, 0, 0, 0};
+  uint32_t pk[64];
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int i = 16 * q4 + (e >> 1);     // pair index 0..63
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), sl2x2, negm);
+      uint64_t p2;
+      if ((i % kPolyEvery) == kPolyEvery - 1) {
+        p2 = exp2_poly_x2(x2);
+      } else {
+        float x0, x1;
+        f2_unpack(x2, x0, x1);
+        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
+      }
       if (partial) {
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * q4 + e >= p.p_rem) s[q4][e] = __float_as_uint(-CUDART_INF_F);
+        float a0, a1;
+        f2_unpack(p2, a0, a1);
+        p2 = f2_pack(2 * i < p_valid ? a0 : 0.f, 2 * i + 1 < p_valid ? a1 : 0.f);
       }
-      float mx8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
-      const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-      const float mx_s = mx * sl2;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (j == 0) {
-        m_use = mx_s;
-      } else if (mx_s > m_use + kRescaleThreshold) {
-        alpha = ex2_approx(m_use - mx_s);
-        m_use = mx_s;
-        rescale = true;
-      }
-      const uint64_t negm = f2_pack(-m_use, -m_use);
-      uint64_t sum2[4] = {0, 0, 0, 0};
-      uint32_t pk[64];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int i = 16 * q4 + (e >> 1);     // pair index 0..63
-          const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), sl2x2, negm);
-          uint64_t p2;
-          if ((i % kPolyEvery) == kPolyEvery - 1) {
-            p2 = exp2_poly_x2(x2);
-          } else {
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-          }
-          if (partial) {
-            float a0, a1;
-            f2_unpack(p2, a0, a1);
-            p2 = f2_pack(2 * i < p.p_rem ? a0 : 0.f, 2 * i + 1 < p.p_rem ? a1 : 0.f);
-          }
-          sum2[i & 3] = f2_add(sum2[i & 3], p2);
-          float a0, a1;
-          f2_unpack(p2, a0, a1);
-          pk[i] = pack_bf16x2(a0, a1);
-        }
-      float s0, s1, s2, s3;
-      f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
-      f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
-      l = l * alpha + ((s0 + s1) + (s2 + s3));
-      if (__any_sync(0xFFFFFFFFu, rescale)) {
-        // O holds the tiles before j: their P V completed before this tile's
-        // S was computed (the issuer waits for it).
-#pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t o[32];
-          tmem_ld32(tO + 32 * q4, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(tO + 32 * q4, o);
-        }
-      }
-      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-      tmem_wait_st();
-      tc_fence_before();
-      arrive_w(&sl.p_full);
+      sum2[i & 3] = f2_add(sum2[i & 3], p2);
+      float a0, a1;
+      f2_unpack(p2, a0, a1);
+      pk[i] = pack_bf16x2(a0, a1);
     }
-    // epilogue: O / l of this unit once its last P V is done
-    if (!waitw(sm, p, &sl.o_full, ph(c))) return;
-    tc_fence_after();
-    const float rl = 1.f / l;
-    const int b = itm.bn / p.N, nh = itm.bn - b * p.N;
-    const int src = rf_src_of_row(p.g, itm.qt * RF_BLOCK + row);
-    __nv_bfloat16* dst = src >= 0 ? p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, nh, src) : nullptr;
+  float s0, s1, s2, s3;
+  f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
+  f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
+  l = l * alpha + ((s0 + s1) + (s2 + s3));
+  if (__any_sync(0xFFFFFFFFu, rescale)) {
+    // O holds the tiles before this one: their P V completed before this
+    // tile's S = Q K^T was issued.
 #pragma unroll 1
     for (int q4 = 0; q4 < 4; ++q4) {
       uint32_t o[32];
       tmem_ld32(tO + 32 * q4, o);
       tmem_wait_ld();
       reg_fence32(o);
-      if (q4 == 3) {
-        // O is in registers: the next unit may start accumulating.
-        tc_fence_before();
-        arrive_w(&sl.o_empty);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+      tmem_st32(tO + 32 * q4, o);
+    }
+  }
+  tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+  tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+  tmem_wait_st();
+  tc_fence_before();
+}
+
+// ---------------------------------------------------------------- one slot
+// The slot's four warps compute the softmax of each tile (thread = query row
+// = TMEM lane) and write the unit's output; the first of them also issues
+// the slot's MMAs: S = Q K^T of a tile once the P V of the previous tile is
+// done (P lives in the S columns), and P V of a tile once all four warps
+// have written P (the rendezvous after each tile).
+__device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem_slot, int bar_id) {
+  const int quad = (threadIdx.x >> 5) & 3;
+  const bool issuer = (quad == 0);
+  const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
+  const uint32_t lane_base = tmem_slot + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tS = lane_base, tO = lane_base + 128;
+  const uint32_t s_tmem = tmem_slot, o_tmem = tmem_slot + 128;
+  const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
+  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.q), 16, 1024);
+  const uint32_t k_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.k), 16, 1024);
+  const uint32_t v_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.v), kHalfBytes, 1024);
+  uint32_t c = 0, t = 0;   // units and tiles of this slot
+  bool ok = true;
+  bool issued = false;     // the issuer has MMAs that may still run
+
+  // S = Q K^T of tile t (issuer warp): K tile t must have landed and the
+  // P V of tile t-1 must be done.
+  auto qk = [&](uint32_t tt, bool last_of_unit) -> bool {
+    if (!waitw(sm, p, &sl.k_full, ph(tt))) return false;
+    if (tt >= 1 && !waitw(sm, p, &sl.pv_done, ph(tt - 1))) return false;
+    tc_fence_after();
+    issue_qk(s_tmem, q_lo, k_lo, hi);
+    mma_commit_elect(&sl.s_full);
+    mma_commit_elect(&sl.k_empty);
+    if (last_of_unit) mma_commit_elect(&sl.q_empty);
+    issued = true;
+    return true;
+  };
+
+  for (;; ++c) {
+    // Every warp of the slot reaches every rendezvous: a warp whose wait
+    // failed carries ok = false to the next one, where all four leave.
+    const uint32_t it = c & 1;
+    Item itm{-1, 0, 0, 0};
+    if (ok) ok = waitw(sm, p, &sl.item_full[it], ph(c >> 1));
+    if (ok) {
+      itm = sl.items[it];
+      arrive_w(&sl.item_empty[it]);
+    }
+    ok = slot_vote(bar_id, ok);
+    if (!ok || itm.bn < 0) break;
+    if (issuer) ok = waitw(sm, p, &sl.q_full, ph(c)) && qk(t, itm.ntiles == 1);
+
+    float m_use = -CUDART_INF_F, l = 0.f;
+    for (int j = 0; j < itm.ntiles; ++j, ++t) {
+      if (ok) ok = waitw(sm, p, &sl.s_full, ph(t));
+      if (ok) {
+        tc_fence_after();
+        const int p_valid = (p.p_rem != 0 && j == p.n_ptiles - 1) ? p.p_rem : RF_BLOCK;
+        softmax_tile(tS, tO, j == 0, p_valid, p.scale_log2, m_use, l);
       }
-      if (dst) {
-        uint32_t w[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
-        uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q4);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+      ok = slot_vote(bar_id, ok);
+      if (!ok) break;
+      if (issuer) {
+        ok = waitw(sm, p, &sl.v_full, ph(t));
+        if (ok) {
+          tc_fence_after();
+          issue_pv(o_tmem, s_tmem, v_lo, hi, j > 0);
+          mma_commit_elect(&sl.pv_done);
+          mma_commit_elect(&sl.v_empty);
+          if (j + 1 < itm.ntiles) ok = qk(t + 1, j + 2 == itm.ntiles);
+        }
       }
     }
-    ++c;
+    // epilogue: O / l of this unit once its last P V is done
+    if (ok) ok = waitw(sm, p, &sl.pv_done, ph(t - 1));
+    if (ok) {
+      tc_fence_after();
+      const float rl = 1.f / l;
+      const int b = itm.bn / p.N, nh = itm.bn - b * p.N;
+      const int src = rf_src_of_row(p.g, itm.qt * RF_BLOCK + row);
+      __nv_bfloat16* dst = src >= 0 ? p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, nh, src) : nullptr;
+#pragma unroll 1
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * q4, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (dst) {
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q4);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      // The next unit's first P V overwrites O only after the rendezvous
+      // that follows its first softmax tile, which ends with this fence.
+      tc_fence_before();
+    }
+  }
+  // Leaving early on an abort: the MMAs already issued must finish before
+  // tensor memory is freed.
+  if (!ok && issuer && issued) {
+    mma_commit_elect(&sl.drain);
+    rf_wait_time(&sl.drain, 0, p.wait_limit_ns / 4);
+    __syncwarp();
   }
 }
 
@@ -467,14 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sl.v_full, 1);
       mbar_init(&sl.v_empty, 1);
       mbar_init(&sl.s_full, 1);
-      mbar_init(&sl.p_full, kSlotWarps);
       mbar_init(&sl.pv_done, 1);
-      mbar_init(&sl.o_full, 1);
-      mbar_init(&sl.o_empty, kSlotWarps);
       mbar_init(&sl.drain, 1);
       for (int i = 0; i < 2; ++i) {
         mbar_init(&sl.item_full[i], 1);
-        mbar_init(&sl.item_empty[i], kSlotWarps + 1);   // softmax warps + issuer warp
+        mbar_init(&sl.item_empty[i], kSlotWarps);
       }
     }
     sm.abort = 0;
@@ -497,15 +528,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     const int z = warp >> 2;
-    softmax_loop(sm, sm.slot[z], p, tmem + 256 * z);
+    slot_loop(sm, sm.slot[z], p, tmem + 256 * z, 1 + z);
   } else {
     regs_decrease<kRegsControl>();
     if (warp == 8 && lane == 0) producer_loop(sm, sm.slot[0], p, &tm_q, &tm_k, &tm_v);
     if (warp == 9 && lane == 0) producer_loop(sm, sm.slot[1], p, &tm_q, &tm_k, &tm_v);
-    if (warp >= 10) {
-      const int z = warp - 10;
-      mma_loop(sm, sm.slot[z], p, tmem + 256 * z, tmem + 256 * z + 128);
-    }
   }
   __syncwarp();
   tc_fence_before();
