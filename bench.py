@@ -1,6 +1,7 @@
 """Benchmark of the rf_v2 block-sparse attention call on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload minimax] [--impl reference]
+                    [--sparsity S] [--dtype bf16|f16] [--precision native|fp8]
 
 One step = one full call (token reorder + pooling, block scores + top-k mask,
 block-sparse attention with the inverse reorder fused) on one batch of seeded
@@ -14,6 +15,11 @@ slowest rank's time.
 
 ``--impl reference`` times the plain CPU oracle on the host cores instead, on
 a bounded sample of the same workload.
+
+``--dtype f16`` runs fp16 inputs and output; ``--precision fp8`` runs the
+attention's two products on e4m3 operands (quantised in the first stage) and
+takes the fp8 tensor peak as twice the measured bf16 one (the nominal
+ratio).
 """
 
 from __future__ import annotations
@@ -62,10 +68,11 @@ def _k3_traffic(heads: int):
     return None
 
 
-def _describe(w) -> str:
+def _describe(w, dtype="bf16", precision="native") -> str:
     t, h, wd = w.latent
+    prec = "" if precision == "native" else f", {precision} e4m3 attention operands"
     return (f"{w.name}: B={w.B}, {w.N} heads, D={w.D}, txt_len={w.txt_len}, latent ({t},{h},{wd}) -> S={w.S}, "
-            f"sparsity {w.sparsity}, {w.layout}, bf16 synthetic ({w.kind})")
+            f"sparsity {w.sparsity}, {w.layout}, {dtype} synthetic ({w.kind}){prec}")
 
 
 # ---------------------------------------------------------------- clocks
@@ -213,6 +220,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=6.0, help="seconds of oracle work per reference step")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"])
+    ap.add_argument("--precision", default="native", choices=["native", "fp8"])
     args = ap.parse_args()
 
     from block_sparse_video_rf_b200 import synth
@@ -235,21 +244,24 @@ def main():
 
     from block_sparse_video_rf_b200 import rfsa
     dev = torch.device("cuda", local)
-    q, k, v = synth.make_inputs(w, device=dev)
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    prec = args.precision
+    default_mode = args.dtype == "bf16" and prec == "native"
+    q, k, v = synth.make_inputs(w, device=dev, dtype=tdtype)
     out = torch.empty_like(q)
     sp = np.float32(w.sparsity)
-    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent, device=dev)
+    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent, device=dev, precision=prec)
     plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, sp)
-    views = rfsa.workspace_views(ws, w.B, w.N, plan)
+    views = rfsa.workspace_views(ws, w.B, w.N, plan, dtype=tdtype, precision=prec)
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
-        rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws)
+        rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws, precision=prec)
         if ev is not None:
             ev[1].record(stream)
-        rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws)
+        rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws, precision=prec)
         if ev is not None:
             ev[2].record(stream)
 
@@ -285,14 +297,24 @@ def main():
     e2e_steps = args.e2e_steps if args.e2e_steps is not None else min(args.steps, 10)
     qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
     oh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
-    rfsa.rf_sparse_attention_host(qh, kh, vh, w.layout, w.txt_len, w.latent, sp, oh)   # warm the caches
+
+    def e2e_call():
+        if default_mode:     # the library's own host-buffer entry point
+            rfsa.rf_sparse_attention_host(qh, kh, vh, w.layout, w.txt_len, w.latent, sp, oh)
+        else:                # host copies around the device call
+            qd, kd, vd = (t.to(dev, non_blocking=True) for t in (qh, kh, vh))
+            od = rfsa.rf_sparse_attention(qd, kd, vd, w.layout, w.txt_len, w.latent, sp, precision=prec)
+            oh.copy_(od, non_blocking=True)
+            torch.cuda.current_stream(dev).synchronize()
+
+    e2e_call()   # warm the caches
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
     for _ in range(e2e_steps):
-        rfsa.rf_sparse_attention_host(qh, kh, vh, w.layout, w.txt_len, w.latent, sp, oh)
+        e2e_call()
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / max(e2e_steps, 1)
@@ -306,21 +328,28 @@ def main():
     if rank == 0:
         peaks, src = _peaks()
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        peak_note = f"{src} bf16_tflops_sustained"
+        if prec == "fp8":
+            peak *= 2.0           # nominal dense fp8 / bf16 ratio: 4.5 / 2.25 PFLOP/s
+            peak_note += " x 2 (nominal fp8 / bf16 ratio)"
+        elif args.dtype == "f16":
+            peak_note += " (fp16 and bf16 have the same nominal peak)"
         k3_tflops = flops / (k3_ms * 1e-3) / 1e12
         tensor_bytes = q.numel() * q.element_size()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": _describe(w), "l2": "inputs larger than L2 (no flush)",
+            "vs_baseline": None, "dtype": args.dtype if prec == "native" else f"e4m3 ({args.dtype} in/out)",
+            "data": "synthetic",
+            "config": {"workload": _describe(w, args.dtype, prec), "l2": "inputs larger than L2 (no flush)",
                        "kept_block_tflop_per_call": flops / 1e12, "k": plan.k, "nb": plan.nb, "ff": plan.ff,
                        "P": plan.P, "ms_prepare": statistics.mean(k1k2), "ms_attention": k3_ms},
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
             "roofline": {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": k3_tflops / peak, "traffic": _k3_traffic(w.N),
-                         "peak_source": f"{src} bf16_tflops_sustained"},
-            "gpu_launches": 3 * args.steps,
+                         "unit": "TFLOP/s", "frac": k3_tflops / peak,
+                         "traffic": _k3_traffic(w.N) if default_mode else None, "peak_source": peak_note},
+            "gpu_launches": (4 if prec == "fp8" else 3) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -65,6 +65,13 @@ rf_status_t check_common(rf_layout_t layout, int B, int S, int N, int D) {
   return RF_OK;
 }
 
+rf_status_t check_types(rf_dtype_t dtype, rf_precision_t precision) {
+  if (dtype != RF_BF16 && dtype != RF_F16) return fail(RF_ERR_ARG, "dtype must be RF_BF16 (0) or RF_F16 (1)");
+  if (precision != RF_PREC_NATIVE && precision != RF_PREC_FP8)
+    return fail(RF_ERR_ARG, "precision must be RF_PREC_NATIVE (0) or RF_PREC_FP8 (1)");
+  return RF_OK;
+}
+
 rf_status_t check_ws(void* ws, size_t ws_bytes, const rf_ws_layout_t& lay) {
   if (!ws) return fail(RF_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(RF_ERR_WORKSPACE, "workspace must be 256-byte aligned");
@@ -163,8 +170,10 @@ rf_status_t rf_plan(int S, int txt_len, int T, int H, int W, int block_size, flo
   return ok();
 }
 
-rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* g, rf_ws_layout_t* lay) {
+rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D, const rf_plan_t* g,
+                                   rf_ws_layout_t* lay) {
   if (!g || !lay) return fail(RF_ERR_ARG, "NULL plan or layout");
+  if (precision != RF_PREC_NATIVE && precision != RF_PREC_FP8) return fail(RF_ERR_ARG, "unknown precision %d", (int)precision);
   if (B <= 0 || N <= 0) return fail(RF_ERR_ARG, "B and N must be positive");
   if (D != RF_HEAD_DIM) return fail(RF_ERR_UNSUPPORTED, "head dim must be 128 (got %d)", D);
   const size_t heads = (size_t)B * N;
@@ -188,86 +197,141 @@ rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* g, rf_ws_l
   L.margin = take(rows * 4);
   L.counter = take(4);
   L.status = take(4);
+  const bool fp8 = precision == RF_PREC_FP8;
+  L.q8 = take(fp8 ? tensor / 2 : 0);
+  L.k8 = take(fp8 ? tensor / 2 : 0);
+  L.v8 = take(fp8 ? tensor / 2 : 0);
+  L.scales = take(fp8 ? 3 * heads * g->n_tiles * 4 : 0);
+  L.vmax = take(fp8 ? heads * 4 : 0);
   L.total = off;
   *lay = L;
   return ok();
 }
 
-size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int T, int H, int W) {
+rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* g, rf_ws_layout_t* lay) {
+  return rf_workspace_layout_ex(RF_PREC_NATIVE, B, N, D, g, lay);
+}
+
+size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int T, int H, int W) {
   rf_plan_t g;
   rf_ws_layout_t L;
   if (rf_plan(S, txt_len, T, H, W, RF_BLOCK, 0.f, &g) != RF_OK) return 0;
-  if (rf_workspace_layout(B, N, D, &g, &L) != RF_OK) return 0;
+  if (rf_workspace_layout_ex(precision, B, N, D, &g, &L) != RF_OK) return 0;
   return L.total;
+}
+
+size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int T, int H, int W) {
+  return rf_workspace_size_ex(RF_PREC_NATIVE, B, S, N, D, txt_len, T, H, W);
+}
+
+rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype, rf_precision_t precision,
+                          rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W,
+                          int block_size, float sparsity, void* ws, size_t ws_bytes, void* stream) {
+  rf_status_t st = check_common(layout, B, S, N, D);
+  if (st != RF_OK) return st;
+  if ((st = check_types(dtype, precision)) != RF_OK) return st;
+  if (!q || !k || !v) return fail(RF_ERR_ARG, "q, k and v must be device pointers");
+  rf_plan_t g;
+  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_ws_layout_t L;
+  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = rf::launch_permute_pool(q, k, v, dtype, layout, B, S, N, g, at<void>(ws, L.q_int),
+                                          at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
+                                          at<float>(ws, L.pooled_k), s);
+  if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
+  e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, at<uint32_t>(ws, L.mask),
+                      at<int>(ws, L.kept), at<float>(ws, L.margin), s);
+  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
+  if (precision == RF_PREC_FP8) {
+    e = rf::launch_quantize_fp8(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int), dtype, B * N, g,
+                                at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
+                                at<float>(ws, L.scales), at<float>(ws, L.vmax), s);
+    if (e != cudaSuccess) return cuda_fail(e, "fp8 quantisation launch");
+  }
+  return ok();
 }
 
 rf_status_t rf_prepare(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N, int D,
                        int txt_len, int T, int H, int W, int block_size, float sparsity, void* ws, size_t ws_bytes,
                        void* stream) {
+  return rf_prepare_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity,
+                       ws, ws_bytes, stream);
+}
+
+rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                         int txt_len, int T, int H, int W, int block_size, float sparsity, float scale, void* out,
+                         void* ws, size_t ws_bytes, void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
-  if (!q || !k || !v) return fail(RF_ERR_ARG, "q, k and v must be device pointers");
+  if ((st = check_types(dtype, precision)) != RF_OK) return st;
+  if (!out) return fail(RF_ERR_ARG, "out must be a device pointer");
   rf_plan_t g;
   if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
   rf_ws_layout_t L;
-  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = rf::launch_permute_pool(q, k, v, layout, B, S, N, g, at<void>(ws, L.q_int), at<void>(ws, L.k_int),
-                                          at<void>(ws, L.v_int), at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k),
-                                          s);
-  if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
-  e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, at<uint32_t>(ws, L.mask),
-                      at<int>(ws, L.kept), at<float>(ws, L.margin), s);
-  if (e != cudaSuccess) return cuda_fail(e, "mask launch");
+  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
+  if (precision == RF_PREC_FP8)
+    e = rf::launch_attention_fp8(at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
+                                 at<float>(ws, L.scales), at<float>(ws, L.vmax), at<uint32_t>(ws, L.mask), dtype,
+                                 layout, B, S, N, g, resolve_scale(scale, D), out, at<int>(ws, L.counter),
+                                 at<int>(ws, L.status), debug_settings(), s);
+  else
+    e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
+                             at<uint32_t>(ws, L.mask), dtype, layout, B, S, N, g, resolve_scale(scale, D), out,
+                             at<int>(ws, L.counter), at<int>(ws, L.status), debug_settings(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
 }
 
 rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W,
                       int block_size, float sparsity, float scale, void* out, void* ws, size_t ws_bytes,
                       void* stream) {
+  return rf_attend_ex(RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out,
+                      ws, ws_bytes, stream);
+}
+
+rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype,
+                                   rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                                   int txt_len, int T, int H, int W, int block_size, float sparsity, float scale,
+                                   void* out, void* ws, size_t ws_bytes, void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
-  if (!out) return fail(RF_ERR_ARG, "out must be a device pointer");
-  rf_plan_t g;
-  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
-  rf_ws_layout_t L;
-  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
-  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
-  cudaError_t e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
-  e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
-                                       at<uint32_t>(ws, L.mask), layout, B, S, N, g, resolve_scale(scale, D), out,
-                                       at<int>(ws, L.counter), at<int>(ws, L.status), debug_settings(),
-                                       static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
-  return ok();
+  if ((st = check_types(dtype, precision)) != RF_OK) return st;
+  if (!q || !k || !v || !out) return fail(RF_ERR_ARG, "q, k, v and out must be device pointers");
+  if (out == q || out == k || out == v) return fail(RF_ERR_ARG, "out must not alias q, k or v");
+  if (!ws) {
+    rf_plan_t g;
+    if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+    rf_ws_layout_t L;
+    if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
+    if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
+    ws_bytes = L.total;
+  }
+  st = rf_prepare_ex(q, k, v, dtype, precision, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, ws,
+                     ws_bytes, stream);
+  if (st != RF_OK) return st;
+  return rf_attend_ex(dtype, precision, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws,
+                      ws_bytes, stream);
 }
 
 rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
                                    int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
                                    float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
-  if (out && (out == q || out == k || out == v)) return fail(RF_ERR_ARG, "out must not alias q, k or v");
-  rf_status_t st = rf_prepare(q, k, v, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, ws, ws_bytes,
-                              stream);
-  if (st != RF_OK) return st;
-  return rf_attend(layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws, ws_bytes, stream);
+  if (!ws) return fail(RF_ERR_WORKSPACE, "workspace is NULL");
+  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size,
+                                sparsity, scale, out, ws, ws_bytes, stream);
 }
 
 rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
                                 int D, int txt_len, int T, int H, int W, int block_size, float sparsity, float scale,
                                 void* out, void* stream) {
-  rf_status_t st = check_common(layout, B, S, N, D);
-  if (st != RF_OK) return st;
-  rf_plan_t g;
-  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
-  rf_ws_layout_t L;
-  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
-  if (!q || !k || !v || !out) return fail(RF_ERR_ARG, "q, k, v and out must be device pointers");
-  void* ws = nullptr;
-  if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
-  return rf_sparse_attention_ws(q, k, v, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws,
-                                L.total, stream);
+  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size,
+                                sparsity, scale, out, nullptr, 0, stream);
 }
 
 rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H,
@@ -348,7 +412,7 @@ rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layo
     return fail(RF_ERR_UNSUPPORTED,
                 "B*N*nb = %zu block rows need %zu bytes of pooled scratch, above the static %u-byte array",
                 (size_t)B * N * g.nb, need, (unsigned)RF_NOALLOC_SCRATCH_BYTES);
-  cudaError_t e = rf::launch_block_mask_noalloc(q, k, layout, B, S, N, g, mask, kept, margin,
+  cudaError_t e = rf::launch_block_mask_noalloc(q, k, RF_BF16, layout, B, S, N, g, mask, kept, margin,
                                                 static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "no-allocation mask launch");
   return ok();

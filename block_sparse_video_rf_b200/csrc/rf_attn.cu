@@ -20,24 +20,36 @@
 //   warps 0-3   slot 0, warps 4-7 slot 1: thread = query row (TMEM lane);
 //               online softmax in exp2 with a lazily updated running max;
 //               most exponentials on the MUFU unit, one pair in four on the
-//               FMA pipe (polynomial); P (bf16) is written over the first 64
-//               columns of the slot's S; at the end of a unit the same
-//               threads write O / l -> bf16 -> the caller's layout.  The
-//               slot's first warp also issues its MMAs (one elected lane):
-//               S = Q K^T: tcgen05 kind::f16, A and B from shared memory;
-//               O += P V:  A = P from tensor memory, B = V MN-major.
+//               FMA pipe (polynomial); P is written over the first columns of
+//               the slot's S; at the end of a unit the same threads write
+//               O / l in the caller's type and layout.  The slot's first warp
+//               also issues its MMAs (one elected lane):
+//                 S = Q K^T:  A and B from shared memory;
+//                 O += P V:   A = P from tensor memory, B = V.
 //               The four warps meet at a named barrier after each tile, so
 //               P V follows P without an mbarrier hand-off.
 //   warps 8, 9  TMA producers of slot 0 and slot 1 (one thread each): Q, then
 //               the K and V tiles of the KV list, 128-byte swizzled boxes of
-//               128 rows x 64 columns.
+//               128 rows x 128 bytes.
 //   warp 10     owns the tensor memory; warps 10 and 11 are otherwise idle.
 // Tensor memory (512 columns): slot z has S at [256 z, 256 z + 128) (P in
-// its first 64 columns) and O at [256 z + 128, 256 z + 256).  Since P
+// its first columns) and O at [256 z + 128, 256 z + 256).  Since P
 // overwrites S, the QK of a slot's next tile is issued once its P V is done.
 // Registers: the control warpgroup (warps 8-11) gives registers to the two
 // slot warpgroups (setmaxnreg 64 / 216: 8 x 32 x 216 + 4 x 32 x 64 =
 // 63,488 <= 384 threads x 168 at launch).
+//
+// Precisions (template parameters):
+//   16-bit: Q, K, V and out bf16 or fp16; tcgen05 kind::f16, 8 MMAs of
+//     128x128x16 per product; P in the input type (64 TMEM columns);
+//     V MN-major; single K and V buffers per slot.
+//   fp8: Q, K, V as e4m3 codes with one fp32 scale per 128-row block
+//     (written by the quantisation kernel; V's blocks stored transposed so
+//     that P V has a K-major B); tcgen05 kind::f8f6f4, 4 MMAs of 128x128x32
+//     per product; S is scaled by sq * sk in the softmax; P is e4m3 (32 TMEM
+//     columns) and carries the V block's scale relative to the head's
+//     largest one (sv / vmax, folded into the exponent), which the epilogue
+//     multiplies back; two K and two V buffers per slot.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -57,31 +69,62 @@ constexpr int kThreads = 384;
 constexpr int kSlots = 2;
 constexpr int kSlotWarps = 4;                            // softmax warps per slot
 constexpr uint32_t kRegsSoftmax = 216, kRegsControl = 64;
-constexpr int kTileBytes = RF_BLOCK * RF_HEAD_DIM * 2;   // 32 KB
-constexpr int kHalfBytes = kTileBytes / 2;               // 64 columns x 128 rows
+constexpr int kBoxBytes = RF_BLOCK * 128;                // one TMA box: 128 rows x 128 bytes
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPolyEvery = 4;                            // pair i uses the polynomial when i % 4 == 3
 constexpr float kRescaleThreshold = 8.0f;                // log2 units
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Compile-time shape of one precision.
+template <bool kF16_, bool kFp8_>
+struct Cfg {
+  static constexpr bool kF16 = kF16_;                    // 16-bit type: fp16 (else bf16); also the output type
+  static constexpr bool kFp8 = kFp8_;
+  static constexpr int kBoxes = kFp8 ? 1 : 2;            // boxes per 128 x 128 tile
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;
+  static constexpr int kKStages = kFp8 ? 2 : 1;
+  static constexpr int kVStages = kFp8 ? 2 : 1;
+  static constexpr int kSteps = kFp8 ? 4 : 8;            // MMAs per product over 128 (K 32 or 16 each)
+  static constexpr int kPCols = kFp8 ? 32 : 64;          // TMEM columns of P
+  static constexpr uint32_t kIdescQK =
+      kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, false, !kF16);
+  static constexpr uint32_t kIdescPV =
+      kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, true, !kF16);
+};
+
 struct Item {
   int bn, qt, ntiles, pad;
 };
 
+// Per-tile factors of the fp8 path, written by the slot's issuer before its
+// arrival on s_full: c = scale * log2(e) * sq * sk (multiplies S), lr =
+// log2(sv / vmax) (added to P's exponent), ir = vmax / sv (l adds P's sum
+// times ir).
+struct TileScale {
+  float c, lr, ir, pad;
+};
+
 // One slot: buffers and barriers of one unit in flight.
+template <class C>
 struct __align__(1024) Slot {
-  uint8_t q[kTileBytes];
-  uint8_t k[kTileBytes];
-  uint8_t v[kTileBytes];
-  uint64_t q_full, q_empty, k_full, k_empty, v_full, v_empty;
-  uint64_t s_full, pv_done;
+  uint8_t q[C::kTileBytes];
+  uint8_t k[C::kKStages][C::kTileBytes];
+  uint8_t v[C::kVStages][C::kTileBytes];
+  uint64_t q_full, q_empty;
+  uint64_t k_full[C::kKStages], k_empty[C::kKStages], v_full[C::kVStages], v_empty[C::kVStages];
+  uint64_t s_full;              // S = Q K^T of a tile done (commit) and its TileScale written (issuer)
+  uint64_t pv_done;
   uint64_t drain;               // the issuer's last commit when it leaves early
   uint64_t item_full[2], item_empty[2];
   Item items[2];
+  float q_scale;                // fp8: the unit's Q block scale (producer, with q_full)
+  float kv_scale[C::kKStages][2];   // fp8: {sk, sv} of the tile in each K stage (producer, with k_full)
+  TileScale ts[2];              // fp8: by tile parity (issuer, with s_full)
 };
 
+template <class C>
 struct Smem {
-  Slot slot[kSlots];
+  Slot<C> slot[kSlots];
   uint32_t tmem_base;
   int abort;
 };
@@ -94,9 +137,11 @@ struct AttnParams {
   int p_rem;         // valid rows of the last prefix tile when it is partial, else 0
   float scale_log2;
   const uint32_t* mask;
+  const float* scales;   // fp8: [3, B*N, n_tiles] block scales of q, k, v
+  const float* vmax;     // fp8: [B*N] largest V block scale of each head
   int* counter;
   int* status;
-  __nv_bfloat16* out;
+  void* out;
   uint64_t wait_limit_ns;   // limit of every device-side wait
   int skip_first_q;         // test control: the first unit's Q load is never issued
 };
@@ -106,12 +151,14 @@ __device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
 }
 
 // Bounded wait by one thread.
-__device__ __forceinline__ bool wait1(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
+template <class C>
+__device__ __forceinline__ bool wait1(Smem<C>& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
   return rf_wait(bar, parity, &sm.abort, p.status, RF_ERR_TIMEOUT, p.wait_limit_ns);
 }
 // Bounded wait by a whole warp, with a warp-uniform outcome (the warp then
 // runs .sync.aligned tcgen05 instructions together or leaves together).
-__device__ __forceinline__ bool waitw(Smem& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
+template <class C>
+__device__ __forceinline__ bool waitw(Smem<C>& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
   return __all_sync(0xFFFFFFFFu, wait1(sm, p, bar, parity));
 }
 // One arrival per warp, after every lane's preceding work (callers fence first).
@@ -168,15 +215,28 @@ struct KvIter {
   }
 };
 
+// One 128 x 128 tile: one box of 128 bytes per row (fp8) or two boxes of 64
+// 16-bit columns.
+template <class C>
+__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row,
+                                          uint64_t policy) {
+  mbar_arrive_expect_tx(bar, C::kTileBytes);
+#pragma unroll
+  for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(dst + b * kBoxBytes, map, bar, b * 64, row, policy);
+}
+
 // Producer of one slot: takes units from the global counter, loads Q and then
-// the K and V tiles of the KV list (one buffer each; K of the next tile as
-// soon as the previous S = Q K^T is done, V as soon as the previous P V is).
-__device__ void producer_loop(Smem& sm, Slot& sl, const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                              const CUtensorMap* tv) {
+// the K and V tiles of the KV list into rings of kKStages / kVStages buffers
+// (K of tile t once S of tile t - stages is done, V once P V of tile
+// t - stages is).  The fp8 path also passes each tile's block scales on.
+template <class C>
+__device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, const CUtensorMap* tq,
+                              const CUtensorMap* tk, const CUtensorMap* tv) {
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
   uint32_t c = 0, nk = 0, nv = 0;   // units, K tiles and V tiles issued
   const int S_int = p.g.S_int;
+  const int BN = p.B * p.N;
   bool ok = true;
   while (ok) {
     const int w = atomicAdd(p.counter, 1);
@@ -204,34 +264,38 @@ __device__ void producer_loop(Smem& sm, Slot& sl, const AttnParams& p, const CUt
     if (itm.bn < 0) break;
 
     const int base = itm.bn * S_int;
+    const float* sc_k = C::kFp8 ? p.scales + ((size_t)BN + itm.bn) * p.g.n_tiles : nullptr;
+    const float* sc_v = C::kFp8 ? p.scales + ((size_t)2 * BN + itm.bn) * p.g.n_tiles : nullptr;
     if (c >= 1 && !wait1(sm, p, &sl.q_empty, ph(c - 1))) {
       ok = false;
       break;
     }
     if (!(p.skip_first_q && c == 0)) {
-      mbar_arrive_expect_tx(&sl.q_full, kTileBytes);
-      tma_load_2d(sl.q, tq, &sl.q_full, 0, base + itm.qt * RF_BLOCK, pol_q);
-      tma_load_2d(sl.q + kHalfBytes, tq, &sl.q_full, 64, base + itm.qt * RF_BLOCK, pol_q);
+      if (C::kFp8) sl.q_scale = p.scales[(size_t)itm.bn * p.g.n_tiles + itm.qt];
+      load_tile<C>(sl.q, tq, &sl.q_full, base + itm.qt * RF_BLOCK, pol_q);
     }
     ++c;
     KvIter kit;
     kit.init(base, p, mrow);
     for (int row = kit.next(); row >= 0 && ok; row = kit.next()) {
-      if (nk >= 1 && !wait1(sm, p, &sl.k_empty, ph(nk - 1))) {
+      const uint32_t ks = nk % C::kKStages, ku = nk / C::kKStages;
+      if (ku >= 1 && !wait1(sm, p, &sl.k_empty[ks], ph(ku - 1))) {
         ok = false;
         break;
       }
-      mbar_arrive_expect_tx(&sl.k_full, kTileBytes);
-      tma_load_2d(sl.k, tk, &sl.k_full, 0, row, pol_kv);
-      tma_load_2d(sl.k + kHalfBytes, tk, &sl.k_full, 64, row, pol_kv);
+      if (C::kFp8) {
+        const int tile = (row - base) / RF_BLOCK;
+        sl.kv_scale[ks][0] = sc_k[tile];
+        sl.kv_scale[ks][1] = sc_v[tile];
+      }
+      load_tile<C>(sl.k[ks], tk, &sl.k_full[ks], row, pol_kv);
       ++nk;
-      if (nv >= 1 && !wait1(sm, p, &sl.v_empty, ph(nv - 1))) {
+      const uint32_t vs = nv % C::kVStages, vu = nv / C::kVStages;
+      if (vu >= 1 && !wait1(sm, p, &sl.v_empty[vs], ph(vu - 1))) {
         ok = false;
         break;
       }
-      mbar_arrive_expect_tx(&sl.v_full, kTileBytes);
-      tma_load_2d(sl.v, tv, &sl.v_full, 0, row, pol_kv);
-      tma_load_2d(sl.v + kHalfBytes, tv, &sl.v_full, 64, row, pol_kv);
+      load_tile<C>(sl.v[vs], tv, &sl.v_full[vs], row, pol_kv);
       ++nv;
     }
   }
@@ -240,32 +304,49 @@ __device__ void producer_loop(Smem& sm, Slot& sl, const AttnParams& p, const CUt
     // time, not cut short by the abort flag).
     const uint64_t lim = p.wait_limit_ns / 4;
     if (c) rf_wait_time(&sl.q_full, ph(c - 1), lim);
-    if (nk) rf_wait_time(&sl.k_full, ph(nk - 1), lim);
-    if (nv) rf_wait_time(&sl.v_full, ph(nv - 1), lim);
+    for (uint32_t st = 0; st < (uint32_t)C::kKStages; ++st) {
+      const uint32_t n = (nk > st) ? (nk - st + C::kKStages - 1) / C::kKStages : 0;   // loads into stage st
+      if (n) rf_wait_time(&sl.k_full[st], ph(n - 1), lim);
+    }
+    for (uint32_t st = 0; st < (uint32_t)C::kVStages; ++st) {
+      const uint32_t n = (nv > st) ? (nv - st + C::kVStages - 1) / C::kVStages : 0;
+      if (n) rf_wait_time(&sl.v_full[st], ph(n - 1), lim);
+    }
   }
 }
 
 // ---------------------------------------------------------------- MMA issue
 // Descriptor low words of the 128-byte swizzled operands; every descriptor
 // used here shares one high word (stride 1024 B, sm_100 version, swizzle).
-// A K step of 16 elements advances a K-major operand by 32 B (2 in the
-// descriptor's 16-byte units), and the second 64-column half by 16 KB.
-// The issuing warp runs this code together; one elected lane issues.
+// A K step (16 16-bit or 32 8-bit elements) advances a K-major operand by
+// 32 B (2 in the descriptor's 16-byte units); the second box of a 16-bit
+// tile (columns 64..127) starts 16 KB further.  The issuing warp runs this
+// code together; one elected lane issues.
+template <class C>
 __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
-  constexpr uint32_t idesc = make_idesc_bf16(128, 128, false);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = ((kk >> 2) * kHalfBytes + (kk & 3) * 32) >> 4;
-    mma_ss_lo_elect(s_tmem, q_lo + off, k_lo + off, hi, idesc, kk > 0);
+  for (int kk = 0; kk < C::kSteps; ++kk) {
+    const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+    if (C::kFp8)
+      mma_ss_lo_elect_f8(s_tmem, q_lo + off, k_lo + off, hi, C::kIdescQK, kk > 0);
+    else
+      mma_ss_lo_elect(s_tmem, q_lo + off, k_lo + off, hi, C::kIdescQK, kk > 0);
   }
 }
-// V is MN-major: a K step of 16 keys advances it by 16 rows of 128 B.
+// P V: a K step takes the next 8 TMEM columns of P (16 16-bit or 32 8-bit
+// keys).  16-bit V is MN-major: 16 keys are 16 rows of 128 B further.  fp8 V
+// is stored transposed (K-major): 32 keys are 32 B further.
+template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
                                          bool accumulate) {
-  constexpr uint32_t idesc = make_idesc_bf16(128, 128, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
-    mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, idesc, (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < C::kSteps; ++kk) {
+    const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+    if (C::kFp8)
+      mma_ts_lo_elect_f8(o_tmem, p_tmem + kk * 8, v_lo + kk * 2, hi, C::kIdescPV, acc);
+    else
+      mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, C::kIdescPV, acc);
+  }
 }
 
 // Rendezvous of a slot's four warps (named barrier `id`, 128 threads) that
@@ -283,14 +364,17 @@ __device__ __forceinline__ bool slot_vote(int id, bool ok) {
 }
 
 // ---------------------------------------------------------------- softmax of one tile
-// Thread = query row.  Reads the row's 128 scores from S, updates the running
-// max m_use (log2 units, lazily: only when a score exceeds it by more than
-// the threshold, then O and l are rescaled), adds the tile's sum to l and
-// writes P = 2^(s * scale * log2 e - m_use) as bf16 over the first 64
-// columns of S.  `p_valid` < 128 masks the keys past the prefix's end.
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool first, int p_valid, float sl2,
-                                             float& m_use, float& l) {
-  const uint64_t sl2x2 = f2_pack(sl2, sl2);
+// Thread = query row.  Reads the row's 128 scores from S, scales them by c
+// (log2 units), updates the running max m_use (lazily: only when a score
+// exceeds it by more than the threshold, then O and l are rescaled), adds
+// the tile's sum of P (times ir) to l and writes P = 2^(s c - m_use + lr)
+// over the first columns of S: as 64 words of two 16-bit values, or (fp8)
+// 32 words of four e4m3 codes.  `p_valid` < 128 masks the keys past the
+// prefix's end.
+template <class C>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool first, int p_valid, float c, float lr,
+                                             float ir, float& m_use, float& l) {
+  const uint64_t c2 = f2_pack(c, c);
   uint32_t s[4][32];
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
@@ -315,7 +399,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
     for (int e = 0; e < 32; e += 2)
       mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
   const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-  const float mx_s = mx * sl2;
+  const float mx_s = mx * c;
   float alpha = 1.f;
   bool rescale = false;
   if (first) {
@@ -325,15 +409,17 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
     m_use = mx_s;
     rescale = true;
   }
-  const uint64_t negm = f2_pack(-m_use, -m_use);
+  const float off = lr - m_use;
+  const uint64_t negm = f2_pack(off, off);
   uint64_t sum2[4] = {0, 0, 0, 0};
-  uint32_t pk[64];
+  uint32_t pk[C::kPCols];
+  float hold0 = 0.f, hold1 = 0.f;   // fp8: the first pair of a 4-key word
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4)
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
       const int i = 16 * q4 + (e >> 1);     // pair index 0..63
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), sl2x2, negm);
+      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), c2, negm);
       uint64_t p2;
       if ((i % kPolyEvery) == kPolyEvery - 1) {
         p2 = exp2_poly_x2(x2);
@@ -350,12 +436,21 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
       sum2[i & 3] = f2_add(sum2[i & 3], p2);
       float a0, a1;
       f2_unpack(p2, a0, a1);
-      pk[i] = pack_bf16x2(a0, a1);
+      if (C::kFp8) {
+        if (i & 1)
+          pk[i >> 1] = pack_e4m3x4(hold0, hold1, a0, a1);
+        else {
+          hold0 = a0;
+          hold1 = a1;
+        }
+      } else {
+        pk[i] = pack_half2<C::kF16>(a0, a1);
+      }
     }
   float s0, s1, s2, s3;
   f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
   f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
-  l = l * alpha + ((s0 + s1) + (s2 + s3));
+  l = l * alpha + ((s0 + s1) + (s2 + s3)) * ir;
   if (__any_sync(0xFFFFFFFFu, rescale)) {
     // O holds the tiles before this one: their P V completed before this
     // tile's S = Q K^T was issued.
@@ -370,8 +465,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
       tmem_st32(tO + 32 * q4, o);
     }
   }
-  tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-  tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+#pragma unroll
+  for (int w = 0; w < C::kPCols; w += 32) tmem_st32(tS + w, *reinterpret_cast<uint32_t(*)[32]>(&pk[w]));
   tmem_wait_st();
   tc_fence_before();
 }
@@ -382,7 +477,8 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
 // the slot's MMAs: S = Q K^T of a tile once the P V of the previous tile is
 // done (P lives in the S columns), and P V of a tile once all four warps
 // have written P (the rendezvous after each tile).
-__device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem_slot, int bar_id) {
+template <class C>
+__device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_t tmem_slot, int bar_id) {
   const int quad = (threadIdx.x >> 5) & 3;
   const bool issuer = (quad == 0);
   const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
@@ -391,23 +487,43 @@ __device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem
   const uint32_t s_tmem = tmem_slot, o_tmem = tmem_slot + 128;
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
   const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.q), 16, 1024);
-  const uint32_t k_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.k), 16, 1024);
-  const uint32_t v_lo = (uint32_t)make_sdesc_sw128(smem_u32(sl.v), kHalfBytes, 1024);
+  const uint32_t k_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sl.k[0]), 16, 1024);
+  const uint32_t v_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sl.v[0]), C::kFp8 ? 16 : kBoxBytes, 1024);
   uint32_t c = 0, t = 0;   // units and tiles of this slot
   bool ok = true;
   bool issued = false;     // the issuer has MMAs that may still run
+  float q_scale = 1.f;     // fp8: the unit's Q block scale (issuer)
+  float unit_vmax = 1.f;   // fp8: the largest V block scale of the unit's head (issuer)
 
-  // S = Q K^T of tile t (issuer warp): K tile t must have landed and the
-  // P V of tile t-1 must be done.
+  // S = Q K^T of tile tt (issuer warp): K tile tt must have landed and the
+  // P V of tile tt - 1 must be done.  Then the tile's fp8 factors go to
+  // ts[tt & 1], and the issuer's arrival on s_full publishes them.
   auto qk = [&](uint32_t tt, bool last_of_unit) -> bool {
-    if (!waitw(sm, p, &sl.k_full, ph(tt))) return false;
+    const uint32_t ks = tt % C::kKStages;
+    if (!waitw(sm, p, &sl.k_full[ks], ph(tt / C::kKStages))) return false;
+    // read before the MMAs: once they finish, the producer may refill the stage
+    const float sk = C::kFp8 ? sl.kv_scale[ks][0] : 0.f, sv = C::kFp8 ? sl.kv_scale[ks][1] : 0.f;
     if (tt >= 1 && !waitw(sm, p, &sl.pv_done, ph(tt - 1))) return false;
     tc_fence_after();
-    issue_qk(s_tmem, q_lo, k_lo, hi);
+    issue_qk<C>(s_tmem, q_lo, k_lo0 + ks * (C::kTileBytes >> 4), hi);
     mma_commit_elect(&sl.s_full);
-    mma_commit_elect(&sl.k_empty);
+    mma_commit_elect(&sl.k_empty[ks]);
     if (last_of_unit) mma_commit_elect(&sl.q_empty);
     issued = true;
+    if ((threadIdx.x & 31) == 0) {
+      if (C::kFp8) {
+        const float vmax = unit_vmax;
+        TileScale f;
+        f.c = p.scale_log2 * q_scale * sk;
+        const bool use_r = sv > 0.f && vmax > 0.f;   // an all-zero V block adds nothing whatever P is
+        f.lr = use_r ? __log2f(sv / vmax) : 0.f;
+        f.ir = use_r ? vmax / sv : 1.f;
+        f.pad = 0.f;
+        sl.ts[tt & 1] = f;
+      }
+      mbar_arrive(&sl.s_full);
+    }
+    __syncwarp();
     return true;
   };
 
@@ -423,7 +539,15 @@ __device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem
     }
     ok = slot_vote(bar_id, ok);
     if (!ok || itm.bn < 0) break;
-    if (issuer) ok = waitw(sm, p, &sl.q_full, ph(c)) && qk(t, itm.ntiles == 1);
+    if (issuer) {
+      ok = waitw(sm, p, &sl.q_full, ph(c));
+      if (C::kFp8 && ok) {
+        q_scale = sl.q_scale;
+        unit_vmax = p.vmax[itm.bn];
+      }
+      if (ok) ok = qk(t, itm.ntiles == 1);
+    }
+    const float out_scale = C::kFp8 ? p.vmax[itm.bn] : 1.f;
 
     float m_use = -CUDART_INF_F, l = 0.f;
     for (int j = 0; j < itm.ntiles; ++j, ++t) {
@@ -431,29 +555,37 @@ __device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem
       if (ok) {
         tc_fence_after();
         const int p_valid = (p.p_rem != 0 && j == p.n_ptiles - 1) ? p.p_rem : RF_BLOCK;
-        softmax_tile(tS, tO, j == 0, p_valid, p.scale_log2, m_use, l);
+        if (C::kFp8) {
+          const TileScale f = sl.ts[t & 1];
+          softmax_tile<C>(tS, tO, j == 0, p_valid, f.c, f.lr, f.ir, m_use, l);
+        } else {
+          softmax_tile<C>(tS, tO, j == 0, p_valid, p.scale_log2, 0.f, 1.f, m_use, l);
+        }
       }
       ok = slot_vote(bar_id, ok);
       if (!ok) break;
       if (issuer) {
-        ok = waitw(sm, p, &sl.v_full, ph(t));
+        const uint32_t vs = t % C::kVStages;
+        ok = waitw(sm, p, &sl.v_full[vs], ph(t / C::kVStages));
         if (ok) {
           tc_fence_after();
-          issue_pv(o_tmem, s_tmem, v_lo, hi, j > 0);
+          issue_pv<C>(o_tmem, s_tmem, v_lo0 + vs * (C::kTileBytes >> 4), hi, j > 0);
           mma_commit_elect(&sl.pv_done);
-          mma_commit_elect(&sl.v_empty);
+          mma_commit_elect(&sl.v_empty[vs]);
           if (j + 1 < itm.ntiles) ok = qk(t + 1, j + 2 == itm.ntiles);
         }
       }
     }
-    // epilogue: O / l of this unit once its last P V is done
+    // epilogue: O * out_scale / l of this unit once its last P V is done
     if (ok) ok = waitw(sm, p, &sl.pv_done, ph(t - 1));
     if (ok) {
       tc_fence_after();
-      const float rl = 1.f / l;
+      const float rl = out_scale / l;
       const int b = itm.bn / p.N, nh = itm.bn - b * p.N;
       const int src = rf_src_of_row(p.g, itm.qt * RF_BLOCK + row);
-      __nv_bfloat16* dst = src >= 0 ? p.out + rf_token_offset(p.layout, p.B, p.S, p.N, b, nh, src) : nullptr;
+      uint16_t* dst = src >= 0
+                          ? static_cast<uint16_t*>(p.out) + rf_token_offset(p.layout, p.B, p.S, p.N, b, nh, src)
+                          : nullptr;
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
         uint32_t o[32];
@@ -464,7 +596,7 @@ __device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
+            w[e] = pack_half2<C::kF16>(__uint_as_float(o[2 * e]) * rl, __uint_as_float(o[2 * e + 1]) * rl);
           uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * q4);
 #pragma unroll
           for (int e = 0; e < 4; ++e) d4[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
@@ -484,23 +616,28 @@ __device__ void slot_loop(Smem& sm, Slot& sl, const AttnParams& p, uint32_t tmem
   }
 }
 
+template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem<C>& sm = *reinterpret_cast<Smem<C>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int z = 0; z < kSlots; ++z) {
-      Slot& sl = sm.slot[z];
+      Slot<C>& sl = sm.slot[z];
       mbar_init(&sl.q_full, 1);
       mbar_init(&sl.q_empty, 1);
-      mbar_init(&sl.k_full, 1);
-      mbar_init(&sl.k_empty, 1);
-      mbar_init(&sl.v_full, 1);
-      mbar_init(&sl.v_empty, 1);
-      mbar_init(&sl.s_full, 1);
+      for (int i = 0; i < C::kKStages; ++i) {
+        mbar_init(&sl.k_full[i], 1);
+        mbar_init(&sl.k_empty[i], 1);
+      }
+      for (int i = 0; i < C::kVStages; ++i) {
+        mbar_init(&sl.v_full[i], 1);
+        mbar_init(&sl.v_empty[i], 1);
+      }
+      mbar_init(&sl.s_full, 2);   // the MMA commit and the issuer's arrival
       mbar_init(&sl.pv_done, 1);
       mbar_init(&sl.drain, 1);
       for (int i = 0; i < 2; ++i) {
@@ -528,11 +665,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 8) {
     regs_increase<kRegsSoftmax>();
     const int z = warp >> 2;
-    slot_loop(sm, sm.slot[z], p, tmem + 256 * z, 1 + z);
+    slot_loop<C>(sm, sm.slot[z], p, tmem + 256 * z, 1 + z);
   } else {
     regs_decrease<kRegsControl>();
-    if (warp == 8 && lane == 0) producer_loop(sm, sm.slot[0], p, &tm_q, &tm_k, &tm_v);
-    if (warp == 9 && lane == 0) producer_loop(sm, sm.slot[1], p, &tm_q, &tm_k, &tm_v);
+    if (warp == 8 && lane == 0) producer_loop<C>(sm, sm.slot[0], p, &tm_q, &tm_k, &tm_v);
+    if (warp == 9 && lane == 0) producer_loop<C>(sm, sm.slot[1], p, &tm_q, &tm_k, &tm_v);
   }
   __syncwarp();
   tc_fence_before();
@@ -558,28 +695,22 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, 128] bf16 row-major, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows) {
+// [rows, 128] elements of `elem_bytes` (2: bf16/fp16, 1: e4m3 codes),
+// row-major; boxes of 128 rows x 128 bytes, 128-byte swizzle.
+bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, CUtensorMapDataType type, int elem_bytes) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {RF_HEAD_DIM, rows};
-  const cuuint64_t strides[1] = {RF_HEAD_DIM * 2};
-  const cuuint32_t box[2] = {64, RF_BLOCK};
+  const cuuint64_t strides[1] = {(cuuint64_t)RF_HEAD_DIM * elem_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), RF_BLOCK};
   const cuuint32_t estr[2] = {1, 1};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
-                             int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
-                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream) {
-  const uint64_t rows = (uint64_t)B * N * g.S_int;
-  CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, q_int, rows) || !make_tile_map(&tk, k_int, rows) || !make_tile_map(&tv, v_int, rows))
-    return cudaErrorInvalidValue;
+AttnParams make_params(const uint32_t* mask, int layout, int B, int S, int N, const rf_plan_t& g, float scale,
+                       void* out, int* counter, int* status, const AttnDebug& dbg) {
   AttnParams p;
   p.g = g;
   p.B = B;
@@ -591,25 +722,66 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
   p.p_rem = g.P % RF_BLOCK;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.mask = mask;
+  p.scales = nullptr;
+  p.vmax = nullptr;
   p.counter = counter;
   p.status = status;
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.out = out;
   p.wait_limit_ns = dbg.wait_limit_ns > 0 ? (uint64_t)dbg.wait_limit_ns : kWaitLimitNs;
   p.skip_first_q = dbg.skip_first_q;
+  return p;
+}
 
+template <class C>
+cudaError_t launch_cfg(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                       cudaStream_t stream) {
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const size_t smem = sizeof(Smem) + 1024;
-  e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(Smem<C>) + 1024;
+  e = cudaFuncSetAttribute(attn_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(counter, 0, sizeof(int), stream);
+  e = cudaMemsetAsync(p.counter, 0, sizeof(int), stream);
   if (e != cudaSuccess) return e;
   const int grid = std::min(sms, p.total_items);
-  attn_kernel<<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+  attn_kernel<C><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
+                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
+                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream) {
+  const uint64_t rows = (uint64_t)B * N * g.S_int;
+  const bool f16 = dtype == RF_F16;
+  const CUtensorMapDataType type = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, q_int, rows, type, 2) || !make_tile_map(&tk, k_int, rows, type, 2) ||
+      !make_tile_map(&tv, v_int, rows, type, 2))
+    return cudaErrorInvalidValue;
+  const AttnParams p = make_params(mask, layout, B, S, N, g, scale, out, counter, status, dbg);
+  return f16 ? launch_cfg<Cfg<true, false>>(tq, tk, tv, p, stream)
+             : launch_cfg<Cfg<false, false>>(tq, tk, tv, p, stream);
+}
+
+cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
+                                 const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
+                                 const rf_plan_t& g, float scale, void* out, int* counter, int* status,
+                                 const AttnDebug& dbg, cudaStream_t stream) {
+  const uint64_t rows = (uint64_t)B * N * g.S_int;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, q8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tk, k8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tv, v8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
+    return cudaErrorInvalidValue;
+  AttnParams p = make_params(mask, layout, B, S, N, g, scale, out, counter, status, dbg);
+  p.scales = scales;
+  p.vmax = vmax;
+  return dtype == RF_F16 ? launch_cfg<Cfg<true, true>>(tq, tk, tv, p, stream)
+                         : launch_cfg<Cfg<false, true>>(tq, tk, tv, p, stream);
 }
 
 }  // namespace rf

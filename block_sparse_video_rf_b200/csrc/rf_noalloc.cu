@@ -16,11 +16,11 @@
 // must be ordered by the caller.  Each call overwrites every element it later
 // reads, so nothing has to start at zero and the previous call's contents do
 // not matter.
-#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
 
+#include "rf_dtype.h"
 #include "rf_geometry.h"
 #include "rf_kernels.h"
 
@@ -35,21 +35,13 @@ constexpr int kThreads = 256;        // 16 column chunks x 16 rows per pass
 constexpr int kRowsPerPass = 16;
 constexpr int kPasses = RF_BLOCK / kRowsPerPass;
 
-__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& u) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __uint_as_float(w[i] << 16);
-    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 // One CTA = one sparse block of one (b, head): the fp32 means of its 128 q
 // rows and 128 k rows, summed in the same order as the reorder kernel's fused
 // pooling (per thread over 8 rows, then over the 16 row groups), so the block
 // means -- and hence the mask -- are identical to the ones of rf_prepare.
-__global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const __nv_bfloat16* __restrict__ q,
-                                                               const __nv_bfloat16* __restrict__ k, int layout, int B,
+template <bool kF16>
+__global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const uint16_t* __restrict__ q,
+                                                               const uint16_t* __restrict__ k, int layout, int B,
                                                                int S, int N, rf_plan_t g, float* __restrict__ pooled_q,
                                                                float* __restrict__ pooled_k) {
   __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
@@ -58,7 +50,7 @@ __global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const __nv_bfloat
   const int b = bn / N, n = bn - b * N;
   const int chunk = threadIdx.x & 15;
   const int rsub = threadIdx.x >> 4;
-  const __nv_bfloat16* srcs[2] = {q, k};
+  const uint16_t* srcs[2] = {q, k};
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -67,7 +59,7 @@ __global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const __nv_bfloat
       const int s = rf_src_of_row(g, g.P_pad + blk * RF_BLOCK + p * kRowsPerPass + rsub);
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(srcs[t] + rf_token_offset(layout, B, S, N, b, n, s) +
                                                            chunk * 8));
-      acc_bf16x8(acc, u);
+      acc_half8<kF16>(acc, u);
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) red[t][rsub][chunk * 8 + i] = acc[i];
@@ -106,7 +98,7 @@ cudaError_t noalloc_scratch(void** ptr) {
   return cudaSuccess;
 }
 
-cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int layout, int B, int S, int N,
+cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int dtype, int layout, int B, int S, int N,
                                       const rf_plan_t& g, uint32_t* mask, int* kept, float* margin,
                                       cudaStream_t stream) {
   void* scratch = nullptr;
@@ -115,9 +107,9 @@ cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int layout, 
   float* pooled_q = static_cast<float*>(scratch);
   float* pooled_k = pooled_q + (size_t)B * N * g.nb * RF_HEAD_DIM;
   dim3 grid(g.nb, B * N);
-  pool_blocks_kernel<<<grid, kThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(q),
-                                                   static_cast<const __nv_bfloat16*>(k), layout, B, S, N, g,
-                                                   pooled_q, pooled_k);
+  auto kern = dtype == RF_F16 ? pool_blocks_kernel<true> : pool_blocks_kernel<false>;
+  kern<<<grid, kThreads, 0, stream>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k), layout, B, S,
+                                      N, g, pooled_q, pooled_k);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_mask(pooled_q, pooled_k, B * N, g, mask, kept, margin, stream);

@@ -5,9 +5,9 @@
 // pooling; inverse reorder at the end.  vllm-omni "RainFusion Attention":
 // 128-token key blocks are pooled (intro); the reorder groups video tokens
 // into 8x8 tiles and promotes the non-aligned rest ("Geometry handling").
-#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "rf_dtype.h"
 #include "rf_geometry.h"
 #include "rf_kernels.h"
 
@@ -19,23 +19,16 @@ constexpr int kPermThreads = 256;   // 16 rows x 16 chunks of 16 bytes per pass
 constexpr int kRowsPerPass = kPermThreads / 16;
 constexpr int kPasses = RF_BLOCK / kRowsPerPass;
 
-__device__ __forceinline__ void acc_bf16x8(float (&acc)[8], const uint4& u) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    acc[2 * i] += __uint_as_float(w[i] << 16);
-    acc[2 * i + 1] += __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
-
 // One CTA = one 128-row internal tile of one (b, head), for q, k and v.
 // Sparse tiles also write the fp32 block means of q and k.  The column sums
 // run in a fixed order (per thread over its 8 rows, then over the 16 row
-// groups), so results are deterministic.
+// groups), so results are deterministic.  Rows are 16-bit values (bf16, or
+// fp16 when kF16) copied bit for bit; only the pooling reads them as numbers.
+template <bool kF16>
 __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
-    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
-    int layout, int B, int S, int N, rf_plan_t g, __nv_bfloat16* __restrict__ q_int, __nv_bfloat16* __restrict__ k_int,
-    __nv_bfloat16* __restrict__ v_int, float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int layout, int B,
+    int S, int N, rf_plan_t g, uint16_t* __restrict__ q_int, uint16_t* __restrict__ k_int, uint16_t* __restrict__ v_int,
+    float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
   __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
   const int tile = blockIdx.x;
   const int bn = blockIdx.y;
@@ -53,8 +46,8 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
   }
   const int64_t dst_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM + chunk * 8;
 
-  const __nv_bfloat16* srcs[3] = {q, k, v};
-  __nv_bfloat16* dsts[3] = {q_int, k_int, v_int};
+  const uint16_t* srcs[3] = {q, k, v};
+  uint16_t* dsts[3] = {q_int, k_int, v_int};
 #pragma unroll
   for (int t = 0; t < 3; ++t) {
     uint4 buf[kPasses];
@@ -70,7 +63,7 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
     if (t < 2 && sparse) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int p = 0; p < kPasses; ++p) acc_bf16x8(acc, buf[p]);
+      for (int p = 0; p < kPasses; ++p) acc_half8<kF16>(acc, buf[p]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) red[t][rsub][chunk * 8 + i] = acc[i];
     }
@@ -87,9 +80,9 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
   *dst = s * (1.0f / RF_BLOCK);
 }
 
-__global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __nv_bfloat16* __restrict__ o_int, int layout,
-                                                                 int B, int S, int N, rf_plan_t g,
-                                                                 __nv_bfloat16* __restrict__ out) {
+__global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const uint16_t* __restrict__ o_int, int layout, int B,
+                                                                 int S, int N, rf_plan_t g,
+                                                                 uint16_t* __restrict__ out) {
   const int tile = blockIdx.x;
   const int bn = blockIdx.y;
   const int b = bn / N, n = bn - b * N;
@@ -109,22 +102,23 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const __nv_bflo
 
 }  // namespace
 
-cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int layout, int B, int S, int N,
-                                const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
+cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int dtype, int layout, int B, int S,
+                                int N, const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
                                 float* pooled_k, cudaStream_t stream) {
   dim3 grid(g.n_tiles, B * N);
-  permute_pool_kernel<<<grid, kPermThreads, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-      static_cast<const __nv_bfloat16*>(v), layout, B, S, N, g, static_cast<__nv_bfloat16*>(q_int),
-      static_cast<__nv_bfloat16*>(k_int), static_cast<__nv_bfloat16*>(v_int), pooled_q, pooled_k);
+  auto kern = dtype == RF_F16 ? permute_pool_kernel<true> : permute_pool_kernel<false>;
+  kern<<<grid, kPermThreads, 0, stream>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
+                                          static_cast<const uint16_t*>(v), layout, B, S, N, g,
+                                          static_cast<uint16_t*>(q_int), static_cast<uint16_t*>(k_int),
+                                          static_cast<uint16_t*>(v_int), pooled_q, pooled_k);
   return cudaGetLastError();
 }
 
 cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N, const rf_plan_t& g, void* out,
                              cudaStream_t stream) {
   dim3 grid(g.n_tiles, B * N);
-  unpermute_kernel<<<grid, kPermThreads, 0, stream>>>(static_cast<const __nv_bfloat16*>(o_int), layout, B, S, N, g,
-                                                      static_cast<__nv_bfloat16*>(out));
+  unpermute_kernel<<<grid, kPermThreads, 0, stream>>>(static_cast<const uint16_t*>(o_int), layout, B, S, N, g,
+                                                      static_cast<uint16_t*>(out));
   return cudaGetLastError();
 }
 

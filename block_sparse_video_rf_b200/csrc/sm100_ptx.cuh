@@ -200,6 +200,30 @@ __device__ __forceinline__ void mma_ts_lo_elect(uint32_t d_tmem, uint32_t a_tmem
       : "memory");
 }
 
+// kind::f8f6f4 forms of the two warp-issued MMAs (A and B fp8 e4m3).
+__device__ __forceinline__ void mma_ss_lo_elect_f8(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t hi,
+                                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 a, b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 a, {%1, %3};\n\tmov.b64 b, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a, b, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_lo), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_lo_elect_f8(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t hi,
+                                                   uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .b64 b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 b, {%2, %3};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], b, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(hi), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when all previously issued tcgen05.mma of this thread complete.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -214,12 +238,26 @@ __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
       : "memory");
 }
 
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, M x N
-// tile; b_mn_major selects an MN-major (transposed) B operand.
+// Instruction descriptor, kind::f16: fp32 accumulator, A and B both bf16
+// (bf16 = true) or both fp16, M x N tile; b_mn_major selects an MN-major
+// (transposed) B operand.
+__host__ __device__ constexpr uint32_t make_idesc_f16kind(int M, int N, bool b_mn_major, bool bf16) {
+  return (1u << 4)                          // D format: f32
+         | ((bf16 ? 1u : 0u) << 7)          // A format: 1 bf16, 0 fp16
+         | ((bf16 ? 1u : 0u) << 10)         // B format: the same
+         | ((b_mn_major ? 1u : 0u) << 16)
+         | ((uint32_t)(N >> 3) << 17)
+         | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t make_idesc_bf16(int M, int N, bool b_mn_major) {
-  return (1u << 4)                      // D format: f32
-         | (1u << 7)                    // A format: bf16
-         | (1u << 10)                   // B format: bf16
+  return make_idesc_f16kind(M, N, b_mn_major, true);
+}
+// Instruction descriptor, kind::f8f6f4: fp32 accumulator, A and B fp8 e4m3
+// (format code 0 in both fields), M x N tile.
+__host__ __device__ constexpr uint32_t make_idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4)                          // D format: f32
+         | (0u << 7)                        // A format: e4m3
+         | (0u << 10)                       // B format: e4m3
          | ((b_mn_major ? 1u : 0u) << 16)
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
@@ -334,6 +372,28 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Two fp32 -> two fp8 e4m3 codes (round to nearest even, saturating to
+// +-448), `lo` in the low byte of the 16-bit result.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// Four fp32 -> four e4m3 codes in one word, element 0 in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a0, float a1, float a2, float a3) {
+  return pack_e4m3x2(a0, a1) | (pack_e4m3x2(a2, a3) << 16);
+}
+// Two fp32 -> two 16-bit values (bf16 or fp16, round to nearest even), `lo`
+// in the low half.
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  return kF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
 }  // namespace rf

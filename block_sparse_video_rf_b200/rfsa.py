@@ -24,12 +24,15 @@ STATUS = {0: "RF_OK", 1: "RF_ERR_LAYOUT", 2: "RF_ERR_ARG", 3: "RF_ERR_UNSUPPORTE
 PLAN_FIELDS = ["S", "txt_len", "T", "H", "W", "Ha", "Wa", "n_promoted", "n_tail", "P", "P_pad", "nb", "ff", "k",
                "dense", "S_int", "n_tiles", "mask_words"]
 WS_FIELDS = ["q_int", "k_int", "v_int", "pooled_q", "pooled_k", "mask", "kept", "margin", "counter", "status",
-             "total"]
+             "q8", "k8", "v8", "scales", "vmax", "total"]
+RF_BF16, RF_F16 = 0, 1
+PRECISIONS = {"native": 0, "fp8": 1}
 
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_debug_set_wait", "rf_block_mask_noalloc", "rf_last_error_string"]
+           "rf_debug_set_wait", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
+           "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex"]
 
 
 class RfPlan(ctypes.Structure):
@@ -69,6 +72,11 @@ def _load():
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "rf_last_error_string": (ctypes.c_char_p, []),
+        "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfWsLayout)]),
+        "rf_workspace_size_ex": (Z, [I, I, I, I, I, I, I, I, I]),
+        "rf_prepare_ex": (I, [P, P, P, I, I] + geo + [I, I, F, P, Z, P]),
+        "rf_attend_ex": (I, [I, I] + geo + [I, I, F, F, P, P, Z, P]),
+        "rf_sparse_attention_ex": (I, [P, P, P, I, I] + geo + [I, I, F, F, P, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -110,60 +118,113 @@ def _scale(scale):
     return float("nan") if scale is None else float(scale)
 
 
+def _dtype(x) -> int:
+    import torch
+    if x.dtype == torch.bfloat16:
+        return RF_BF16
+    if x.dtype == torch.float16:
+        return RF_F16
+    raise RfError(2, f"q, k, v must be bfloat16 or float16 (got {x.dtype})")
+
+
+def _prec(precision: str) -> int:
+    if precision not in PRECISIONS:
+        raise RfError(2, f"precision must be one of {sorted(PRECISIONS)}")
+    return PRECISIONS[precision]
+
+
+def _plain(x, precision: str) -> bool:
+    """bf16 at native precision goes through the plain entry points."""
+    return _dtype(x) == RF_BF16 and _prec(precision) == 0
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
 def rf_plan(S: int, txt_len: int, latent, sparsity: float, block_size: int = 128) -> RfPlan:
     p = RfPlan()
     _check(LIB.rf_plan(S, txt_len, *latent, block_size, float(sparsity), ctypes.byref(p)))
     return p
 
 
-def rf_workspace_layout(B: int, N: int, D: int, plan: RfPlan) -> RfWsLayout:
+def rf_workspace_layout(B: int, N: int, D: int, plan: RfPlan, precision: str = "native") -> RfWsLayout:
     lay = RfWsLayout()
-    _check(LIB.rf_workspace_layout(B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
+    if precision == "native":
+        _check(LIB.rf_workspace_layout(B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
+    else:
+        _check(LIB.rf_workspace_layout_ex(_prec(precision), B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
     return lay
 
 
-def rf_workspace_size(B, S, N, D, txt_len, latent) -> int:
-    return int(LIB.rf_workspace_size(B, S, N, D, txt_len, *latent))
+def rf_workspace_size(B, S, N, D, txt_len, latent, precision: str = "native") -> int:
+    if precision == "native":
+        return int(LIB.rf_workspace_size(B, S, N, D, txt_len, *latent))
+    return int(LIB.rf_workspace_size_ex(_prec(precision), B, S, N, D, txt_len, *latent))
 
 
 def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: float, scale=None, out=None,
-                        block_size: int = 128, stream=None):
-    """The whole rf_v2 call on device tensors; returns ``out`` (shape and layout of q)."""
+                        block_size: int = 128, stream=None, precision: str = "native"):
+    """The whole rf_v2 call on device tensors; returns ``out`` (shape, layout and type of q).
+
+    q, k, v: bf16 or fp16; precision "native" or "fp8" (see include/rfsa.h)."""
     import torch
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
-    _check(LIB.rf_sparse_attention(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
-                                   *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
-                                   _stream(q, stream)))
+    lay = LAYOUTS.get(layout, -1)
+    if _plain(q, precision):
+        _check(LIB.rf_sparse_attention(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
+                                       float(sparsity), _scale(scale), _ptr(out), _stream(q, stream)))
+    else:
+        _check(LIB.rf_sparse_attention_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D,
+                                          txt_len, *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
+                                          None, 0, _stream(q, stream)))
     return out
 
 
 def rf_sparse_attention_ws(q, k, v, layout, txt_len, latent, sparsity, workspace, scale=None, out=None,
-                           block_size=128, stream=None):
+                           block_size=128, stream=None, precision: str = "native"):
     import torch
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
-    _check(LIB.rf_sparse_attention_ws(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
-                                      *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
-                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
-                                      _stream(q, stream)))
+    lay = LAYOUTS.get(layout, -1)
+    if _plain(q, precision):
+        _check(LIB.rf_sparse_attention_ws(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
+                                          float(sparsity), _scale(scale), _ptr(out), _ptr(workspace),
+                                          _nbytes(workspace), _stream(q, stream)))
+    else:
+        _check(LIB.rf_sparse_attention_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D,
+                                          txt_len, *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
+                                          _ptr(workspace), _nbytes(workspace), _stream(q, stream)))
     return out
 
 
-def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size=128, stream=None):
+def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size=128, stream=None,
+               precision: str = "native"):
     B, S, N, D = _dims(q, layout)
-    _check(LIB.rf_prepare(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
-                          block_size, float(sparsity), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                          _stream(q, stream)))
+    lay = LAYOUTS.get(layout, -1)
+    if _plain(q, precision):
+        _check(LIB.rf_prepare(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
+                              float(sparsity), _ptr(workspace), _nbytes(workspace), _stream(q, stream)))
+    else:
+        _check(LIB.rf_prepare_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D, txt_len,
+                                 *latent, block_size, float(sparsity), _ptr(workspace), _nbytes(workspace),
+                                 _stream(q, stream)))
 
 
-def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, block_size=128, stream=None):
+def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, block_size=128, stream=None,
+              precision: str = "native"):
     B, S, N, D = _dims(out, layout)
-    _check(LIB.rf_attend(LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent, block_size, float(sparsity),
-                         _scale(scale), _ptr(out), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                         _stream(out, stream)))
+    lay = LAYOUTS.get(layout, -1)
+    if _plain(out, precision):
+        _check(LIB.rf_attend(lay, B, S, N, D, txt_len, *latent, block_size, float(sparsity), _scale(scale),
+                             _ptr(out), _ptr(workspace), _nbytes(workspace), _stream(out, stream)))
+    else:
+        _check(LIB.rf_attend_ex(_dtype(out), _prec(precision), lay, B, S, N, D, txt_len, *latent, block_size,
+                                float(sparsity), _scale(scale), _ptr(out), _ptr(workspace), _nbytes(workspace),
+                                _stream(out, stream)))
     return out
 
 
@@ -207,10 +268,13 @@ def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
     return st.value
 
 
-def workspace_views(workspace, B, N, plan):
-    """Typed torch views of the workspace regions (for inspection and tests)."""
+def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"):
+    """Typed torch views of the workspace regions (for inspection and tests).
+
+    dtype: torch type of the internal q/k/v copies (the input type; default bf16)."""
     import torch
-    lay = rf_workspace_layout(B, N, 128, plan)
+    dtype = dtype or torch.bfloat16
+    lay = rf_workspace_layout(B, N, 128, plan, precision)
     raw = workspace.view(torch.uint8)
     heads = B * N
 
@@ -219,10 +283,20 @@ def workspace_views(workspace, B, N, plan):
         return raw[off:off + nbytes].view(dtype).view(shape)
 
     nb, words = plan.nb, plan.mask_words
-    return {
-        "q_int": view(lay.q_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
-        "k_int": view(lay.k_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
-        "v_int": view(lay.v_int, heads * plan.S_int * 128, torch.bfloat16, (B, N, plan.S_int, 128)),
+    fp8 = {}
+    if precision == "fp8":
+        n8 = heads * plan.S_int * 128
+        fp8 = {
+            "q8": view(lay.q8, n8, torch.uint8, (B, N, plan.S_int, 128)),
+            "k8": view(lay.k8, n8, torch.uint8, (B, N, plan.S_int, 128)),
+            "v8": view(lay.v8, n8, torch.uint8, (B, N, plan.n_tiles, 128, 128)),
+            "scales": view(lay.scales, 3 * heads * plan.n_tiles, torch.float32, (3, B, N, plan.n_tiles)),
+            "vmax": view(lay.vmax, heads, torch.float32, (B, N)),
+        }
+    return fp8 | {
+        "q_int": view(lay.q_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
+        "k_int": view(lay.k_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
+        "v_int": view(lay.v_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
         "pooled_q": view(lay.pooled_q, heads * nb * 128, torch.float32, (B, N, nb, 128)),
         "pooled_k": view(lay.pooled_k, heads * nb * 128, torch.float32, (B, N, nb, 128)),
         "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),
@@ -231,9 +305,9 @@ def workspace_views(workspace, B, N, plan):
     }
 
 
-def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda"):
+def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda", precision: str = "native"):
     import torch
-    n = rf_workspace_size(B, S, N, D, txt_len, latent)
+    n = rf_workspace_size(B, S, N, D, txt_len, latent, precision)
     if n == 0:
         raise RfError(2, "bad arguments for the workspace size")
     return torch.empty(n, dtype=torch.uint8, device=device)

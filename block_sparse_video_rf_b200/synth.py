@@ -132,8 +132,9 @@ def _rope(w: Workload, x, device):
     return torch.cat([a * c - b * s, a * s + b * c, x[..., 96:]], dim=-1)
 
 
-def make_inputs(w: Workload, device="cpu"):
-    """Seeded bf16 q, k, v in ``w.layout`` ([B,S,N,D] or [B,N,S,D])."""
+def make_inputs(w: Workload, device="cpu", dtype=torch.bfloat16):
+    """Seeded q, k, v in ``w.layout`` ([B,S,N,D] or [B,N,S,D]), rounded to
+    ``dtype`` (bfloat16 or float16) from the same fp32 draws."""
     device = torch.device(device)
     gen = torch.Generator(device=device)
     gen.manual_seed(1000 + w.seed)
@@ -151,7 +152,7 @@ def make_inputs(w: Workload, device="cpu"):
             q, k = q + sm, k + sm
         elif w.kind == "rope":
             q, k = _rope(w, q, device), _rope(w, k, device)
-        outs.append((q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16)))
+        outs.append((q.to(dtype), k.to(dtype), v.to(dtype)))
         del q, k, v
     q, k, v = (torch.stack([o[i] for o in outs], 0) for i in range(3))   # [B,S,N,D]
     if w.layout == "BNSD":

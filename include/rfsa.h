@@ -9,9 +9,10 @@
  * page "RainFusion Attention" (intro; "Configuration"; "Geometry handling").
  *
  * Conventions for every entry point:
- *  - q, k, v, out: DEVICE pointers to bf16, caller-owned, contiguous, in the
- *    layout given (RF_BSND = [B, S, N, D], RF_BNSD = [B, N, S, D]); out has
- *    the shape and layout of q and must not alias q, k or v.
+ *  - q, k, v, out: DEVICE pointers to bf16 (fp16 through the _ex entry
+ *    points with dtype RF_F16), caller-owned, contiguous, in the layout
+ *    given (RF_BSND = [B, S, N, D], RF_BNSD = [B, N, S, D]); out has the
+ *    shape, layout and element type of q and must not alias q, k or v.
  *  - D and block_size must be 128.
  *  - S = txt_len + latent_t * latent_h * latent_w.  latent (0, 0, 0) means
  *    "no video geometry": the call is dense softmax attention over S.
@@ -39,6 +40,21 @@ extern "C" {
 #endif
 
 typedef enum { RF_BSND = 0, RF_BNSD = 1 } rf_layout_t;
+
+/* Element type of q, k, v and out (lite_boost.ops.sparse_attention accepts
+ * float16 and bfloat16). */
+typedef enum { RF_BF16 = 0, RF_F16 = 1 } rf_dtype_t;
+
+/* Arithmetic of the attention's two products.  RF_PREC_NATIVE: Q K^T and P V
+ * on the tensor cores in the input type (bf16 or fp16) with fp32
+ * accumulation.  RF_PREC_FP8: Q, K and V quantised to fp8 e4m3 with one
+ * fp32 scale per 128-row block of the internal layout (per tensor and head:
+ * scale = amax(|x|) over the block / 448, code = e4m3 round-to-nearest-even
+ * with saturation of x * (448 / amax), all-zero blocks get scale 0); Q K^T
+ * and P V then run as e4m3 x e4m3 tensor-core products with fp32
+ * accumulation, P quantised to e4m3 per tile.  The block mask is the same in
+ * both: it is computed from the unquantised inputs. */
+typedef enum { RF_PREC_NATIVE = 0, RF_PREC_FP8 = 1 } rf_precision_t;
 
 typedef enum {
   RF_OK = 0,
@@ -76,14 +92,21 @@ typedef struct {
 } rf_plan_t;
 
 /* Byte offsets of the regions of a workspace (all 256-byte aligned).
- * q_int/k_int/v_int: bf16 [B, N, S_int, 128]; pooled_q/pooled_k: fp32
+ * q_int/k_int/v_int: 16-bit (input type) [B, N, S_int, 128]; pooled_q/pooled_k: fp32
  * [B, N, nb, 128] (block means); mask: uint32 [B, N, nb, mask_words], bit j
  * of row i set when query block i reads key block j; kept: int32 [B, N, nb]
  * (bits set per row); margin: fp32 [B, N, nb] (relative gap between the
  * k-th and (k+1)-th block score of the row, +inf when not defined);
- * counter: int32 work counter; status: int32 device status word. */
+ * counter: int32 work counter; status: int32 device status word.
+ * Only with RF_PREC_FP8 (zero-sized otherwise): q8/k8: e4m3 codes
+ * [B, N, S_int, 128]; v8: e4m3 codes of V with each 128-row block stored
+ * transposed ([B, N, n_tiles, 128 channels, 128 rows]); scales: fp32
+ * [3 (q, k, v), B, N, n_tiles]; vmax: fp32 [B, N], the largest V block scale
+ * of each head. */
 typedef struct {
-  size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status, total;
+  size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status;
+  size_t q8, k8, v8, scales, vmax;
+  size_t total;
 } rf_ws_layout_t;
 
 /* Host-only: validate a geometry and fill *plan.  No CUDA call. */
@@ -95,6 +118,13 @@ rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* plan, rf_w
 
 /* Host-only: bytes of workspace rf_sparse_attention_ws needs (0 on bad arguments). */
 size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int latent_t, int latent_h, int latent_w);
+
+/* Host-only: the same for a given precision (RF_PREC_FP8 adds the e4m3
+ * tensors and scales). */
+rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D, const rf_plan_t* plan,
+                                   rf_ws_layout_t* layout);
+size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int latent_t,
+                            int latent_h, int latent_w);
 
 /* The whole rf_v2 call, with a workspace cached by the library per device
  * (grown with cudaMalloc on first use of a larger shape; never shrunk). */
@@ -125,8 +155,28 @@ rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_le
                       int latent_w, int block_size, float sparsity, float scale, void* out, void* workspace,
                       size_t ws_bytes, void* stream);
 
-/* Inverse reorder alone: o_int bf16 [B, N, S_int, 128] (internal order) ->
- * out in the caller's layout.  Pad rows are skipped. */
+/* rf_prepare / rf_attend / rf_sparse_attention_ws for any input type and
+ * precision (the plain entry points are these with RF_BF16, RF_PREC_NATIVE).
+ * The workspace must come from rf_workspace_size_ex for the same precision;
+ * rf_sparse_attention_ex takes workspace = NULL (ws_bytes ignored) to use the
+ * library's cached workspace.  Invalid dtype or precision: RF_ERR_ARG.
+ * RF_PREC_FP8 stage 1 also quantises the reordered q, k, v (q8/k8/v8,
+ * scales, vmax); its stage 2 reads only those. */
+rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype, rf_precision_t precision,
+                          rf_layout_t layout, int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
+                          int latent_w, int block_size, float sparsity, void* workspace, size_t ws_bytes,
+                          void* stream);
+rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                         int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
+                         float scale, void* out, void* workspace, size_t ws_bytes, void* stream);
+rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype,
+                                   rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                                   int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
+                                   float sparsity, float scale, void* out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* Inverse reorder alone: o_int [B, N, S_int, 128] of 16-bit values (internal
+ * order) -> out in the caller's layout.  Pad rows are skipped. */
 rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len,
                          int latent_t, int latent_h, int latent_w, void* out, void* stream);
 

@@ -28,3 +28,4 @@ from .rf_v2 import (  # noqa: F401
     to_bnsd,
     from_bnsd,
 )
+from . import fp8  # noqa: F401

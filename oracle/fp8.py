@@ -1,0 +1,153 @@
+"""fp8 e4m3 operands of the attention (the fp8 precision), written out plainly.
+
+TEST INFRASTRUCTURE ONLY: the product path never imports this module.
+
+Sources: [SA] MindSpore Lite "lite_boost.ops.sparse_attention" lists an fp8
+precision for the attention; the pages fix no scaling rule.  READING (the
+CUDA library takes the same one; the two share no code):
+
+  R14 Q, K and V are quantised per 128-row block of the internal layout
+      (the attention's tile: each prefix tile, padded with zero rows, and
+      each sparse block), per tensor and (b, head):
+        amax  = max |x| over the block's 128 x 128 values;
+        inv   = fp32(448 / amax)           (448: the largest finite e4m3);
+        code  = e4m3(fp32(x * inv))        round to nearest, ties to even,
+                                           saturating at +-448;
+        scale = fp32(amax / 448);
+      an all-zero block has scale 0 and codes 0.  The dequantised operand is
+      e4m3_value(code) * scale.  The block mask is computed from the
+      unquantised inputs, exactly as at native precision.
+  R15 The fp8 attention output is the oracle's attention (fp64) over the
+      dequantised Q, K and V.  The tensor-core path also rounds P to e4m3
+      before P V; that rounding is not modelled here and is covered by the
+      fp8 tolerance of the tests.
+
+The e4m3 format (OCP 8-bit floating point, E4M3): 1 sign bit, 4 exponent
+bits with bias 7, 3 mantissa bits; exponent field 0 holds subnormals
+m * 2^-9; no infinities; exponent 15 with mantissa 7 is NaN, so the largest
+finite value is 1.75 * 2^8 = 448.
+
+Parity: the value table and the rounding are pinned against torch's
+float8_e4m3fn conversion and against a brute-force nearest-value search in
+``tests/test_oracle_fp8.py``.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import rf_v2
+
+E4M3_MAX = 448.0
+
+
+def e4m3_values() -> np.ndarray:
+    """The value of each of the 256 codes (fp64; NaN for the two NaN codes)."""
+    vals = np.empty(256, dtype=np.float64)
+    for code in range(256):
+        sign = -1.0 if code & 0x80 else 1.0
+        e = (code >> 3) & 0xF
+        m = code & 0x7
+        if e == 0xF and m == 0x7:
+            vals[code] = np.nan
+        elif e == 0:
+            vals[code] = sign * m * 2.0 ** -9
+        else:
+            vals[code] = sign * (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+_VALUES = e4m3_values()
+
+
+def _binade(a: np.ndarray) -> np.ndarray:
+    """floor(log2(a)) for a > 0, exactly (frexp: a = m 2^p with m in [0.5, 1))."""
+    return np.frexp(a)[1].astype(np.int64) - 1
+
+
+def e4m3_round(x) -> np.ndarray:
+    """Codes (uint8) of fp32 values: round to nearest, ties to even mantissa,
+    |x| above 448 saturating to 448 (R14), negative values that round to zero
+    giving -0 (code 0x80).  NaN inputs are not expected."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    pos = a > 0
+    e = np.where(pos, np.maximum(_binade(np.where(pos, a, 1.0)), -6), 0)   # below 2^-6: subnormal spacing 2^-9
+    quantum = np.ldexp(1.0, e - 3)                                           # 3 mantissa bits
+    q = np.round(a / quantum) * quantum                                      # np.round: halves to even
+    q = np.where(a >= E4M3_MAX, E4M3_MAX, np.minimum(q, E4M3_MAX))
+    # code of the rounded magnitude
+    normal = q >= 2.0 ** -6
+    eq = np.where(normal, _binade(np.where(normal, q, 1.0)), 0)
+    mant = np.where(normal, q / np.ldexp(1.0, eq) * 8 - 8, q / 2.0 ** -9)
+    code = np.where(normal, ((eq + 7) << 3), 0) + np.round(mant).astype(np.int64)
+    code = np.where(np.signbit(x), code | 0x80, code)                      # the sign survives underflow: -0
+    return code.astype(np.uint8)
+
+
+def quantize_block(x: np.ndarray):
+    """R14 for one block: (codes uint8 like x, scale fp32)."""
+    xf = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(xf))) if xf.size else np.float32(0.0)
+    if amax == 0:
+        return np.zeros(xf.shape, dtype=np.uint8), np.float32(0.0)
+    inv = np.float32(np.float32(E4M3_MAX) / amax)
+    v = (xf * inv).astype(np.float32)
+    return e4m3_round(v), np.float32(amax / np.float32(E4M3_MAX))
+
+
+def dequantize(codes: np.ndarray, scale) -> np.ndarray:
+    return _VALUES[np.asarray(codes, dtype=np.int64)] * float(scale)
+
+
+def internal_tiles(g: rf_v2.Geometry) -> list[np.ndarray]:
+    """Token indices of each 128-row block of the internal layout, -1 for the
+    zero pad rows: the prefix in order (the whole sequence when dense),
+    padded to a multiple of 128, then the sparse blocks."""
+    pre = np.arange(g.S) if g.dense else np.asarray(g.prefix, dtype=np.int64)
+    pad = (-len(pre)) % rf_v2.BLOCK
+    rows = np.concatenate([pre, -np.ones(pad, dtype=np.int64)])
+    tiles = [rows[i:i + rf_v2.BLOCK] for i in range(0, len(rows), rf_v2.BLOCK)]
+    if not g.dense:
+        tiles += [np.asarray(b, dtype=np.int64) for b in g.blocks]
+    return tiles
+
+
+def quantize_head(xh: np.ndarray, g: rf_v2.Geometry):
+    """R14 for one (b, head) tensor [S, D] in token order: returns the
+    dequantised tensor (fp64, token order), the codes per internal tile
+    ([n_tiles, 128, D], pad rows 0) and the scales [n_tiles] (fp32)."""
+    S, D = xh.shape
+    tiles = internal_tiles(g)
+    xq = np.zeros((S, D), dtype=np.float64)
+    codes = np.zeros((len(tiles), rf_v2.BLOCK, D), dtype=np.uint8)
+    scales = np.zeros(len(tiles), dtype=np.float32)
+    for t, rows in enumerate(tiles):
+        valid = rows >= 0
+        block = np.zeros((rf_v2.BLOCK, D), dtype=np.float32)
+        block[valid] = xh[rows[valid]]
+        c, s = quantize_block(block)
+        codes[t], scales[t] = c, s
+        xq[rows[valid]] = dequantize(c[valid], s)
+    return xq, codes, scales
+
+
+def rf_sparse_attention_fp8(q, k, v, layout: str, txt_len: int, latent, sparsity: float,
+                            scale: float | None = None):
+    """The whole call at fp8 precision (R14, R15): returns (out fp64 in the
+    caller's layout, mask, margin, geometry)."""
+    if not (np.isfinite(sparsity) and 0.0 <= sparsity <= 1.0):
+        raise ValueError("sparsity must be finite and in [0, 1]")
+    qb, kb, vb = (rf_v2.to_bnsd(np.asarray(a), layout) for a in (q, k, v))
+    B, N, S, D = qb.shape
+    if scale is None:
+        scale = D ** -0.5
+    T, H, W = latent
+    g = rf_v2.geometry(S, txt_len, T, H, W)
+    mask, margin = rf_v2.build_mask(qb, kb, g, sparsity)
+    out = np.empty((B, N, S, D), dtype=np.float64)
+    for b in range(B):
+        for n in range(N):
+            qd, kd, vd = (quantize_head(x[b, n], g)[0] for x in (qb, kb, vb))
+            out[b, n] = rf_v2.attention_rows(qd, kd, vd, g, mask[b, n] if not g.dense else None, scale)
+    return rf_v2.from_bnsd(out, layout), mask, margin, g

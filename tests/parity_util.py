@@ -63,6 +63,27 @@ def assert_close(got, ref, what=""):
     return mx, mean
 
 
+def fp8_bounds(v_deq: np.ndarray):
+    """Output tolerance of the fp8 path against the oracle over the
+    dequantised operands, from the arithmetic the oracle leaves out: P is
+    rounded to e4m3 (3 mantissa bits, round to nearest even), a relative
+    error of at most 2^-4 per weight.  An output row is a weighted mean of V
+    rows, so its error is at most 2^-4 * max |V| if every weight errs the
+    same way; with errors of mixed sign and an average size well below
+    2^-5, the mean error stays under 2^-6 * mean |V|."""
+    a = np.abs(np.asarray(v_deq, dtype=np.float64))
+    return 2.0 ** -4 * float(a.max()), 2.0 ** -6 * float(a.mean())
+
+
+def assert_close_fp8(got, ref, v_deq, what=""):
+    mx_tol, mean_tol = fp8_bounds(v_deq)
+    mx, mean = compare_outputs(got, ref)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    assert mx <= mx_tol and mean <= mean_tol, \
+        f"{what}: max-abs {mx:.3e} (<= {mx_tol:.3e}), mean-abs {mean:.3e} (<= {mean_tol:.3e})"
+    return mx, mean
+
+
 def mask_mismatch(gpu_words: np.ndarray, ref_bool: np.ndarray, ref_margin: np.ndarray):
     """Rows whose mask differs, split into excused near-ties and real mismatches."""
     nb = ref_bool.shape[-1]

@@ -122,3 +122,35 @@ def test_workspace_layout_is_aligned_and_sized(rfsa):
     tensor = 56 * 62848 * 128 * 2
     assert lay.k_int - lay.q_int >= tensor and lay.total > 3 * tensor
     assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42)) == lay.total
+
+
+def test_ex_entry_points_validate_dtype_and_precision(rfsa):
+    L = rfsa.LIB
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    geo = (0, 1, 4096, 2, 128, 0, 4, 32, 32, 128, 0.5, 0.0)
+    # dtype 5 / precision 3 -> RF_ERR_ARG before any CUDA call
+    assert L.rf_sparse_attention_ex(fake, fake, fake, 5, 0, *geo, P(0x2000), None, 0, None) == 2
+    assert b"dtype" in L.rf_last_error_string()
+    assert L.rf_sparse_attention_ex(fake, fake, fake, 0, 3, *geo, P(0x2000), None, 0, None) == 2
+    assert b"precision" in L.rf_last_error_string()
+    assert L.rf_prepare_ex(fake, fake, fake, 1, 1, *geo[:-1], P(0x10000), 16, None) == 5   # fp8 workspace too small
+    assert L.rf_attend_ex(1, 9, *geo, P(0x2000), P(0x10000), 1 << 40, None) == 2
+    assert rfsa.rf_workspace_size(1, 4096, 2, 128, 0, (4, 32, 32), precision="fp8") > 0
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_workspace_layout(1, 2, 128, rfsa.rf_plan(4096, 0, (4, 32, 32), 0.5), precision="fp4")
+
+
+def test_fp8_workspace_layout(rfsa):
+    p = rfsa.rf_plan(62752, 256, (62, 24, 42), 0.8)
+    nat = rfsa.rf_workspace_layout(1, 56, 128, p)
+    lay = rfsa.rf_workspace_layout(1, 56, 128, p, precision="fp8")
+    offs = [getattr(lay, f) for f in rfsa.WS_FIELDS]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    codes = 56 * 62848 * 128
+    assert lay.k8 - lay.q8 >= codes and lay.v8 - lay.k8 >= codes and lay.scales - lay.v8 >= codes
+    assert lay.vmax - lay.scales >= 3 * 56 * p.n_tiles * 4 and lay.total - lay.vmax >= 56 * 4
+    # the native layout is the same up to the fp8 regions, which it leaves empty
+    assert [getattr(nat, f) for f in rfsa.WS_FIELDS[:10]] == offs[:10]
+    assert nat.q8 == nat.k8 == nat.v8 == nat.scales == nat.vmax == nat.total
+    assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42), precision="fp8") == lay.total

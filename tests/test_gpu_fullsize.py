@@ -2,32 +2,34 @@
 times, on sampled heads and rows the oracle computes one by one.
 
 The mask of each sampled head is compared bit for bit (near-ties excused);
-output rows are compared within max-abs 2e-2 / mean-abs 2e-3.  Sampled rows
-cover text rows, promoted rows, the partial prefix tile, first-frame blocks
-and sparse blocks."""
+output rows are compared within max-abs 2e-2 / mean-abs 2e-3 (bf16, fp16),
+or against the oracle over the dequantised operands within the fp8 bounds
+of ``parity_util.fp8_bounds``.  Sampled rows cover text rows, promoted rows,
+the partial prefix tile, first-frame blocks and sparse blocks."""
 
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from parity_util import assert_close, mask_mismatch, unpack_mask
+from oracle import fp8
+from parity_util import assert_close, assert_close_fp8, mask_mismatch, unpack_mask
 
 pytestmark = pytest.mark.gpu
 
 
-def _run(name, **over):
+def _run(name, dtype=torch.bfloat16, precision="native", **over):
     from block_sparse_video_rf_b200 import rfsa, synth
     w = synth.workload(name, **over)
-    q, k, v = synth.make_inputs(w, device="cuda")
+    q, k, v = synth.make_inputs(w, device="cuda", dtype=dtype)
     sp = np.float32(w.sparsity)
-    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent)
+    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent, precision=precision)
     out = torch.empty_like(q)
-    rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws)
-    rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws)
+    rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws, precision=precision)
+    rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws, precision=precision)
     plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, sp)
     assert rfsa.rf_read_status(ws, w.B, w.N, 128, plan) == 0
-    views = rfsa.workspace_views(ws, w.B, w.N, plan)
+    views = rfsa.workspace_views(ws, w.B, w.N, plan, dtype=dtype, precision=precision)
     return w, q, k, v, out, plan, views
 
 
@@ -54,10 +56,14 @@ def _sample_rows(g, rng, per_kind=6):
     ("minimax", {"sparsity": 0.9}, (11,)),
     ("minimax", {"sparsity": 0.0}, (40,)),
     ("wan", {}, (0, 39)),
+    ("minimax", {"dtype": torch.float16}, (7,)),
+    ("minimax", {"precision": "fp8"}, (5, 50)),
 ])
 def test_full_size_sampled(name, over, heads):
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
+    over = dict(over)
+    precision = over.get("precision", "native")
     w, q, k, v, out, plan, views = _run(name, **over)
     g = oracle.geometry(w.S, w.txt_len, *w.latent)
     assert plan.nb == g.nb and plan.P == len(g.prefix)
@@ -71,6 +77,11 @@ def test_full_size_sampled(name, over, heads):
         assert bad == 0, f"head {n}: {bad} mask rows differ outside near-ties ({excused} excused, {near} near-ties)"
         gpu_mask = unpack_mask(words[0, n], g.nb)
         rows = _sample_rows(g, rng)
-        ref = oracle.attention_rows(qh, kh, vh, g, gpu_mask, scale, rows=rows)
         got = out[0, torch.from_numpy(rows).cuda(), n].float().cpu().numpy()
-        assert_close(got, ref, f"{name} head {n}")
+        if precision == "fp8":
+            qd, kd, vd = (fp8.quantize_head(x, g)[0] for x in (qh, kh, vh))
+            ref = oracle.attention_rows(qd, kd, vd, g, gpu_mask, scale, rows=rows)
+            assert_close_fp8(got, ref, vd, f"{name} fp8 head {n}")
+        else:
+            ref = oracle.attention_rows(qh, kh, vh, g, gpu_mask, scale, rows=rows)
+            assert_close(got, ref, f"{name} head {n}")
