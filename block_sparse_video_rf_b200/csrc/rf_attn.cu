@@ -18,9 +18,11 @@
 // warps, so that while the softmax of one slot runs the tensor pipe works on
 // the other slot's MMAs:
 //   warps 0-3   slot 0, warps 4-7 slot 1: thread = query row (TMEM lane);
-//               online softmax in exp2 with a lazily updated running max;
-//               most exponentials on the MUFU unit, one pair in four on the
-//               FMA pipe (polynomial); P is written over the first columns of
+//               online softmax in exp2 with a lazily updated running max
+//               (a tile computes its own maximum only when its P would
+//               exceed the format's range); most exponentials on the MUFU
+//               unit, one pair in four (fp8: three) on the FMA pipe
+//               (polynomial); P is written over the first columns of
 //               the slot's S; at the end of a unit the same threads write
 //               O / l in the caller's type and layout.  The slot's first warp
 //               also issues its MMAs (one elected lane):
@@ -71,7 +73,7 @@ constexpr int kSlotWarps = 4;                            // softmax warps per sl
 constexpr uint32_t kRegsSoftmax = 216, kRegsControl = 64;
 constexpr int kBoxBytes = RF_BLOCK * 128;                // one TMA box: 128 rows x 128 bytes
 constexpr uint32_t kTmemCols = 512;
-constexpr int kPolyEvery = 4;                            // pair i uses the polynomial when i % 4 == 3
+
 constexpr float kRescaleThreshold = 8.0f;                // log2 units
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
@@ -86,6 +88,9 @@ struct Cfg {
   static constexpr int kVStages = kFp8 ? 2 : 1;
   static constexpr int kSteps = kFp8 ? 4 : 8;            // MMAs per product over 128 (K 32 or 16 each)
   static constexpr int kPCols = kFp8 ? 32 : 64;          // TMEM columns of P
+  // exponent pair i runs the polynomial on the FMA pipe when i % kPolyEvery == kPolyEvery - 1
+  // (the rest on MUFU): measured best split for each path
+  static constexpr int kPolyEvery = kFp8 ? 3 : 4;
   static constexpr uint32_t kIdescQK =
       kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, false, !kF16);
   static constexpr uint32_t kIdescPV =
@@ -364,55 +369,15 @@ __device__ __forceinline__ bool slot_vote(int id, bool ok) {
 }
 
 // ---------------------------------------------------------------- softmax of one tile
-// Thread = query row.  Reads the row's 128 scores from S, scales them by c
-// (log2 units), updates the running max m_use (lazily: only when a score
-// exceeds it by more than the threshold, then O and l are rescaled), adds
-// the tile's sum of P (times ir) to l and writes P = 2^(s c - m_use + lr)
-// over the first columns of S: as 64 words of two 16-bit values, or (fp8)
-// 32 words of four e4m3 codes.  `p_valid` < 128 masks the keys past the
-// prefix's end.
+// P = 2^(s c + off) for the row's 128 scores s (already in registers), with
+// the tile's sum of P; writes the packed P words.
 template <class C>
-__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool first, int p_valid, float c, float lr,
-                                             float ir, float& m_use, float& l) {
+__device__ __forceinline__ float exp_tile(const uint32_t (&s)[4][32], float c, float off, int p_valid,
+                                          uint32_t (&pk)[C::kPCols]) {
   const uint64_t c2 = f2_pack(c, c);
-  uint32_t s[4][32];
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
-  tmem_wait_ld();
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
-
-  const bool partial = p_valid < RF_BLOCK;
-  if (partial) {
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (32 * q4 + e >= p_valid) s[q4][e] = __float_as_uint(-CUDART_INF_F);
-  }
-  float mx8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-    for (int e = 0; e < 32; e += 2)
-      mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
-  const float mx = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-  const float mx_s = mx * c;
-  float alpha = 1.f;
-  bool rescale = false;
-  if (first) {
-    m_use = mx_s;
-  } else if (mx_s > m_use + kRescaleThreshold) {
-    alpha = ex2_approx(m_use - mx_s);
-    m_use = mx_s;
-    rescale = true;
-  }
-  const float off = lr - m_use;
   const uint64_t negm = f2_pack(off, off);
+  const bool partial = p_valid < RF_BLOCK;
   uint64_t sum2[4] = {0, 0, 0, 0};
-  uint32_t pk[C::kPCols];
   float hold0 = 0.f, hold1 = 0.f;   // fp8: the first pair of a 4-key word
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4)
@@ -421,7 +386,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
       const int i = 16 * q4 + (e >> 1);     // pair index 0..63
       const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), c2, negm);
       uint64_t p2;
-      if ((i % kPolyEvery) == kPolyEvery - 1) {
+      if ((i % C::kPolyEvery) == C::kPolyEvery - 1) {
         p2 = exp2_poly_x2(x2);
       } else {
         float x0, x1;
@@ -450,7 +415,75 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
   float s0, s1, s2, s3;
   f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
   f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
-  l = l * alpha + ((s0 + s1) + (s2 + s3)) * ir;
+  return (s0 + s1) + (s2 + s3);
+}
+
+template <class C>
+__device__ __forceinline__ void load_scores(uint32_t tS, int p_valid, uint32_t (&s)[4][32]) {
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
+  if (p_valid < RF_BLOCK) {
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (32 * q4 + e >= p_valid) s[q4][e] = __float_as_uint(-CUDART_INF_F);
+  }
+}
+
+__device__ __forceinline__ float row_max(const uint32_t (&s)[4][32]) {
+  float mx8[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+    for (int e = 0; e < 32; e += 2)
+      mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
+  return max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+}
+
+// Thread = query row.  Reads the row's 128 scores from S and writes P =
+// 2^(s c - m_use + lr) over the first columns of S (64 words of two 16-bit
+// values, or (fp8) 32 words of four e4m3 codes), adding the tile's sum of P
+// times ir to l.  The running max m_use (log2 units) is set by the unit's
+// first tile; later tiles use it as it stands and look at their own maximum
+// only when their sum shows a P above the format's limit (sum > kSumLimit,
+// or not finite): then the scores are read again, m_use moves up to the
+// tile's maximum if that exceeds it by more than the threshold (rescaling O
+// and l), and P is computed again.  `p_valid` < 128 masks the keys past the
+// prefix's end.
+template <class C>
+__device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool first, int p_valid, float c, float lr,
+                                             float ir, float& m_use, float& l) {
+  // P above this sum may exceed 448 (e4m3) / lose fp32 headroom (16-bit)
+  constexpr float kSumLimit = C::kFp8 ? 448.f : 65536.f;
+  uint32_t s[4][32];
+  uint32_t pk[C::kPCols];
+  load_scores<C>(tS, p_valid, s);
+  float alpha = 1.f;
+  bool rescale = false;
+  float tsum;
+  if (first) {
+    m_use = row_max(s) * c;
+    tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+  } else {
+    tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+    if (__any_sync(0xFFFFFFFFu, !(tsum <= kSumLimit))) {
+      load_scores<C>(tS, p_valid, s);
+      const float mx_s = row_max(s) * c;
+      if (mx_s > m_use + kRescaleThreshold) {
+        alpha = ex2_approx(m_use - mx_s);
+        m_use = mx_s;
+        rescale = true;
+      }
+      tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+    }
+  }
+  l = l * alpha + tsum * ir;
   if (__any_sync(0xFFFFFFFFu, rescale)) {
     // O holds the tiles before this one: their P V completed before this
     // tile's S = Q K^T was issued.

@@ -195,3 +195,30 @@ def test_repeat_calls_are_deterministic(rfsa):
     b = rfsa.rf_sparse_attention(q, k, v, w.layout, w.txt_len, w.latent, 0.8)
     torch.cuda.synchronize()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+@pytest.mark.parametrize("precision", ["native", "fp8"])
+def test_running_max_that_grows_after_the_first_tile(rfsa, precision):
+    # The text prefix tile comes first and holds small scores; the video keys are
+    # scaled up, so later tiles exceed the first tile's maximum by far and the
+    # kernel must raise its running max (and rescale O and l) mid-row.
+    from oracle import fp8
+    from parity_util import assert_close_fp8
+    w, q, k, v = _inputs("tiny", txt_len=128, latent=(4, 32, 32), N=2, seed=31)
+    k = k.clone()
+    k[:, w.txt_len:] *= 6.0
+    out = rfsa.rf_sparse_attention(q, k, v, w.layout, w.txt_len, w.latent, np.float32(w.sparsity),
+                                   precision=precision)
+    torch.cuda.synchronize()
+    if precision == "native":
+        ref, _, _, _ = oracle.rf_sparse_attention(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent,
+                                                  float(np.float32(w.sparsity)))
+        assert_close(to_np(out), ref, "growing max")
+    else:
+        ref, _, _, g = fp8.rf_sparse_attention_fp8(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent,
+                                                   float(np.float32(w.sparsity)))
+        vb = to_bnsd_np(v, w.layout)
+        for n in range(w.N):
+            vd = fp8.quantize_head(vb[0, n], g)[0]
+            assert_close_fp8(to_bnsd_np(out, w.layout)[0, n], oracle.to_bnsd(ref, w.layout)[0, n], vd,
+                             f"growing max fp8 n{n}")
