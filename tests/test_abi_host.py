@@ -154,3 +154,12 @@ def test_fp8_workspace_layout(rfsa):
     assert [getattr(nat, f) for f in rfsa.WS_FIELDS[:10]] == offs[:10]
     assert nat.q8 == nat.k8 == nat.v8 == nat.scales == nat.vmax == nat.total
     assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42), precision="fp8") == lay.total
+
+
+def test_block_count_limit(rfsa):
+    # 4096 sparse blocks are accepted, more are not (RF_ERR_UNSUPPORTED)
+    p = rfsa.rf_plan(64 * 64 * 128, 0, (128, 64, 64), 0.5)
+    assert p.nb == 4096
+    with pytest.raises(rfsa.RfError) as e:
+        rfsa.rf_plan(64 * 64 * 129, 0, (129, 64, 64), 0.5)     # 4128 blocks
+    assert e.value.code == 3

@@ -222,3 +222,33 @@ def test_running_max_that_grows_after_the_first_tile(rfsa, precision):
             vd = fp8.quantize_head(vb[0, n], g)[0]
             assert_close_fp8(to_bnsd_np(out, w.layout)[0, n], oracle.to_bnsd(ref, w.layout)[0, n], vd,
                              f"growing max fp8 n{n}")
+
+
+@pytest.mark.parametrize("layout", ["BSND", "BNSD"])
+def test_batch_of_two(rfsa, layout):
+    # B = 2: every (b, head) has its own mask and work units; the permutation is shared
+    w, q, k, v = _inputs("tiny", B=2, N=2, txt_len=37, latent=(6, 24, 40), sparsity=0.6, layout=layout, seed=41)
+    ws, plan, views = _run_prepare(rfsa, w, q, k, v)
+    g, mask, margin = _oracle_mask(w, q, k)
+    bad, excused, near = mask_mismatch(views["mask"].cpu().numpy().view(np.uint32), mask, margin)
+    assert bad == 0
+    out = torch.empty_like(q)
+    views["mask"].copy_(torch.from_numpy(pack_mask(mask).view(np.int32)).cuda())
+    rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, np.float32(w.sparsity), ws)
+    assert rfsa.rf_read_status(ws, w.B, w.N, 128, plan) == 0
+    qb, kb, vb = (to_bnsd_np(t, w.layout) for t in (q, k, v))
+    got = to_bnsd_np(out, w.layout)
+    for b in range(2):
+        for n in range(2):
+            ref = oracle.attention_rows(qb[b, n], kb[b, n], vb[b, n], g, mask[b, n], w.D ** -0.5)
+            assert_close(got[b, n], ref, f"B=2 b{b} n{n}")
+
+
+def test_sparsity_one_keeps_prefix_and_first_frame(rfsa):
+    # sparsity 1 keeps no top-k block: sparse rows read the prefix and the forced first-frame blocks only
+    w, q, k, v = _inputs("tiny", txt_len=64, latent=(4, 32, 32), sparsity=1.0, N=2, seed=42)
+    out = rfsa.rf_sparse_attention(q, k, v, w.layout, w.txt_len, w.latent, 1.0)
+    torch.cuda.synchronize()
+    ref, mask, _, g = oracle.rf_sparse_attention(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent, 1.0)
+    assert (mask[0, :, g.ff:].sum(-1) == g.ff).all()
+    assert_close(to_np(out), ref, "s=1")
