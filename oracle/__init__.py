@@ -16,6 +16,7 @@ from .rf_v2 import (  # noqa: F401
     TILE,
     Geometry,
     geometry,
+    is_dense,
     kept_count,
     pool_blocks,
     block_scores,

@@ -100,25 +100,28 @@ def dequantize(codes: np.ndarray, scale) -> np.ndarray:
     return _VALUES[np.asarray(codes, dtype=np.int64)] * float(scale)
 
 
-def internal_tiles(g: rf_v2.Geometry) -> list[np.ndarray]:
+def internal_tiles(g: rf_v2.Geometry, dense: bool | None = None) -> list[np.ndarray]:
     """Token indices of each 128-row block of the internal layout, -1 for the
     zero pad rows: the prefix in order (the whole sequence when dense),
-    padded to a multiple of 128, then the sparse blocks."""
-    pre = np.arange(g.S) if g.dense else np.asarray(g.prefix, dtype=np.int64)
+    padded to a multiple of 128, then the sparse blocks.  ``dense``
+    overrides g.dense (a call is dense when either geometry is, R9)."""
+    dense = g.dense if dense is None else dense
+    pre = np.arange(g.S) if dense else np.asarray(g.prefix, dtype=np.int64)
     pad = (-len(pre)) % rf_v2.BLOCK
     rows = np.concatenate([pre, -np.ones(pad, dtype=np.int64)])
     tiles = [rows[i:i + rf_v2.BLOCK] for i in range(0, len(rows), rf_v2.BLOCK)]
-    if not g.dense:
+    if not dense:
         tiles += [np.asarray(b, dtype=np.int64) for b in g.blocks]
     return tiles
 
 
-def quantize_head(xh: np.ndarray, g: rf_v2.Geometry):
+def quantize_head(xh: np.ndarray, g: rf_v2.Geometry, dense: bool | None = None):
     """R14 for one (b, head) tensor [S, D] in token order: returns the
     dequantised tensor (fp64, token order), the codes per internal tile
-    ([n_tiles, 128, D], pad rows 0) and the scales [n_tiles] (fp32)."""
+    ([n_tiles, 128, D], pad rows 0) and the scales [n_tiles] (fp32).
+    ``dense`` as in internal_tiles."""
     S, D = xh.shape
-    tiles = internal_tiles(g)
+    tiles = internal_tiles(g, dense)
     xq = np.zeros((S, D), dtype=np.float64)
     codes = np.zeros((len(tiles), rf_v2.BLOCK, D), dtype=np.uint8)
     scales = np.zeros(len(tiles), dtype=np.float32)
@@ -133,9 +136,11 @@ def quantize_head(xh: np.ndarray, g: rf_v2.Geometry):
 
 
 def rf_sparse_attention_fp8(q, k, v, layout: str, txt_len: int, latent, sparsity: float,
-                            scale: float | None = None):
+                            scale: float | None = None, latent_k=None):
     """The whole call at fp8 precision (R14, R15): returns (out fp64 in the
-    caller's layout, mask, margin, geometry)."""
+    caller's layout, mask, margin, geometry).  ``latent_k`` as in
+    ``rf_v2.rf_sparse_attention``: k and v are then quantised by the blocks
+    of their own geometry."""
     if not (np.isfinite(sparsity) and 0.0 <= sparsity <= 1.0):
         raise ValueError("sparsity must be finite and in [0, 1]")
     qb, kb, vb = (rf_v2.to_bnsd(np.asarray(a), layout) for a in (q, k, v))
@@ -144,10 +149,14 @@ def rf_sparse_attention_fp8(q, k, v, layout: str, txt_len: int, latent, sparsity
         scale = D ** -0.5
     T, H, W = latent
     g = rf_v2.geometry(S, txt_len, T, H, W)
-    mask, margin = rf_v2.build_mask(qb, kb, g, sparsity)
+    gk = None if latent_k is None else rf_v2.geometry(kb.shape[2], txt_len, *latent_k)
+    gkv = g if gk is None else gk
+    mask, margin = rf_v2.build_mask(qb, kb, g, sparsity, gk)
+    dense = rf_v2.is_dense(g, gk)
     out = np.empty((B, N, S, D), dtype=np.float64)
     for b in range(B):
         for n in range(N):
-            qd, kd, vd = (quantize_head(x[b, n], g)[0] for x in (qb, kb, vb))
-            out[b, n] = rf_v2.attention_rows(qd, kd, vd, g, mask[b, n] if not g.dense else None, scale)
-    return rf_v2.from_bnsd(out, layout), mask, margin, g
+            qd = quantize_head(qb[b, n], g, dense)[0]
+            kd, vd = (quantize_head(x[b, n], gkv, dense)[0] for x in (kb, vb))
+            out[b, n] = rf_v2.attention_rows(qd, kd, vd, g, None if dense else mask[b, n], scale, gk=gk)
+    return rf_v2.from_bnsd(out, layout), mask, margin, (g if gk is None else (g, gk))

@@ -32,6 +32,13 @@ is the same one the CUDA library implements (the two share no code):
      key; every query attends to every prefix key.
   R8 fewer than 32 sparse blocks, or no geometry, means dense attention
      over the whole sequence.
+  R9 a key/value geometry of its own ([SA] ``latent_shape_k``, which
+     defaults to the query's): queries are reordered, pooled and blocked by
+     the query geometry, keys and values by theirs, and both share txt_len.
+     Block scores are nb_q x nb_k; k counts key blocks (R5 over nb_k); the
+     forced columns are the key geometry's first-frame blocks and the dense
+     rows the query geometry's; every query attends to the key prefix.  If
+     either side is dense (R8), the call is dense attention.
 
 Parity status of each function is stated in its docstring; the pins live in
 ``tests/test_oracle_*.py``.
@@ -159,7 +166,7 @@ def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
     return (qbar.astype(np.float64) @ kbar.astype(np.float64).T).astype(np.float32)
 
 
-def topk_mask(scores: np.ndarray, k: int, first_frame: np.ndarray):
+def topk_mask(scores: np.ndarray, k: int, first_frame: np.ndarray, first_frame_cols: np.ndarray | None = None):
     """Kept key blocks per query block, and the gap at the k-th score.
 
     [SA] pipeline: top-k sparse mask generation; [RF] intro: attend to the
@@ -169,41 +176,53 @@ def topk_mask(scores: np.ndarray, k: int, first_frame: np.ndarray):
     keeps all blocks.  ``margin[i]`` = (s_(k) - s_(k+1)) / max(|s_(k)|, 1e-30)
     over the sorted row (inf when k is 0 or nb, or for first-frame rows).
 
+    With a key geometry of its own (R9) the matrix is nb_q x nb_k:
+    ``first_frame`` marks the dense rows, ``first_frame_cols`` (default:
+    the same) the forced columns.
+
     Parity: the selection is pinned against an exhaustive subset search on
     tiny rows, including exact ties.
     """
-    nb = scores.shape[0]
-    mask = np.zeros((nb, nb), dtype=bool)
-    margin = np.full(nb, np.inf, dtype=np.float64)
-    for i in range(nb):
+    nbq, nb = scores.shape
+    ffc = first_frame if first_frame_cols is None else first_frame_cols
+    mask = np.zeros((nbq, nb), dtype=bool)
+    margin = np.full(nbq, np.inf, dtype=np.float64)
+    for i in range(nbq):
         if first_frame[i]:
             mask[i, :] = True
             continue
         row = scores[i]
         order = np.lexsort((np.arange(nb), -row))       # primary: score desc; then index asc
         mask[i, order[:k]] = True
-        mask[i, first_frame] = True
+        mask[i, ffc] = True
         if 0 < k < nb:
             sk, sk1 = float(row[order[k - 1]]), float(row[order[k]])
             margin[i] = (sk - sk1) / max(abs(sk), 1e-30)
     return mask, margin
 
 
-def build_mask(q_bnsd: np.ndarray, k_bnsd: np.ndarray, g: Geometry, sparsity: float):
-    """Block mask for every (b, head): [B, N, nb, nb] bool and margins [B, N, nb]."""
+def is_dense(g: Geometry, gk: Geometry | None = None) -> bool:
+    """R8, R9: dense attention when either side is."""
+    return g.dense or (gk is not None and gk.dense)
+
+
+def build_mask(q_bnsd: np.ndarray, k_bnsd: np.ndarray, g: Geometry, sparsity: float, gk: Geometry | None = None):
+    """Block mask for every (b, head): [B, N, nb_q, nb_k] bool and margins [B, N, nb_q].
+
+    ``gk`` is the key geometry (R9); None means the query's."""
     B, N = q_bnsd.shape[:2]
-    nb = g.nb
-    mask = np.ones((B, N, nb, nb), dtype=bool)
-    margin = np.full((B, N, nb), np.inf)
-    if g.dense:
+    gk = g if gk is None else gk
+    mask = np.ones((B, N, g.nb, gk.nb), dtype=bool)
+    margin = np.full((B, N, g.nb), np.inf)
+    if is_dense(g, gk):
         return mask, margin
-    k = kept_count(nb, sparsity)
+    k = kept_count(gk.nb, sparsity)
     for b in range(B):
         for n in range(N):
             qbar = pool_blocks(q_bnsd[b, n], g.blocks)
-            kbar = pool_blocks(k_bnsd[b, n], g.blocks)
+            kbar = pool_blocks(k_bnsd[b, n], gk.blocks)
             s = block_scores(qbar, kbar)
-            mask[b, n], margin[b, n] = topk_mask(s, k, g.first_frame)
+            mask[b, n], margin[b, n] = topk_mask(s, k, g.first_frame, gk.first_frame)
     return mask, margin
 
 
@@ -211,17 +230,19 @@ def build_mask(q_bnsd: np.ndarray, k_bnsd: np.ndarray, g: Geometry, sparsity: fl
 # Attention over each row's key set
 # ---------------------------------------------------------------------------
 
-def key_set(g: Geometry, mask_bn: np.ndarray, row_block: int | None) -> np.ndarray:
-    """Token indices a query attends to.
+def key_set(g: Geometry, mask_bn: np.ndarray, row_block: int | None, gk: Geometry | None = None) -> np.ndarray:
+    """Token indices (of the key sequence) a query attends to.
 
-    ``row_block`` is the sparse block holding the query, or None for a
-    prefix (dense) query.  R7: prefix queries and first-frame blocks see
-    every key; a sparse query block sees the prefix plus its kept blocks.
+    ``row_block`` is the query geometry's sparse block holding the query, or
+    None for a prefix (dense) query; ``gk`` the key geometry (R9, default
+    the query's).  R7: prefix queries and first-frame blocks see every key;
+    a sparse query block sees the key prefix plus its kept key blocks.
     """
-    if g.dense or row_block is None or g.first_frame[row_block]:
-        return np.arange(g.S)
+    gk = g if gk is None else gk
+    if is_dense(g, gk) or row_block is None or g.first_frame[row_block]:
+        return np.arange(gk.S)
     kept = np.nonzero(mask_bn[row_block])[0]
-    return np.concatenate([g.prefix, g.blocks[kept].ravel()])
+    return np.concatenate([gk.prefix, gk.blocks[kept].ravel()])
 
 
 def _softmax_attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -> np.ndarray:
@@ -232,14 +253,15 @@ def _softmax_attend(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float) -
     return (e @ v) / e.sum(axis=1, keepdims=True)
 
 
-def attention_rows(qh, kh, vh, g: Geometry, mask_bn, scale: float, rows=None, chunk=512):
+def attention_rows(qh, kh, vh, g: Geometry, mask_bn, scale: float, rows=None, chunk=512, gk: Geometry | None = None):
     """rain_fusion_attention for one (b, head): fp64 output rows.
 
     [SA] pipeline: rain_fusion_attention over the masked key set; [SA]
     ``scale`` (default head_dim ** -0.5).  ``qh/kh/vh`` are [S, D] in the
     caller's token order, so the inverse reorder ([SA] pipeline, last step)
     is implicit: row r of the result is token r.  ``rows`` restricts the
-    output to the given token indices (all when None).
+    output to the given token indices (all when None).  ``gk`` is the key
+    geometry (R9; None: the query's); kh and vh then have its length.
 
     Parity: the dense case is pinned against torch's scaled-dot-product
     attention; masked cases against the same routine given an explicit
@@ -253,14 +275,14 @@ def attention_rows(qh, kh, vh, g: Geometry, mask_bn, scale: float, rows=None, ch
 
     # which sparse block (if any) holds each token
     block_of = np.full(S, -1, dtype=np.int64)
-    if not g.dense:
+    if not is_dense(g, gk):
         block_of[g.blocks.ravel()] = np.repeat(np.arange(g.nb), BLOCK)
 
     groups: dict[int, list[int]] = {}
     for pos, r in enumerate(rows):
         groups.setdefault(int(block_of[r]), []).append(pos)
     for blk, positions in groups.items():
-        keys = key_set(g, mask_bn, None if blk < 0 else blk)
+        keys = key_set(g, mask_bn, None if blk < 0 else blk, gk)
         kk, vv = k64[keys], v64[keys]
         positions = np.asarray(positions)
         for c in range(0, len(positions), chunk):
@@ -296,12 +318,14 @@ def from_bnsd(x: np.ndarray, layout: str) -> np.ndarray:
 
 
 def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: float,
-                        scale: float | None = None):
+                        scale: float | None = None, latent_k=None):
     """The whole rf_v2 call ([SA]): returns (out fp64 in the caller's layout, mask, margin, geometry).
 
     ``q, k, v`` are float arrays (bf16 values widened) in BSND or BNSD.
     [SA] ``scale`` defaults to head_dim ** -0.5; [SG] and [RF] bound
-    sparsity to [0, 1].
+    sparsity to [0, 1].  ``latent_k`` ([SA] ``latent_shape_k``, R9) gives k
+    and v a geometry of their own; the returned geometry is then the pair
+    (query, key).
     """
     if not (np.isfinite(sparsity) and 0.0 <= sparsity <= 1.0):
         raise ValueError("sparsity must be finite and in [0, 1]")
@@ -311,10 +335,11 @@ def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: fl
         scale = D ** -0.5
     T, H, W = latent
     g = geometry(S, txt_len, T, H, W)
-    mask, margin = build_mask(qb, kb, g, sparsity)
+    gk = None if latent_k is None else geometry(kb.shape[2], txt_len, *latent_k)
+    mask, margin = build_mask(qb, kb, g, sparsity, gk)
     out = np.empty((B, N, S, D), dtype=np.float64)
     for b in range(B):
         for n in range(N):
-            out[b, n] = attention_rows(qb[b, n], kb[b, n], vb[b, n], g, mask[b, n] if not g.dense else None,
-                                       scale)
-    return from_bnsd(out, layout), mask, margin, g
+            out[b, n] = attention_rows(qb[b, n], kb[b, n], vb[b, n], g, None if is_dense(g, gk) else mask[b, n],
+                                       scale, gk=gk)
+    return from_bnsd(out, layout), mask, margin, (g if gk is None else (g, gk))

@@ -357,3 +357,89 @@ def test_sparsity_range_is_checked():
             oracle.rf_sparse_attention(q, q, q, "BSND", 0, (4, 32, 32), s)
     with pytest.raises(ValueError):
         oracle.to_bnsd(q, "SBND")
+
+
+# ---------------------------------------------------------------- a key geometry of its own (R9)
+
+def test_key_geometry_equal_to_query_changes_nothing():
+    txt, T, H, W, D = 16, 4, 32, 40, 128
+    S = txt + T * H * W
+    q, k, v = _qkv(S, D, 60)
+    a, ma, _, _ = oracle.rf_sparse_attention(q[None, :, None], k[None, :, None], v[None, :, None], "BSND", txt,
+                                             (T, H, W), 0.6)
+    b, mb, _, _ = oracle.rf_sparse_attention(q[None, :, None], k[None, :, None], v[None, :, None], "BSND", txt,
+                                             (T, H, W), 0.6, latent_k=(T, H, W))
+    np.testing.assert_array_equal(ma, mb)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_key_geometry_sparsity_zero_is_rectangular_sdpa():
+    txt, D = 40, 128
+    Sq, Sk = txt + 2 * 32 * 64, txt + 3 * 32 * 48
+    q = _rand((Sq, D), 61)
+    k, v = _rand((Sk, D), 62), _rand((Sk, D), 63)
+    out, mask, _, (gq, gk) = oracle.rf_sparse_attention(q[None, :, None], k[None, :, None], v[None, :, None], "BSND",
+                                                        txt, (2, 32, 64), 0.0, latent_k=(3, 32, 48))
+    assert not gq.dense and not gk.dense and mask.shape == (1, 1, gq.nb, gk.nb) and mask.all()
+    np.testing.assert_allclose(out[0, :, 0], _sdpa(q, k, v, D ** -0.5), rtol=0, atol=1e-10)
+
+
+def test_key_geometry_either_side_dense_is_dense():
+    txt, D = 7, 128
+    Sq, Sk = txt + 3 * 16 * 16, txt + 4 * 32 * 32        # the query side has 6 blocks: dense
+    q = _rand((Sq, D), 64)
+    k, v = _rand((Sk, D), 65), _rand((Sk, D), 66)
+    out, _, _, (gq, gk) = oracle.rf_sparse_attention(q[None, :, None], k[None, :, None], v[None, :, None], "BSND",
+                                                     txt, (3, 16, 16), 0.9, latent_k=(4, 32, 32))
+    assert gq.dense and not gk.dense
+    np.testing.assert_allclose(out[0, :, 0], _sdpa(q, k, v, D ** -0.5), rtol=0, atol=1e-10)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_rectangular_topk_matches_exhaustive_search(seed):
+    rng = np.random.default_rng(100 + seed)
+    nbq, nbk = int(rng.integers(3, 7)), int(rng.integers(5, 10))
+    scores = rng.integers(-3, 4, size=(nbq, nbk)).astype(np.float32)
+    ffq = np.zeros(nbq, bool)
+    ffq[0] = True
+    ffk = np.zeros(nbk, bool)
+    ffk[:2] = True
+    for k in range(0, nbk + 1):
+        mask, _ = oracle.topk_mask(scores, k, ffq, ffk)
+        assert mask.shape == (nbq, nbk) and mask[0].all()
+        for i in range(1, nbq):
+            assert set(np.nonzero(mask[i])[0].tolist()) == _brute_topk(scores[i], k) | {0, 1}
+
+
+def test_key_geometry_one_hot_value_probe():
+    """As the square probe, with query blocks from one grid and key blocks from another."""
+    txt, D = 16, 128
+    lq, lk = (4, 32, 32), (5, 32, 40)
+    Sq, Sk = txt + 4 * 32 * 32, txt + 5 * 32 * 40
+    gq, gk = oracle.geometry(Sq, txt, *lq), oracle.geometry(Sk, txt, *lk)
+    assert gq.nb == 32 and gk.nb == 50 and gq.ff == 8 and gk.ff == 10
+    rng = np.random.default_rng(5)
+    w = rng.permutation(gk.nb).astype(np.float32) / 8.0 + 0.25
+    q = np.zeros((Sq, D), np.float32)
+    k = np.zeros((Sk, D), np.float32)
+    v = np.zeros((Sk, D), np.float32)
+    sign = np.ones(gq.nb, np.float32)
+    sign[1::2] = -1.0
+    for j in range(gk.nb):
+        k[gk.blocks[j], 0] = w[j]
+        v[gk.blocks[j], j] = 1.0
+    for i in range(gq.nb):
+        q[gq.blocks[i], 0] = sign[i]
+    q[gq.prefix, 0] = 1.0
+    v[gk.prefix, 127] = 1.0
+    kk = oracle.kept_count(gk.nb, 0.7)
+    out, mask, _, _ = oracle.rf_sparse_attention(q[None, :, None], k[None, :, None], v[None, :, None], "BSND",
+                                                 txt, lq, 0.7, latent_k=lk)
+    top = set(np.argsort(-w)[:kk].tolist())
+    bottom = set(np.argsort(w)[:kk].tolist())
+    for i in range(gq.nb):
+        expect = set(range(gk.nb)) if i < gq.ff else (top if sign[i] > 0 else bottom) | set(range(gk.ff))
+        row = out[0, gq.blocks[i][3], 0]
+        assert set(np.nonzero(row[:gk.nb] > 0)[0].tolist()) == expect, i
+        assert row[127] > 0
+        assert set(np.nonzero(mask[0, 0, i])[0].tolist()) == expect
