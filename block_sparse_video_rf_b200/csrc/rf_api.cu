@@ -170,16 +170,61 @@ rf_status_t rf_plan(int S, int txt_len, int T, int H, int W, int block_size, flo
   return ok();
 }
 
+}  // extern "C"
+
+namespace {
+
+// The dense form of a plan: the whole sequence is the prefix, in its own order.
+void densify(rf_plan_t* p) {
+  p->dense = 1;
+  p->P = p->S;
+  p->nb = p->ff = p->k = 0;
+  p->n_promoted = p->n_tail = 0;
+  p->P_pad = (p->P + RF_BLOCK - 1) / RF_BLOCK * RF_BLOCK;
+  p->S_int = p->P_pad;
+  p->n_tiles = p->S_int / RF_BLOCK;
+  p->mask_words = 0;
+}
+
+// Plans of the query geometry and of the key/value geometry (S_kv <= 0: the
+// query's).  Both share txt_len; if either is dense the call is (both plans
+// dense).
+rf_status_t make_plans(int S, int txt_len, int T, int H, int W, int S_kv, int kv_t, int kv_h, int kv_w, int block_size,
+                       float sparsity, rf_plan_t* g, rf_plan_t* gk) {
+  rf_status_t st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, g);
+  if (st != RF_OK) return st;
+  if (S_kv <= 0) {
+    *gk = *g;
+    return RF_OK;
+  }
+  if ((st = rf_plan(S_kv, txt_len, kv_t, kv_h, kv_w, block_size, sparsity, gk)) != RF_OK) return st;
+  if (g->dense || gk->dense) {
+    densify(g);
+    densify(gk);
+  }
+  return RF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rf_status_t rf_plan_kv(int S, int txt_len, int T, int H, int W, int S_kv, int kv_t, int kv_h, int kv_w, int block_size,
+                       float sparsity, rf_plan_t* plan, rf_plan_t* plan_kv) {
+  if (!plan || !plan_kv) return fail(RF_ERR_ARG, "plan pointer is NULL");
+  rf_status_t st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, plan, plan_kv);
+  return st == RF_OK ? ok() : st;
+}
+
 rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D, const rf_plan_t* g,
-                                   rf_ws_layout_t* lay) {
+                                   const rf_plan_t* gk, rf_ws_layout_t* lay) {
   if (!g || !lay) return fail(RF_ERR_ARG, "NULL plan or layout");
+  if (!gk) gk = g;
   if (precision != RF_PREC_NATIVE && precision != RF_PREC_FP8) return fail(RF_ERR_ARG, "unknown precision %d", (int)precision);
   if (B <= 0 || N <= 0) return fail(RF_ERR_ARG, "B and N must be positive");
   if (D != RF_HEAD_DIM) return fail(RF_ERR_UNSUPPORTED, "head dim must be 128 (got %d)", D);
   const size_t heads = (size_t)B * N;
-  const size_t tensor = heads * g->S_int * RF_HEAD_DIM * 2;
-  const size_t pooled = heads * g->nb * RF_HEAD_DIM * 4;
-  const size_t rows = heads * g->nb;
+  const size_t rows_q = heads * g->S_int, rows_k = heads * gk->S_int;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at_off = off;
@@ -187,21 +232,22 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
     return at_off;
   };
   rf_ws_layout_t L{};
-  L.q_int = take(tensor);
-  L.k_int = take(tensor);
-  L.v_int = take(tensor);
-  L.pooled_q = take(pooled);
-  L.pooled_k = take(pooled);
-  L.mask = take(rows * g->mask_words * 4);
-  L.kept = take(rows * 4);
-  L.margin = take(rows * 4);
+  // the work counter and the status word first: their places depend on nothing
   L.counter = take(4);
   L.status = take(4);
+  L.q_int = take(rows_q * RF_HEAD_DIM * 2);
+  L.k_int = take(rows_k * RF_HEAD_DIM * 2);
+  L.v_int = take(rows_k * RF_HEAD_DIM * 2);
+  L.pooled_q = take(heads * g->nb * RF_HEAD_DIM * 4);
+  L.pooled_k = take(heads * gk->nb * RF_HEAD_DIM * 4);
+  L.mask = take(heads * g->nb * gk->mask_words * 4);
+  L.kept = take(heads * g->nb * 4);
+  L.margin = take(heads * g->nb * 4);
   const bool fp8 = precision == RF_PREC_FP8;
-  L.q8 = take(fp8 ? tensor / 2 : 0);
-  L.k8 = take(fp8 ? tensor / 2 : 0);
-  L.v8 = take(fp8 ? tensor / 2 : 0);
-  L.scales = take(fp8 ? 3 * heads * g->n_tiles * 4 : 0);
+  L.q8 = take(fp8 ? rows_q * RF_HEAD_DIM : 0);
+  L.k8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
+  L.v8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
+  L.scales = take(fp8 ? heads * (g->n_tiles + 2 * (size_t)gk->n_tiles) * 4 : 0);
   L.vmax = take(fp8 ? heads * 4 : 0);
   L.total = off;
   *lay = L;
@@ -209,44 +255,47 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
 }
 
 rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* g, rf_ws_layout_t* lay) {
-  return rf_workspace_layout_ex(RF_PREC_NATIVE, B, N, D, g, lay);
+  return rf_workspace_layout_ex(RF_PREC_NATIVE, B, N, D, g, nullptr, lay);
 }
 
-size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int T, int H, int W) {
-  rf_plan_t g;
+size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int T, int H, int W,
+                            int S_kv, int kv_t, int kv_h, int kv_w) {
+  rf_plan_t g, gk;
   rf_ws_layout_t L;
-  if (rf_plan(S, txt_len, T, H, W, RF_BLOCK, 0.f, &g) != RF_OK) return 0;
-  if (rf_workspace_layout_ex(precision, B, N, D, &g, &L) != RF_OK) return 0;
+  if (make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, RF_BLOCK, 0.f, &g, &gk) != RF_OK) return 0;
+  if (rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L) != RF_OK) return 0;
   return L.total;
 }
 
 size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int T, int H, int W) {
-  return rf_workspace_size_ex(RF_PREC_NATIVE, B, S, N, D, txt_len, T, H, W);
+  return rf_workspace_size_ex(RF_PREC_NATIVE, B, S, N, D, txt_len, T, H, W, 0, 0, 0, 0);
 }
 
 rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype, rf_precision_t precision,
-                          rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W,
-                          int block_size, float sparsity, void* ws, size_t ws_bytes, void* stream) {
+                          rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W, int S_kv,
+                          int kv_t, int kv_h, int kv_w, int block_size, float sparsity, void* ws, size_t ws_bytes,
+                          void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!q || !k || !v) return fail(RF_ERR_ARG, "q, k and v must be device pointers");
-  rf_plan_t g;
-  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_plan_t g, gk;
+  if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
+    return st;
   rf_ws_layout_t L;
-  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L)) != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e = rf::launch_permute_pool(q, k, v, dtype, layout, B, S, N, g, at<void>(ws, L.q_int),
+  cudaError_t e = rf::launch_permute_pool(q, k, v, dtype, layout, B, S, gk.S, N, g, gk, at<void>(ws, L.q_int),
                                           at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
                                           at<float>(ws, L.pooled_k), s);
   if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
-  e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, at<uint32_t>(ws, L.mask),
+  e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, gk, at<uint32_t>(ws, L.mask),
                       at<int>(ws, L.kept), at<float>(ws, L.margin), s);
   if (e != cudaSuccess) return cuda_fail(e, "mask launch");
   if (precision == RF_PREC_FP8) {
     e = rf::launch_quantize_fp8(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int), dtype, B * N, g,
-                                at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
+                                gk, at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
                                 at<float>(ws, L.scales), at<float>(ws, L.vmax), s);
     if (e != cudaSuccess) return cuda_fail(e, "fp8 quantisation launch");
   }
@@ -256,21 +305,22 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
 rf_status_t rf_prepare(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N, int D,
                        int txt_len, int T, int H, int W, int block_size, float sparsity, void* ws, size_t ws_bytes,
                        void* stream) {
-  return rf_prepare_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity,
-                       ws, ws_bytes, stream);
+  return rf_prepare_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, 0, 0, 0, 0, block_size,
+                       sparsity, ws, ws_bytes, stream);
 }
 
 rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
-                         int txt_len, int T, int H, int W, int block_size, float sparsity, float scale, void* out,
-                         void* ws, size_t ws_bytes, void* stream) {
+                         int txt_len, int T, int H, int W, int S_kv, int kv_t, int kv_h, int kv_w, int block_size,
+                         float sparsity, float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!out) return fail(RF_ERR_ARG, "out must be a device pointer");
-  rf_plan_t g;
-  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  rf_plan_t g, gk;
+  if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
+    return st;
   rf_ws_layout_t L;
-  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
+  if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L)) != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), s);
@@ -278,11 +328,11 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
   if (precision == RF_PREC_FP8)
     e = rf::launch_attention_fp8(at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
                                  at<float>(ws, L.scales), at<float>(ws, L.vmax), at<uint32_t>(ws, L.mask), dtype,
-                                 layout, B, S, N, g, resolve_scale(scale, D), out, at<int>(ws, L.counter),
+                                 layout, B, S, N, g, gk, resolve_scale(scale, D), out, at<int>(ws, L.counter),
                                  at<int>(ws, L.status), debug_settings(), s);
   else
     e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
-                             at<uint32_t>(ws, L.mask), dtype, layout, B, S, N, g, resolve_scale(scale, D), out,
+                             at<uint32_t>(ws, L.mask), dtype, layout, B, S, N, g, gk, resolve_scale(scale, D), out,
                              at<int>(ws, L.counter), at<int>(ws, L.status), debug_settings(), s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
@@ -291,47 +341,49 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
 rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H, int W,
                       int block_size, float sparsity, float scale, void* out, void* ws, size_t ws_bytes,
                       void* stream) {
-  return rf_attend_ex(RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out,
-                      ws, ws_bytes, stream);
+  return rf_attend_ex(RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, 0, 0, 0, 0, block_size, sparsity,
+                      scale, out, ws, ws_bytes, stream);
 }
 
 rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype,
                                    rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
-                                   int txt_len, int T, int H, int W, int block_size, float sparsity, float scale,
-                                   void* out, void* ws, size_t ws_bytes, void* stream) {
+                                   int txt_len, int T, int H, int W, int S_kv, int kv_t, int kv_h, int kv_w,
+                                   int block_size, float sparsity, float scale, void* out, void* ws, size_t ws_bytes,
+                                   void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!q || !k || !v || !out) return fail(RF_ERR_ARG, "q, k, v and out must be device pointers");
   if (out == q || out == k || out == v) return fail(RF_ERR_ARG, "out must not alias q, k or v");
   if (!ws) {
-    rf_plan_t g;
-    if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+    rf_plan_t g, gk;
+    if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
+      return st;
     rf_ws_layout_t L;
-    if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &L)) != RF_OK) return st;
+    if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L)) != RF_OK) return st;
     if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
     ws_bytes = L.total;
   }
-  st = rf_prepare_ex(q, k, v, dtype, precision, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, ws,
-                     ws_bytes, stream);
+  st = rf_prepare_ex(q, k, v, dtype, precision, layout, B, S, N, D, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w,
+                     block_size, sparsity, ws, ws_bytes, stream);
   if (st != RF_OK) return st;
-  return rf_attend_ex(dtype, precision, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity, scale, out, ws,
-                      ws_bytes, stream);
+  return rf_attend_ex(dtype, precision, layout, B, S, N, D, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size,
+                      sparsity, scale, out, ws, ws_bytes, stream);
 }
 
 rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
                                    int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
                                    float scale, void* out, void* ws, size_t ws_bytes, void* stream) {
   if (!ws) return fail(RF_ERR_WORKSPACE, "workspace is NULL");
-  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size,
-                                sparsity, scale, out, ws, ws_bytes, stream);
+  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, 0, 0, 0, 0,
+                                block_size, sparsity, scale, out, ws, ws_bytes, stream);
 }
 
 rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
                                 int D, int txt_len, int T, int H, int W, int block_size, float sparsity, float scale,
                                 void* out, void* stream) {
-  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, block_size,
-                                sparsity, scale, out, nullptr, 0, stream);
+  return rf_sparse_attention_ex(q, k, v, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, 0, 0, 0, 0,
+                                block_size, sparsity, scale, out, nullptr, 0, stream);
 }
 
 rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len, int T, int H,
@@ -384,9 +436,11 @@ rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const
                            void* stream) {
   if (!status) return fail(RF_ERR_ARG, "status pointer is NULL");
   rf_ws_layout_t L;
-  rf_status_t st = rf_workspace_layout(B, N, D, g, &L);
-  if (st != RF_OK) return st;
-  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  rf_status_t st = rf_workspace_layout(B, N, D, g, &L);   // validates the arguments; the status word's place
+  if (st != RF_OK) return st;                             // does not depend on them
+  if (!ws) return fail(RF_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return fail(RF_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < L.status + sizeof(int)) return fail(RF_ERR_WORKSPACE, "workspace too small for its status word");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int h = 0;
   cudaError_t e = cudaMemcpyAsync(&h, at<int>(ws, L.status), sizeof(int), cudaMemcpyDeviceToHost, s);

@@ -8,8 +8,10 @@
 // key blocks.
 //
 // Work unit: one 128-row query tile of one (b, head).  Its KV list is every
-// prefix tile, then either every sparse block (dense tile) or the blocks set
-// in its mask row, in ascending order.  Persistent CTAs (one per SM) take
+// key prefix tile, then either every key block (dense tile) or the blocks
+// set in its mask row, in ascending order.  Keys and values may have a
+// geometry of their own (lite_boost.ops.sparse_attention, latent_shape_k):
+// query tiles follow the query plan, KV tiles the key plan.  Persistent CTAs (one per SM) take
 // units from a global counter in (head, tile) order, dense tiles of a head
 // first, so the heads in flight keep their K/V in L2.
 //
@@ -135,14 +137,16 @@ struct Smem {
 };
 
 struct AttnParams {
-  rf_plan_t g;
-  int B, S, N, layout;
+  rf_plan_t g;       // query geometry (units, dense rows, the output's token order)
+  rf_plan_t gk;      // key/value geometry (KV lists; the same as g unless k and v have their own)
+  int B, S, N, layout;   // S: query sequence length (the output's)
   int total_items;
-  int n_ptiles;      // prefix tiles (P_pad / 128)
-  int p_rem;         // valid rows of the last prefix tile when it is partial, else 0
+  int n_ptiles;      // query prefix tiles (g.P_pad / 128)
+  int n_ptiles_k;    // key prefix tiles (gk.P_pad / 128)
+  int p_rem_k;       // valid rows of the last key prefix tile when it is partial, else 0
   float scale_log2;
-  const uint32_t* mask;
-  const float* scales;   // fp8: [3, B*N, n_tiles] block scales of q, k, v
+  const uint32_t* mask;  // [B*N, g.nb, gk.mask_words]
+  const float* scales;   // fp8: q [B*N, g.n_tiles], then k and v [B*N, gk.n_tiles] block scales
   const float* vmax;     // fp8: [B*N] largest V block scale of each head
   int* counter;
   int* status;
@@ -193,9 +197,9 @@ struct KvIter {
   uint32_t bits;
   __device__ void init(int base_, const AttnParams& p, const uint32_t* mrow_) {
     base = base_;
-    n_ptiles = p.n_ptiles;
-    nb = p.g.nb;
-    words = p.g.mask_words;
+    n_ptiles = p.n_ptiles_k;
+    nb = p.gk.nb;
+    words = p.gk.mask_words;
     mrow = mrow_;
     t = 0;
     wd = 0;
@@ -240,7 +244,7 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
   uint32_t c = 0, nk = 0, nv = 0;   // units, K tiles and V tiles issued
-  const int S_int = p.g.S_int;
+  const int S_int_k = p.gk.S_int;
   const int BN = p.B * p.N;
   bool ok = true;
   while (ok) {
@@ -256,28 +260,28 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
       itm.bn = w / p.g.n_tiles;
       itm.qt = w - itm.bn * p.g.n_tiles;
       if (is_dense_tile(p, itm.qt)) {
-        itm.ntiles = p.g.n_tiles;
+        itm.ntiles = p.gk.n_tiles;
       } else {
-        mrow = p.mask + ((size_t)itm.bn * p.g.nb + (itm.qt - p.n_ptiles)) * p.g.mask_words;
+        mrow = p.mask + ((size_t)itm.bn * p.g.nb + (itm.qt - p.n_ptiles)) * p.gk.mask_words;
         int cnt = 0;
-        for (int wd = 0; wd < p.g.mask_words; ++wd) cnt += __popc(mrow[wd]);
-        itm.ntiles = p.n_ptiles + cnt;
+        for (int wd = 0; wd < p.gk.mask_words; ++wd) cnt += __popc(mrow[wd]);
+        itm.ntiles = p.n_ptiles_k + cnt;
       }
     }
     sl.items[it] = itm;
     mbar_arrive(&sl.item_full[it]);
     if (itm.bn < 0) break;
 
-    const int base = itm.bn * S_int;
-    const float* sc_k = C::kFp8 ? p.scales + ((size_t)BN + itm.bn) * p.g.n_tiles : nullptr;
-    const float* sc_v = C::kFp8 ? p.scales + ((size_t)2 * BN + itm.bn) * p.g.n_tiles : nullptr;
+    const int base = itm.bn * S_int_k;   // the unit's KV rows
+    const float* sc_k = C::kFp8 ? p.scales + (size_t)BN * p.g.n_tiles + (size_t)itm.bn * p.gk.n_tiles : nullptr;
+    const float* sc_v = C::kFp8 ? sc_k + (size_t)BN * p.gk.n_tiles : nullptr;
     if (c >= 1 && !wait1(sm, p, &sl.q_empty, ph(c - 1))) {
       ok = false;
       break;
     }
     if (!(p.skip_first_q && c == 0)) {
       if (C::kFp8) sl.q_scale = p.scales[(size_t)itm.bn * p.g.n_tiles + itm.qt];
-      load_tile<C>(sl.q, tq, &sl.q_full, base + itm.qt * RF_BLOCK, pol_q);
+      load_tile<C>(sl.q, tq, &sl.q_full, itm.bn * p.g.S_int + itm.qt * RF_BLOCK, pol_q);
     }
     ++c;
     KvIter kit;
@@ -587,7 +591,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
       if (ok) ok = waitw(sm, p, &sl.s_full, ph(t));
       if (ok) {
         tc_fence_after();
-        const int p_valid = (p.p_rem != 0 && j == p.n_ptiles - 1) ? p.p_rem : RF_BLOCK;
+        const int p_valid = (p.p_rem_k != 0 && j == p.n_ptiles_k - 1) ? p.p_rem_k : RF_BLOCK;
         if (C::kFp8) {
           const TileScale f = sl.ts[t & 1];
           softmax_tile<C>(tS, tO, j == 0, p_valid, f.c, f.lr, f.ir, m_use, l);
@@ -742,17 +746,19 @@ bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, CUtensorMa
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-AttnParams make_params(const uint32_t* mask, int layout, int B, int S, int N, const rf_plan_t& g, float scale,
-                       void* out, int* counter, int* status, const AttnDebug& dbg) {
+AttnParams make_params(const uint32_t* mask, int layout, int B, int S, int N, const rf_plan_t& g,
+                       const rf_plan_t& gk, float scale, void* out, int* counter, int* status, const AttnDebug& dbg) {
   AttnParams p;
   p.g = g;
+  p.gk = gk;
   p.B = B;
   p.S = S;
   p.N = N;
   p.layout = layout;
   p.total_items = B * N * g.n_tiles;
   p.n_ptiles = g.P_pad / RF_BLOCK;
-  p.p_rem = g.P % RF_BLOCK;
+  p.n_ptiles_k = gk.P_pad / RF_BLOCK;
+  p.p_rem_k = gk.P % RF_BLOCK;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.mask = mask;
   p.scales = nullptr;
@@ -786,31 +792,32 @@ cudaError_t launch_cfg(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 }  // namespace
 
 cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
-                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
-                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream) {
-  const uint64_t rows = (uint64_t)B * N * g.S_int;
+                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, const rf_plan_t& gk,
+                             float scale, void* out, int* counter, int* status, const AttnDebug& dbg,
+                             cudaStream_t stream) {
+  const uint64_t rows_q = (uint64_t)B * N * g.S_int, rows_k = (uint64_t)B * N * gk.S_int;
   const bool f16 = dtype == RF_F16;
   const CUtensorMapDataType type = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, q_int, rows, type, 2) || !make_tile_map(&tk, k_int, rows, type, 2) ||
-      !make_tile_map(&tv, v_int, rows, type, 2))
+  if (!make_tile_map(&tq, q_int, rows_q, type, 2) || !make_tile_map(&tk, k_int, rows_k, type, 2) ||
+      !make_tile_map(&tv, v_int, rows_k, type, 2))
     return cudaErrorInvalidValue;
-  const AttnParams p = make_params(mask, layout, B, S, N, g, scale, out, counter, status, dbg);
+  const AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, dbg);
   return f16 ? launch_cfg<Cfg<true, false>>(tq, tk, tv, p, stream)
              : launch_cfg<Cfg<false, false>>(tq, tk, tv, p, stream);
 }
 
 cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
                                  const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
-                                 const rf_plan_t& g, float scale, void* out, int* counter, int* status,
-                                 const AttnDebug& dbg, cudaStream_t stream) {
-  const uint64_t rows = (uint64_t)B * N * g.S_int;
+                                 const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out, int* counter,
+                                 int* status, const AttnDebug& dbg, cudaStream_t stream) {
+  const uint64_t rows_q = (uint64_t)B * N * g.S_int, rows_k = (uint64_t)B * N * gk.S_int;
   CUtensorMap tq, tk, tv;
-  if (!make_tile_map(&tq, q8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
-      !make_tile_map(&tk, k8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
-      !make_tile_map(&tv, v8, rows, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
+  if (!make_tile_map(&tq, q8, rows_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tk, k8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tv, v8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
     return cudaErrorInvalidValue;
-  AttnParams p = make_params(mask, layout, B, S, N, g, scale, out, counter, status, dbg);
+  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, dbg);
   p.scales = scales;
   p.vmax = vmax;
   return dtype == RF_F16 ? launch_cfg<Cfg<true, true>>(tq, tk, tv, p, stream)

@@ -8,21 +8,23 @@
 
 namespace rf {
 
-// K1: token reorder into [B, N, S_int, 128] 16-bit rows for q, k, v (pad
-// rows zeroed), with the fp32 block means of q and k for the sparse blocks;
-// dtype (rf_dtype_t) says how the pooling reads the values.
+// K1: token reorder into [B, N, S_int, 128] 16-bit rows for q (query plan g,
+// S rows) and k, v (key plan gk, Sk rows; pad rows zeroed), with the fp32
+// block means of q and k for the sparse blocks; dtype (rf_dtype_t) says how
+// the pooling reads the values.
 cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int dtype, int layout, int B, int S,
-                                int N, const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
-                                float* pooled_k, cudaStream_t stream);
+                                int Sk, int N, const rf_plan_t& g, const rf_plan_t& gk, void* q_int, void* k_int,
+                                void* v_int, float* pooled_q, float* pooled_k, cudaStream_t stream);
 
 // K4: inverse reorder of an internal-order tensor into the caller's layout.
 cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N, const rf_plan_t& g, void* out,
                              cudaStream_t stream);
 
-// K2: block scores + top-k + forced first-frame blocks -> bit mask rows,
-// kept counts and k-th-score margins.
-cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g, uint32_t* mask,
-                        int* kept, float* margin, cudaStream_t stream);
+// K2: block scores (g.nb query blocks x gk.nb key blocks) + top-k (gk.k) +
+// forced first-frame blocks (key columns gk.ff, query rows g.ff) -> bit mask
+// rows, kept counts and k-th-score margins.
+cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g,
+                        const rf_plan_t& gk, uint32_t* mask, int* kept, float* margin, cudaStream_t stream);
 
 // Test controls of the attention kernel's bounded waits (see rf_debug_set_wait).
 struct AttnDebug {
@@ -34,21 +36,23 @@ struct AttnDebug {
 // straight to the caller's layout (inverse reorder fused in the epilogue).
 // Operands and output in dtype (rf_dtype_t).
 cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
-                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, float scale, void* out,
-                             int* counter, int* status, const AttnDebug& dbg, cudaStream_t stream);
+                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, const rf_plan_t& gk,
+                             float scale, void* out, int* counter, int* status, const AttnDebug& dbg,
+                             cudaStream_t stream);
 
-// fp8 quantisation of the reordered q, k, v (RF_PREC_FP8): per (tensor, head,
-// 128-row block) scale = amax / 448 and e4m3 codes; V's blocks stored
-// transposed; vmax[bn] = the largest V block scale of head bn.
+// fp8 quantisation of the reordered q (plan g), k and v (plan gk)
+// (RF_PREC_FP8): per (tensor, head, 128-row block) scale = amax / 448 and
+// e4m3 codes; V's blocks stored transposed; scales = q [BN, g.n_tiles], k and
+// v [BN, gk.n_tiles]; vmax[bn] = the largest V block scale of head bn.
 cudaError_t launch_quantize_fp8(const void* q_int, const void* k_int, const void* v_int, int dtype, int BN,
-                                const rf_plan_t& g, uint8_t* q8, uint8_t* k8, uint8_t* v8, float* scales,
-                                float* vmax, cudaStream_t stream);
+                                const rf_plan_t& g, const rf_plan_t& gk, uint8_t* q8, uint8_t* k8, uint8_t* v8,
+                                float* scales, float* vmax, cudaStream_t stream);
 
 // K3 on the e4m3 tensors of launch_quantize_fp8; output in dtype.
 cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
                                  const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
-                                 const rf_plan_t& g, float scale, void* out, int* counter, int* status,
-                                 const AttnDebug& dbg, cudaStream_t stream);
+                                 const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out, int* counter,
+                                 int* status, const AttnDebug& dbg, cudaStream_t stream);
 
 // Block mask with the pooled means in the library's static scratch array
 // (no device allocation); see rf_block_mask_noalloc.

@@ -7,7 +7,8 @@
 // pipeline: block pooling -> top-k sparse mask generation.
 //
 // Per (b, head): s_ij = qbar_i . kbar_j in fp32 (sequential FMA over the 128
-// channels).  Row i keeps the k largest scores, equal scores going to the
+// channels), i over the query geometry's blocks, j over the key geometry's
+// (the same unless k and v have their own, lite_boost latent_shape_k).  Row i keeps the k largest scores, equal scores going to the
 // lower block index, plus the first-frame blocks; first-frame rows keep
 // everything.  The k-th score is found by a 32-step MSB-first search over
 // order-preserving integer keys, one warp per row.
@@ -130,11 +131,14 @@ __device__ __forceinline__ void select_row(const uint32_t* __restrict__ keys_s, 
   }
 }
 
+// nbq query blocks (the first ffq of them dense rows) against nb key blocks
+// (the first ff of them forced columns); k kept per row.
 template <int QC, int PL>
 __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const float* __restrict__ pooled_q,
-                                                           const float* __restrict__ pooled_k, int nb, int ff, int k,
-                                                           int words, uint32_t* __restrict__ mask,
-                                                           int* __restrict__ kept, float* __restrict__ margin) {
+                                                           const float* __restrict__ pooled_k, int nbq, int ffq,
+                                                           int nb, int ff, int k, int words,
+                                                           uint32_t* __restrict__ mask, int* __restrict__ kept,
+                                                           float* __restrict__ margin) {
   extern __shared__ __align__(16) float smem[];
   float* qs = smem;                        // [QC][kPad]
   float* ks = qs + QC * kPad;              // [64][kPad]
@@ -144,12 +148,12 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const float* __restr
   const int i0 = blockIdx.x * QC;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   constexpr int RPW = QC / 8;               // query rows per warp
-  const float* pq = pooled_q + (size_t)bn * nb * RF_HEAD_DIM;
+  const float* pq = pooled_q + (size_t)bn * nbq * RF_HEAD_DIM;
   const float* pk = pooled_k + (size_t)bn * nb * RF_HEAD_DIM;
 
   for (int idx = tid; idx < QC * 32; idx += kMaskThreads) {
     const int r = idx >> 5, d4 = idx & 31;
-    const float4 v = (i0 + r < nb) ? __ldg(reinterpret_cast<const float4*>(pq + (size_t)(i0 + r) * RF_HEAD_DIM) + d4)
+    const float4 v = (i0 + r < nbq) ? __ldg(reinterpret_cast<const float4*>(pq + (size_t)(i0 + r) * RF_HEAD_DIM) + d4)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     *reinterpret_cast<float4*>(qs + r * kPad + 4 * d4) = v;
   }
@@ -195,9 +199,9 @@ __global__ void __launch_bounds__(kMaskThreads) mask_kernel(const float* __restr
   for (int rr = 0; rr < RPW; ++rr) {
     const int lr = warp * RPW + rr;
     const int i = i0 + lr;
-    if (i >= nb) break;
-    select_row<PL>(sc + lr * row_stride, nb, ff, k, words, i < ff, mask + ((size_t)bn * nb + i) * words,
-                   kept + (size_t)bn * nb + i, margin + (size_t)bn * nb + i);
+    if (i >= nbq) break;
+    select_row<PL>(sc + lr * row_stride, nb, ff, k, words, i < ffq, mask + ((size_t)bn * nbq + i) * words,
+                   kept + (size_t)bn * nbq + i, margin + (size_t)bn * nbq + i);
   }
 }
 
@@ -207,35 +211,37 @@ size_t mask_smem_bytes(int words) {
 }
 
 template <int QC, int PL>
-cudaError_t launch_mask_qc_pl(const float* pq, const float* pk, int BN, int nb, int ff, int k, int words,
+cudaError_t launch_mask_qc_pl(const float* pq, const float* pk, int BN, const rf_plan_t& g, const rf_plan_t& gk,
                               uint32_t* mask, int* kept, float* margin, cudaStream_t stream) {
-  const size_t smem = mask_smem_bytes<QC>(words);
+  const size_t smem = mask_smem_bytes<QC>(gk.mask_words);
   cudaError_t e = cudaFuncSetAttribute(mask_kernel<QC, PL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((nb + QC - 1) / QC, BN);
-  mask_kernel<QC, PL><<<grid, kMaskThreads, smem, stream>>>(pq, pk, nb, ff, k, words, mask, kept, margin);
+  dim3 grid((g.nb + QC - 1) / QC, BN);
+  mask_kernel<QC, PL><<<grid, kMaskThreads, smem, stream>>>(pq, pk, g.nb, g.ff, gk.nb, gk.ff, gk.k, gk.mask_words,
+                                                            mask, kept, margin);
   return cudaGetLastError();
 }
 
 template <int QC>
-cudaError_t launch_mask_qc(const float* pq, const float* pk, int BN, int nb, int ff, int k, int words, uint32_t* mask,
-                           int* kept, float* margin, cudaStream_t stream) {
-  if (words <= 16) return launch_mask_qc_pl<QC, 16>(pq, pk, BN, nb, ff, k, words, mask, kept, margin, stream);
-  if (words <= 32) return launch_mask_qc_pl<QC, 32>(pq, pk, BN, nb, ff, k, words, mask, kept, margin, stream);
-  return launch_mask_qc_pl<QC, 128>(pq, pk, BN, nb, ff, k, words, mask, kept, margin, stream);
+cudaError_t launch_mask_qc(const float* pq, const float* pk, int BN, const rf_plan_t& g, const rf_plan_t& gk,
+                           uint32_t* mask, int* kept, float* margin, cudaStream_t stream) {
+  const int words = gk.mask_words;
+  if (words <= 16) return launch_mask_qc_pl<QC, 16>(pq, pk, BN, g, gk, mask, kept, margin, stream);
+  if (words <= 32) return launch_mask_qc_pl<QC, 32>(pq, pk, BN, g, gk, mask, kept, margin, stream);
+  return launch_mask_qc_pl<QC, 128>(pq, pk, BN, g, gk, mask, kept, margin, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g, uint32_t* mask,
-                        int* kept, float* margin, cudaStream_t stream) {
-  if (g.nb == 0) return cudaSuccess;
+cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, const rf_plan_t& g,
+                        const rf_plan_t& gk, uint32_t* mask, int* kept, float* margin, cudaStream_t stream) {
+  if (g.nb == 0 || gk.nb == 0) return cudaSuccess;
   const size_t limit = 200 * 1024;
-  if (mask_smem_bytes<32>(g.mask_words) <= limit)
-    return launch_mask_qc<32>(pooled_q, pooled_k, BN, g.nb, g.ff, g.k, g.mask_words, mask, kept, margin, stream);
-  if (mask_smem_bytes<16>(g.mask_words) <= limit)
-    return launch_mask_qc<16>(pooled_q, pooled_k, BN, g.nb, g.ff, g.k, g.mask_words, mask, kept, margin, stream);
-  return launch_mask_qc<8>(pooled_q, pooled_k, BN, g.nb, g.ff, g.k, g.mask_words, mask, kept, margin, stream);
+  if (mask_smem_bytes<32>(gk.mask_words) <= limit)
+    return launch_mask_qc<32>(pooled_q, pooled_k, BN, g, gk, mask, kept, margin, stream);
+  if (mask_smem_bytes<16>(gk.mask_words) <= limit)
+    return launch_mask_qc<16>(pooled_q, pooled_k, BN, g, gk, mask, kept, margin, stream);
+  return launch_mask_qc<8>(pooled_q, pooled_k, BN, g, gk, mask, kept, margin, stream);
 }
 
 }  // namespace rf

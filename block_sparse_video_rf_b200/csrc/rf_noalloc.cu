@@ -112,7 +112,7 @@ cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int dtype, i
                                       N, g, pooled_q, pooled_k);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_mask(pooled_q, pooled_k, B * N, g, mask, kept, margin, stream);
+  return launch_mask(pooled_q, pooled_k, B * N, g, g, mask, kept, margin, stream);
 }
 
 }  // namespace rf

@@ -7,6 +7,8 @@
 // into 8x8 tiles and promotes the non-aligned rest ("Geometry handling").
 #include <cuda_runtime.h>
 
+#include <cstring>
+
 #include "rf_dtype.h"
 #include "rf_geometry.h"
 #include "rf_kernels.h"
@@ -19,16 +21,23 @@ constexpr int kPermThreads = 256;   // 16 rows x 16 chunks of 16 bytes per pass
 constexpr int kRowsPerPass = kPermThreads / 16;
 constexpr int kPasses = RF_BLOCK / kRowsPerPass;
 
-// One CTA = one 128-row internal tile of one (b, head), for q, k and v.
-// Sparse tiles also write the fp32 block means of q and k.  The column sums
-// run in a fixed order (per thread over its 8 rows, then over the 16 row
-// groups), so results are deterministic.  Rows are 16-bit values (bf16, or
-// fp16 when kF16) copied bit for bit; only the pooling reads them as numbers.
+// Up to three tensors of one geometry (plan g, S rows in the caller's layout).
+struct PermArgs {
+  const uint16_t* src[3];
+  uint16_t* dst[3];
+  float* pooled[2];   // block means of tensors 0 and 1 (nullptr: not pooled)
+  int count;          // tensors in use
+};
+
+// One CTA = one 128-row internal tile of one (b, head), for each tensor.
+// Sparse tiles also write the fp32 block means of the pooled tensors.  The
+// column sums run in a fixed order (per thread over its 8 rows, then over the
+// 16 row groups), so results are deterministic.  Rows are 16-bit values
+// (bf16, or fp16 when kF16) copied bit for bit; only the pooling reads them as
+// numbers.
 template <bool kF16>
-__global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
-    const uint16_t* __restrict__ q, const uint16_t* __restrict__ k, const uint16_t* __restrict__ v, int layout, int B,
-    int S, int N, rf_plan_t g, uint16_t* __restrict__ q_int, uint16_t* __restrict__ k_int, uint16_t* __restrict__ v_int,
-    float* __restrict__ pooled_q, float* __restrict__ pooled_k) {
+__global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(PermArgs a, int layout, int B, int S, int N,
+                                                                    rf_plan_t g) {
   __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
   const int tile = blockIdx.x;
   const int bn = blockIdx.y;
@@ -46,21 +55,21 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
   }
   const int64_t dst_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM + chunk * 8;
 
-  const uint16_t* srcs[3] = {q, k, v};
-  uint16_t* dsts[3] = {q_int, k_int, v_int};
 #pragma unroll
   for (int t = 0; t < 3; ++t) {
+    if (t >= a.count) break;
+    const uint16_t* src = a.src[t];
+    uint16_t* dst = a.dst[t];
     uint4 buf[kPasses];
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
-      buf[p] = src_off[p] < 0 ? make_uint4(0, 0, 0, 0)
-                              : __ldcs(reinterpret_cast<const uint4*>(srcs[t] + src_off[p]));
+      buf[p] = src_off[p] < 0 ? make_uint4(0, 0, 0, 0) : __ldcs(reinterpret_cast<const uint4*>(src + src_off[p]));
     }
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
-      *reinterpret_cast<uint4*>(dsts[t] + dst_base + (int64_t)(p * kRowsPerPass + rsub) * RF_HEAD_DIM) = buf[p];
+      *reinterpret_cast<uint4*>(dst + dst_base + (int64_t)(p * kRowsPerPass + rsub) * RF_HEAD_DIM) = buf[p];
     }
-    if (t < 2 && sparse) {
+    if (t < 2 && sparse && a.pooled[t]) {
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int p = 0; p < kPasses; ++p) acc_half8<kF16>(acc, buf[p]);
@@ -72,12 +81,12 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(
   __syncthreads();
   // 256 threads: 2 tensors x 128 columns.
   const int t = threadIdx.x >> 7, c = threadIdx.x & 127;
+  if (!a.pooled[t]) return;
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < kRowsPerPass; ++i) s += red[t][i][c];
   const int blk = tile - g.P_pad / RF_BLOCK;
-  float* dst = (t == 0 ? pooled_q : pooled_k) + ((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c;
-  *dst = s * (1.0f / RF_BLOCK);
+  a.pooled[t][((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c] = s * (1.0f / RF_BLOCK);
 }
 
 __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const uint16_t* __restrict__ o_int, int layout, int B,
@@ -103,14 +112,23 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const uint16_t*
 }  // namespace
 
 cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int dtype, int layout, int B, int S,
-                                int N, const rf_plan_t& g, void* q_int, void* k_int, void* v_int, float* pooled_q,
-                                float* pooled_k, cudaStream_t stream) {
-  dim3 grid(g.n_tiles, B * N);
+                                int Sk, int N, const rf_plan_t& g, const rf_plan_t& gk, void* q_int, void* k_int,
+                                void* v_int, float* pooled_q, float* pooled_k, cudaStream_t stream) {
   auto kern = dtype == RF_F16 ? permute_pool_kernel<true> : permute_pool_kernel<false>;
-  kern<<<grid, kPermThreads, 0, stream>>>(static_cast<const uint16_t*>(q), static_cast<const uint16_t*>(k),
-                                          static_cast<const uint16_t*>(v), layout, B, S, N, g,
-                                          static_cast<uint16_t*>(q_int), static_cast<uint16_t*>(k_int),
-                                          static_cast<uint16_t*>(v_int), pooled_q, pooled_k);
+  auto s16 = [](const void* x) { return static_cast<const uint16_t*>(x); };
+  auto d16 = [](void* x) { return static_cast<uint16_t*>(x); };
+  PermArgs a{};
+  if (S == Sk && std::memcmp(&g, &gk, sizeof(rf_plan_t)) == 0) {   // one geometry: one pass over q, k, v
+    a = PermArgs{{s16(q), s16(k), s16(v)}, {d16(q_int), d16(k_int), d16(v_int)}, {pooled_q, pooled_k}, 3};
+    kern<<<dim3(g.n_tiles, B * N), kPermThreads, 0, stream>>>(a, layout, B, S, N, g);
+    return cudaGetLastError();
+  }
+  a = PermArgs{{s16(q), nullptr, nullptr}, {d16(q_int), nullptr, nullptr}, {pooled_q, nullptr}, 1};
+  kern<<<dim3(g.n_tiles, B * N), kPermThreads, 0, stream>>>(a, layout, B, S, N, g);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  a = PermArgs{{s16(k), s16(v), nullptr}, {d16(k_int), d16(v_int), nullptr}, {pooled_k, nullptr}, 2};
+  kern<<<dim3(gk.n_tiles, B * N), kPermThreads, 0, stream>>>(a, layout, B, Sk, N, gk);
   return cudaGetLastError();
 }
 

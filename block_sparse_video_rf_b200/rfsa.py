@@ -32,7 +32,7 @@ PRECISIONS = {"native": 0, "fp8": 1}
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
            "rf_debug_set_wait", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
-           "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex"]
+           "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv"]
 
 
 class RfPlan(ctypes.Structure):
@@ -72,11 +72,13 @@ def _load():
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "rf_last_error_string": (ctypes.c_char_p, []),
-        "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfWsLayout)]),
-        "rf_workspace_size_ex": (Z, [I, I, I, I, I, I, I, I, I]),
-        "rf_prepare_ex": (I, [P, P, P, I, I] + geo + [I, I, F, P, Z, P]),
-        "rf_attend_ex": (I, [I, I] + geo + [I, I, F, F, P, P, Z, P]),
-        "rf_sparse_attention_ex": (I, [P, P, P, I, I] + geo + [I, I, F, F, P, P, Z, P]),
+        "rf_plan_kv": (I, [I, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan)]),
+        "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan),
+                                       ctypes.POINTER(RfWsLayout)]),
+        "rf_workspace_size_ex": (Z, [I, I, I, I, I, I, I, I, I, I, I, I, I]),
+        "rf_prepare_ex": (I, [P, P, P, I, I] + geo + [I, I, I, I, I, I, F, P, Z, P]),
+        "rf_attend_ex": (I, [I, I] + geo + [I, I, I, I, I, I, F, F, P, P, Z, P]),
+        "rf_sparse_attention_ex": (I, [P, P, P, I, I] + geo + [I, I, I, I, I, I, F, F, P, P, Z, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -142,87 +144,108 @@ def _nbytes(t):
     return t.numel() * t.element_size()
 
 
+def _kv(k, layout: str, latent_k):
+    """(S_kv, kv_t, kv_h, kv_w) of the _ex entry points: zeros when k and v share q's geometry."""
+    if latent_k is None:
+        return (0, 0, 0, 0)
+    return (_dims(k, layout)[1], *latent_k)
+
+
 def rf_plan(S: int, txt_len: int, latent, sparsity: float, block_size: int = 128) -> RfPlan:
     p = RfPlan()
     _check(LIB.rf_plan(S, txt_len, *latent, block_size, float(sparsity), ctypes.byref(p)))
     return p
 
 
-def rf_workspace_layout(B: int, N: int, D: int, plan: RfPlan, precision: str = "native") -> RfWsLayout:
+def rf_plan_kv(S: int, txt_len: int, latent, S_kv: int, latent_k, sparsity: float, block_size: int = 128):
+    """(query plan, key/value plan) of a call whose k and v have a geometry of their own."""
+    p, pk = RfPlan(), RfPlan()
+    _check(LIB.rf_plan_kv(S, txt_len, *latent, S_kv, *latent_k, block_size, float(sparsity), ctypes.byref(p),
+                          ctypes.byref(pk)))
+    return p, pk
+
+
+def rf_workspace_layout(B: int, N: int, D: int, plan: RfPlan, precision: str = "native",
+                        plan_kv: RfPlan | None = None) -> RfWsLayout:
     lay = RfWsLayout()
-    if precision == "native":
+    if precision == "native" and plan_kv is None:
         _check(LIB.rf_workspace_layout(B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
     else:
-        _check(LIB.rf_workspace_layout_ex(_prec(precision), B, N, D, ctypes.byref(plan), ctypes.byref(lay)))
+        _check(LIB.rf_workspace_layout_ex(_prec(precision), B, N, D, ctypes.byref(plan),
+                                          ctypes.byref(plan_kv) if plan_kv is not None else None, ctypes.byref(lay)))
     return lay
 
 
-def rf_workspace_size(B, S, N, D, txt_len, latent, precision: str = "native") -> int:
-    if precision == "native":
+def rf_workspace_size(B, S, N, D, txt_len, latent, precision: str = "native", S_kv: int = 0, latent_k=None) -> int:
+    if precision == "native" and latent_k is None:
         return int(LIB.rf_workspace_size(B, S, N, D, txt_len, *latent))
-    return int(LIB.rf_workspace_size_ex(_prec(precision), B, S, N, D, txt_len, *latent))
+    kv = (S_kv, *latent_k) if latent_k is not None else (0, 0, 0, 0)
+    return int(LIB.rf_workspace_size_ex(_prec(precision), B, S, N, D, txt_len, *latent, *kv))
 
 
 def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: float, scale=None, out=None,
-                        block_size: int = 128, stream=None, precision: str = "native"):
+                        block_size: int = 128, stream=None, precision: str = "native", latent_k=None):
     """The whole rf_v2 call on device tensors; returns ``out`` (shape, layout and type of q).
 
-    q, k, v: bf16 or fp16; precision "native" or "fp8" (see include/rfsa.h)."""
+    q, k, v: bf16 or fp16; precision "native" or "fp8"; latent_k: the (t, h, w)
+    of k and v when they have a geometry of their own (see include/rfsa.h)."""
     import torch
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
     lay = LAYOUTS.get(layout, -1)
-    if _plain(q, precision):
+    if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_sparse_attention(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
                                        float(sparsity), _scale(scale), _ptr(out), _stream(q, stream)))
     else:
         _check(LIB.rf_sparse_attention_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D,
-                                          txt_len, *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
-                                          None, 0, _stream(q, stream)))
+                                          txt_len, *latent, *_kv(k, layout, latent_k), block_size, float(sparsity),
+                                          _scale(scale), _ptr(out), None, 0, _stream(q, stream)))
     return out
 
 
 def rf_sparse_attention_ws(q, k, v, layout, txt_len, latent, sparsity, workspace, scale=None, out=None,
-                           block_size=128, stream=None, precision: str = "native"):
+                           block_size=128, stream=None, precision: str = "native", latent_k=None):
     import torch
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
     lay = LAYOUTS.get(layout, -1)
-    if _plain(q, precision):
+    if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_sparse_attention_ws(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
                                           float(sparsity), _scale(scale), _ptr(out), _ptr(workspace),
                                           _nbytes(workspace), _stream(q, stream)))
     else:
         _check(LIB.rf_sparse_attention_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D,
-                                          txt_len, *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
-                                          _ptr(workspace), _nbytes(workspace), _stream(q, stream)))
+                                          txt_len, *latent, *_kv(k, layout, latent_k), block_size, float(sparsity),
+                                          _scale(scale), _ptr(out), _ptr(workspace), _nbytes(workspace),
+                                          _stream(q, stream)))
     return out
 
 
 def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size=128, stream=None,
-               precision: str = "native"):
+               precision: str = "native", latent_k=None):
     B, S, N, D = _dims(q, layout)
     lay = LAYOUTS.get(layout, -1)
-    if _plain(q, precision):
+    if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_prepare(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
                               float(sparsity), _ptr(workspace), _nbytes(workspace), _stream(q, stream)))
     else:
         _check(LIB.rf_prepare_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N, D, txt_len,
-                                 *latent, block_size, float(sparsity), _ptr(workspace), _nbytes(workspace),
-                                 _stream(q, stream)))
+                                 *latent, *_kv(k, layout, latent_k), block_size, float(sparsity), _ptr(workspace),
+                                 _nbytes(workspace), _stream(q, stream)))
 
 
 def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, block_size=128, stream=None,
-              precision: str = "native"):
+              precision: str = "native", S_kv: int = 0, latent_k=None):
     B, S, N, D = _dims(out, layout)
     lay = LAYOUTS.get(layout, -1)
-    if _plain(out, precision):
+    kv = (S_kv, *latent_k) if latent_k is not None else (0, 0, 0, 0)
+    if _plain(out, precision) and latent_k is None:
         _check(LIB.rf_attend(lay, B, S, N, D, txt_len, *latent, block_size, float(sparsity), _scale(scale),
                              _ptr(out), _ptr(workspace), _nbytes(workspace), _stream(out, stream)))
     else:
-        _check(LIB.rf_attend_ex(_dtype(out), _prec(precision), lay, B, S, N, D, txt_len, *latent, block_size,
+        _check(LIB.rf_attend_ex(_dtype(out), _prec(precision), lay, B, S, N, D, txt_len, *latent, *kv, block_size,
                                 float(sparsity), _scale(scale), _ptr(out), _ptr(workspace), _nbytes(workspace),
                                 _stream(out, stream)))
     return out
@@ -268,13 +291,15 @@ def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
     return st.value
 
 
-def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"):
+def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native", plan_kv=None):
     """Typed torch views of the workspace regions (for inspection and tests).
 
-    dtype: torch type of the internal q/k/v copies (the input type; default bf16)."""
+    dtype: torch type of the internal q/k/v copies (the input type; default bf16).
+    plan_kv: the key/value plan when k and v have a geometry of their own."""
     import torch
     dtype = dtype or torch.bfloat16
-    lay = rf_workspace_layout(B, N, 128, plan, precision)
+    lay = rf_workspace_layout(B, N, 128, plan, precision, plan_kv)
+    pk = plan if plan_kv is None else plan_kv
     raw = workspace.view(torch.uint8)
     heads = B * N
 
@@ -282,32 +307,35 @@ def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"
         nbytes = count * torch.empty((), dtype=dtype).element_size()
         return raw[off:off + nbytes].view(dtype).view(shape)
 
-    nb, words = plan.nb, plan.mask_words
+    nb, nbk, words = plan.nb, pk.nb, pk.mask_words
     fp8 = {}
     if precision == "fp8":
-        n8 = heads * plan.S_int * 128
+        nq, nk = plan.n_tiles, pk.n_tiles
         fp8 = {
-            "q8": view(lay.q8, n8, torch.uint8, (B, N, plan.S_int, 128)),
-            "k8": view(lay.k8, n8, torch.uint8, (B, N, plan.S_int, 128)),
-            "v8": view(lay.v8, n8, torch.uint8, (B, N, plan.n_tiles, 128, 128)),
-            "scales": view(lay.scales, 3 * heads * plan.n_tiles, torch.float32, (3, B, N, plan.n_tiles)),
+            "q8": view(lay.q8, heads * plan.S_int * 128, torch.uint8, (B, N, plan.S_int, 128)),
+            "k8": view(lay.k8, heads * pk.S_int * 128, torch.uint8, (B, N, pk.S_int, 128)),
+            "v8": view(lay.v8, heads * pk.S_int * 128, torch.uint8, (B, N, nk, 128, 128)),
+            "q_scales": view(lay.scales, heads * nq, torch.float32, (B, N, nq)),
+            "k_scales": view(lay.scales + 4 * heads * nq, heads * nk, torch.float32, (B, N, nk)),
+            "v_scales": view(lay.scales + 4 * heads * (nq + nk), heads * nk, torch.float32, (B, N, nk)),
             "vmax": view(lay.vmax, heads, torch.float32, (B, N)),
         }
     return fp8 | {
         "q_int": view(lay.q_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
-        "k_int": view(lay.k_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
-        "v_int": view(lay.v_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
+        "k_int": view(lay.k_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
+        "v_int": view(lay.v_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
         "pooled_q": view(lay.pooled_q, heads * nb * 128, torch.float32, (B, N, nb, 128)),
-        "pooled_k": view(lay.pooled_k, heads * nb * 128, torch.float32, (B, N, nb, 128)),
+        "pooled_k": view(lay.pooled_k, heads * nbk * 128, torch.float32, (B, N, nbk, 128)),
         "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),
         "kept": view(lay.kept, heads * nb, torch.int32, (B, N, nb)),
         "margin": view(lay.margin, heads * nb, torch.float32, (B, N, nb)),
     }
 
 
-def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda", precision: str = "native"):
+def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda", precision: str = "native", S_kv: int = 0,
+                    latent_k=None):
     import torch
-    n = rf_workspace_size(B, S, N, D, txt_len, latent, precision)
+    n = rf_workspace_size(B, S, N, D, txt_len, latent, precision, S_kv, latent_k)
     if n == 0:
         raise RfError(2, "bad arguments for the workspace size")
     return torch.empty(n, dtype=torch.uint8, device=device)

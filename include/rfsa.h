@@ -97,12 +97,15 @@ typedef struct {
  * of row i set when query block i reads key block j; kept: int32 [B, N, nb]
  * (bits set per row); margin: fp32 [B, N, nb] (relative gap between the
  * k-th and (k+1)-th block score of the row, +inf when not defined);
- * counter: int32 work counter; status: int32 device status word.
+ * counter: int32 work counter; status: int32 device status word (both at
+ * the start of the workspace, whatever the geometry).
+ * With a key/value geometry of its own, k_int/v_int/pooled_k and the mask
+ * columns follow the key plan.
  * Only with RF_PREC_FP8 (zero-sized otherwise): q8/k8: e4m3 codes
  * [B, N, S_int, 128]; v8: e4m3 codes of V with each 128-row block stored
  * transposed ([B, N, n_tiles, 128 channels, 128 rows]); scales: fp32
- * [3 (q, k, v), B, N, n_tiles]; vmax: fp32 [B, N], the largest V block scale
- * of each head. */
+ * q [B, N, n_tiles_q], then k and v [B, N, n_tiles_kv]; vmax: fp32 [B, N],
+ * the largest V block scale of each head. */
 typedef struct {
   size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status;
   size_t q8, k8, v8, scales, vmax;
@@ -113,6 +116,13 @@ typedef struct {
 rf_status_t rf_plan(int S, int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
                     rf_plan_t* plan);
 
+/* Host-only: the plans of a call whose keys and values have a geometry of
+ * their own (S_kv, kv_t, kv_h, kv_w as in rf_prepare_ex; S_kv <= 0: the
+ * query's, and *plan_kv = *plan).  If either geometry is dense both plans
+ * come back dense (the whole sequence as the prefix, in its own order). */
+rf_status_t rf_plan_kv(int S, int txt_len, int latent_t, int latent_h, int latent_w, int S_kv, int kv_t, int kv_h,
+                       int kv_w, int block_size, float sparsity, rf_plan_t* plan, rf_plan_t* plan_kv);
+
 /* Host-only: workspace regions for B x N heads of head dim D under `plan`. */
 rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* plan, rf_ws_layout_t* layout);
 
@@ -120,11 +130,12 @@ rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* plan, rf_w
 size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int latent_t, int latent_h, int latent_w);
 
 /* Host-only: the same for a given precision (RF_PREC_FP8 adds the e4m3
- * tensors and scales). */
+ * tensors and scales) and a key/value geometry of its own (plan_kv NULL, or
+ * S_kv <= 0: the query's; see rf_prepare_ex). */
 rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D, const rf_plan_t* plan,
-                                   rf_ws_layout_t* layout);
+                                   const rf_plan_t* plan_kv, rf_ws_layout_t* layout);
 size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int latent_t,
-                            int latent_h, int latent_w);
+                            int latent_h, int latent_w, int S_kv, int kv_t, int kv_h, int kv_w);
 
 /* The whole rf_v2 call, with a workspace cached by the library per device
  * (grown with cudaMalloc on first use of a larger shape; never shrunk). */
@@ -155,25 +166,39 @@ rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_le
                       int latent_w, int block_size, float sparsity, float scale, void* out, void* workspace,
                       size_t ws_bytes, void* stream);
 
-/* rf_prepare / rf_attend / rf_sparse_attention_ws for any input type and
- * precision (the plain entry points are these with RF_BF16, RF_PREC_NATIVE).
- * The workspace must come from rf_workspace_size_ex for the same precision;
- * rf_sparse_attention_ex takes workspace = NULL (ws_bytes ignored) to use the
- * library's cached workspace.  Invalid dtype or precision: RF_ERR_ARG.
- * RF_PREC_FP8 stage 1 also quantises the reordered q, k, v (q8/k8/v8,
- * scales, vmax); its stage 2 reads only those. */
+/* rf_prepare / rf_attend / rf_sparse_attention_ws for any input type,
+ * precision and key/value geometry (the plain entry points are these with
+ * RF_BF16, RF_PREC_NATIVE and S_kv = 0).
+ * - Key/value geometry (lite_boost.ops.sparse_attention, latent_shape_k):
+ *   S_kv <= 0 means k and v have q's length and geometry (kv_* ignored).
+ *   Otherwise k and v hold S_kv = txt_len + kv_t * kv_h * kv_w tokens
+ *   (kv latent (0, 0, 0): no geometry) in the same layout, with the same
+ *   txt_len: q is reordered and blocked by its geometry, k and v by theirs;
+ *   block scores are nb_q x nb_kv, k counts key blocks, the forced columns
+ *   are the key geometry's first-frame blocks and the dense rows the query
+ *   geometry's, every query attends to the key prefix; if either geometry is
+ *   dense (no geometry, or fewer than 32 blocks) the call is dense attention
+ *   of every query over every key.  out has q's shape.  The mask region is
+ *   [B, N, nb_q, ceil(nb_kv / 32)].
+ * - The workspace must come from rf_workspace_size_ex with the same
+ *   precision and geometries; rf_sparse_attention_ex takes workspace = NULL
+ *   (ws_bytes ignored) to use the library's cached workspace.
+ * - Invalid dtype or precision: RF_ERR_ARG.
+ * - RF_PREC_FP8 stage 1 also quantises the reordered q, k, v (q8/k8/v8,
+ *   scales, vmax); its stage 2 reads only those. */
 rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype, rf_precision_t precision,
                           rf_layout_t layout, int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
-                          int latent_w, int block_size, float sparsity, void* workspace, size_t ws_bytes,
-                          void* stream);
+                          int latent_w, int S_kv, int kv_t, int kv_h, int kv_w, int block_size, float sparsity,
+                          void* workspace, size_t ws_bytes, void* stream);
 rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
-                         int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
-                         float scale, void* out, void* workspace, size_t ws_bytes, void* stream);
+                         int txt_len, int latent_t, int latent_h, int latent_w, int S_kv, int kv_t, int kv_h,
+                         int kv_w, int block_size, float sparsity, float scale, void* out, void* workspace,
+                         size_t ws_bytes, void* stream);
 rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype,
                                    rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
-                                   int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
-                                   float sparsity, float scale, void* out, void* workspace, size_t ws_bytes,
-                                   void* stream);
+                                   int txt_len, int latent_t, int latent_h, int latent_w, int S_kv, int kv_t,
+                                   int kv_h, int kv_w, int block_size, float sparsity, float scale, void* out,
+                                   void* workspace, size_t ws_bytes, void* stream);
 
 /* Inverse reorder alone: o_int [B, N, S_int, 128] of 16-bit values (internal
  * order) -> out in the caller's layout.  Pad rows are skipped. */
@@ -191,7 +216,9 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
 
 /* Synchronises `stream`, reads the workspace status word into *status
  * (0 = fine, otherwise an rf_status_t code recorded by a kernel) and clears
- * it.  Returns RF_OK or RF_ERR_CUDA. */
+ * it.  The status word sits at the same place in every workspace (any
+ * precision or key geometry); the plan only validates the arguments.
+ * Returns RF_OK, RF_ERR_ARG, RF_ERR_WORKSPACE or RF_ERR_CUDA. */
 rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                            int* status, void* stream);
 

@@ -113,14 +113,22 @@ def test_entry_points_validate_before_any_cuda_call(rfsa):
                                     fake, P(0x10000), 1 << 40, None) == 2
 
 
+def _regions_disjoint(lay, sizes):
+    spans = sorted((getattr(lay, f), getattr(lay, f) + n) for f, n in sizes.items() if n)
+    return all(a_end <= b_start for (_, a_end), (b_start, _) in zip(spans, spans[1:])) and spans[-1][1] <= lay.total
+
+
 def test_workspace_layout_is_aligned_and_sized(rfsa):
     p = rfsa.rf_plan(62752, 256, (62, 24, 42), 0.8)
     lay = rfsa.rf_workspace_layout(1, 56, 128, p)
     offs = [getattr(lay, f) for f in rfsa.WS_FIELDS]
     assert all(o % 256 == 0 for o in offs)
-    assert offs == sorted(offs)
+    assert lay.counter == 0 and lay.status == 256          # independent of the geometry
     tensor = 56 * 62848 * 128 * 2
-    assert lay.k_int - lay.q_int >= tensor and lay.total > 3 * tensor
+    rows = 56 * p.nb
+    assert _regions_disjoint(lay, {"counter": 4, "status": 4, "q_int": tensor, "k_int": tensor, "v_int": tensor,
+                                   "pooled_q": rows * 512, "pooled_k": rows * 512, "mask": rows * p.mask_words * 4,
+                                   "kept": rows * 4, "margin": rows * 4})
     assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42)) == lay.total
 
 
@@ -128,7 +136,7 @@ def test_ex_entry_points_validate_dtype_and_precision(rfsa):
     L = rfsa.LIB
     P = ctypes.c_void_p
     fake = P(0x1000)
-    geo = (0, 1, 4096, 2, 128, 0, 4, 32, 32, 128, 0.5, 0.0)
+    geo = (0, 1, 4096, 2, 128, 0, 4, 32, 32, 0, 0, 0, 0, 128, 0.5, 0.0)
     # dtype 5 / precision 3 -> RF_ERR_ARG before any CUDA call
     assert L.rf_sparse_attention_ex(fake, fake, fake, 5, 0, *geo, P(0x2000), None, 0, None) == 2
     assert b"dtype" in L.rf_last_error_string()
@@ -136,6 +144,9 @@ def test_ex_entry_points_validate_dtype_and_precision(rfsa):
     assert b"precision" in L.rf_last_error_string()
     assert L.rf_prepare_ex(fake, fake, fake, 1, 1, *geo[:-1], P(0x10000), 16, None) == 5   # fp8 workspace too small
     assert L.rf_attend_ex(1, 9, *geo, P(0x2000), P(0x10000), 1 << 40, None) == 2
+    # a key/value geometry whose length does not match its latent -> RF_ERR_ARG
+    kv_bad = (0, 1, 4096, 2, 128, 0, 4, 32, 32, 5000, 4, 32, 40, 128, 0.5, 0.0)
+    assert L.rf_sparse_attention_ex(fake, fake, fake, 0, 0, *kv_bad, P(0x2000), None, 0, None) == 2
     assert rfsa.rf_workspace_size(1, 4096, 2, 128, 0, (4, 32, 32), precision="fp8") > 0
     with pytest.raises(rfsa.RfError):
         rfsa.rf_workspace_layout(1, 2, 128, rfsa.rf_plan(4096, 0, (4, 32, 32), 0.5), precision="fp4")
@@ -146,10 +157,10 @@ def test_fp8_workspace_layout(rfsa):
     nat = rfsa.rf_workspace_layout(1, 56, 128, p)
     lay = rfsa.rf_workspace_layout(1, 56, 128, p, precision="fp8")
     offs = [getattr(lay, f) for f in rfsa.WS_FIELDS]
-    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    assert all(o % 256 == 0 for o in offs)
     codes = 56 * 62848 * 128
-    assert lay.k8 - lay.q8 >= codes and lay.v8 - lay.k8 >= codes and lay.scales - lay.v8 >= codes
-    assert lay.vmax - lay.scales >= 3 * 56 * p.n_tiles * 4 and lay.total - lay.vmax >= 56 * 4
+    assert _regions_disjoint(lay, {"q_int": 2 * codes, "v_int": 2 * codes, "q8": codes, "k8": codes, "v8": codes,
+                                   "scales": 3 * 56 * p.n_tiles * 4, "vmax": 56 * 4})
     # the native layout is the same up to the fp8 regions, which it leaves empty
     assert [getattr(nat, f) for f in rfsa.WS_FIELDS[:10]] == offs[:10]
     assert nat.q8 == nat.k8 == nat.v8 == nat.scales == nat.vmax == nat.total
@@ -163,3 +174,24 @@ def test_block_count_limit(rfsa):
     with pytest.raises(rfsa.RfError) as e:
         rfsa.rf_plan(64 * 64 * 129, 0, (129, 64, 64), 0.5)     # 4128 blocks
     assert e.value.code == 3
+
+
+def test_key_geometry_workspace(rfsa):
+    import oracle
+    pq = rfsa.rf_plan(16 + 4 * 32 * 32, 16, (4, 32, 32), 0.7)
+    pk = rfsa.rf_plan(16 + 5 * 32 * 40, 16, (5, 32, 40), 0.7)
+    assert pq.nb == 32 and pk.nb == 50
+    lay = rfsa.rf_workspace_layout(2, 3, 128, pq, "native", pk)
+    heads = 6
+    assert _regions_disjoint(lay, {"q_int": heads * pq.S_int * 256, "k_int": heads * pk.S_int * 256,
+                                   "v_int": heads * pk.S_int * 256, "pooled_q": heads * pq.nb * 512,
+                                   "pooled_k": heads * pk.nb * 512, "mask": heads * pq.nb * pk.mask_words * 4,
+                                   "kept": heads * pq.nb * 4, "margin": heads * pq.nb * 4})
+    n = rfsa.rf_workspace_size(2, 16 + 4096, 3, 128, 16, (4, 32, 32), "native", 16 + 6400, (5, 32, 40))
+    assert n == lay.total
+    # either side dense makes both dense: the query side here has 6 blocks, so a
+    # sparse key geometry sizes the workspace like a key side without geometry
+    assert oracle.geometry(7 + 768, 7, 3, 16, 16).dense
+    n2 = rfsa.rf_workspace_size(1, 7 + 768, 1, 128, 7, (3, 16, 16), "native", 7 + 6400, (5, 32, 40))
+    n3 = rfsa.rf_workspace_size(1, 7 + 768, 1, 128, 7, (3, 16, 16), "native", 7 + 6400, (0, 0, 0))
+    assert n2 == n3 > 0

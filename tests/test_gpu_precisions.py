@@ -135,19 +135,19 @@ def test_fp8_quantisation_is_bit_exact(rfsa, case, dtype):
     g = oracle.geometry(w.S, w.txt_len, *w.latent)
     n_tiles = plan.n_tiles
     assert len(fp8.internal_tiles(g)) == n_tiles
-    scales = views["scales"].cpu().numpy()
-    for ti, (src, key) in enumerate(((q, "q8"), (k, "k8"), (v, "v8"))):
+    for src, key in ((q, "q"), (k, "k"), (v, "v")):
         xb = to_bnsd_np(src, w.layout)
-        got = views[key].cpu().numpy()
+        got = views[key + "8"].cpu().numpy()
+        scales = views[key + "_scales"].cpu().numpy()
         for b in range(w.B):
             for n in range(w.N):
                 _, codes, sc = fp8.quantize_head(xb[b, n], g)
-                np.testing.assert_array_equal(scales[ti, b, n].view(np.uint32), sc.view(np.uint32))
-                if key == "v8":
+                np.testing.assert_array_equal(scales[b, n].view(np.uint32), sc.view(np.uint32))
+                if key == "v":
                     np.testing.assert_array_equal(got[b, n], codes.transpose(0, 2, 1))
                 else:
                     np.testing.assert_array_equal(got[b, n].reshape(n_tiles, 128, 128), codes)
-    np.testing.assert_array_equal(views["vmax"].cpu().numpy(), scales[2].max(axis=-1))
+    np.testing.assert_array_equal(views["vmax"].cpu().numpy(), views["v_scales"].cpu().numpy().max(axis=-1))
 
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
