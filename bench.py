@@ -52,15 +52,22 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+# The attention kernels' sources, hashed together to tie a traffic capture to the code it measured.
+K3_SOURCES = ("rf_attn_common.cuh", "rf_attn_chain.cu", "rf_attn.cu")
+
+
 def _k3_traffic(heads: int):
     """DRAM bytes per attention launch from the committed ncu summary, scaled to
     ``heads``; None when the kernel source changed since the capture."""
     import hashlib
-    src = os.path.join(ROOT, "block_sparse_video_rf_b200", "csrc", "rf_attn.cu")
+    csrc = os.path.join(ROOT, "block_sparse_video_rf_b200", "csrc")
     path = os.path.join(ROOT, "profiles", "k3_traffic.txt")
     if not os.path.exists(path):
         return None
-    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for name in K3_SOURCES:
+        h.update(open(os.path.join(csrc, name), "rb").read())
+    digest = h.hexdigest()[:16]
     for line in open(path):
         parts = line.split()
         if len(parts) >= 3 and not line.startswith("#") and parts[0] == "attn_kernel" and parts[1] == digest:
@@ -349,7 +356,9 @@ def main():
             "roofline": {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": k3_tflops / peak,
                          "traffic": _k3_traffic(w.N) if default_mode else None, "peak_source": peak_note},
-            "gpu_launches": (4 if prec == "fp8" else 3) * args.steps,
+            # K1, K2 and K3 (fp8: and the quantisation pass; 16-bit: K3 is the chain kernel and its
+            # second pass, which returns at once when no unit was handed to it)
+            "gpu_launches": 4 * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -249,6 +249,7 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
   L.v8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
   L.scales = take(fp8 ? heads * (g->n_tiles + 2 * (size_t)gk->n_tiles) * 4 : 0);
   L.vmax = take(fp8 ? heads * 4 : 0);
+  L.redo = take(fp8 ? 0 : (2 + heads * g->n_tiles) * 4);
   L.total = off;
   *lay = L;
   return ok();
@@ -333,7 +334,7 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
   else
     e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
                              at<uint32_t>(ws, L.mask), dtype, layout, B, S, N, g, gk, resolve_scale(scale, D), out,
-                             at<int>(ws, L.counter), at<int>(ws, L.status), debug_settings(), s);
+                             at<int>(ws, L.counter), at<int>(ws, L.status), at<int>(ws, L.redo), debug_settings(), s);
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return ok();
 }
@@ -478,6 +479,15 @@ rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q) {
   std::lock_guard<std::mutex> lock(g_debug_mu);
   g_debug.wait_limit_ns = wait_limit_ns;
   g_debug.skip_first_q = skip_first_q;
+  return ok();
+}
+
+rf_status_t rf_debug_set_path(int path, float sum_limit) {
+  if ((path != 0 && path != 1) || !(sum_limit >= 0.f))
+    return fail(RF_ERR_ARG, "path must be 0 or 1 and sum_limit >= 0");
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  g_debug.path = path;
+  g_debug.sum_limit = sum_limit;
   return ok();
 }
 

@@ -1,19 +1,15 @@
-// Block-sparse flash attention on sm_100a tensor cores (K3).
+// Block-sparse flash attention on sm_100a tensor cores (K3), two query
+// tiles per CTA: the fp8 path, and the second pass of the 16-bit path (the
+// units chain_kernel hands back, see rf_attn_chain.cu).
 //
-// lite_boost.ops.sparse_attention, rf_v2 pipeline: rain_fusion_attention
-// over the kept KV blocks, then the inverse reorder (fused here: each output
-// row is written straight to its token's place in the caller's layout).
 // vllm-omni "RainFusion Attention", intro: prefix rows and first-frame
 // blocks stay dense; every other query block attends to its highest-scoring
-// key blocks.
-//
-// Work unit: one 128-row query tile of one (b, head).  Its KV list is every
-// key prefix tile, then either every key block (dense tile) or the blocks
-// set in its mask row, in ascending order.  Keys and values may have a
-// geometry of their own (lite_boost.ops.sparse_attention, latent_shape_k):
-// query tiles follow the query plan, KV tiles the key plan.  Persistent CTAs (one per SM) take
+// key blocks.  Keys and values may have a geometry of their own
+// (lite_boost.ops.sparse_attention, latent_shape_k): query tiles follow the
+// query plan, KV tiles the key plan.  Persistent CTAs (one per SM) take
 // units from a global counter in (head, tile) order, dense tiles of a head
-// first, so the heads in flight keep their K/V in L2.
+// first, so the heads in flight keep their K/V in L2; in list mode they take
+// the units listed by chain_kernel instead.
 //
 // A CTA runs two units at once in two independent slots, each with its own
 // Q/K/V shared-memory buffers, its own S and O in tensor memory and its own
@@ -54,16 +50,7 @@
 //     columns) and carries the V block's scale relative to the head's
 //     largest one (sv / vmax, folded into the exponent), which the epilogue
 //     multiplies back; two K and two V buffers per slot.
-#include <cuda.h>
-#include <cuda_bf16.h>
-#include <cuda_runtime.h>
-#include <math_constants.h>
-
-#include <algorithm>
-
-#include "rf_geometry.h"
-#include "rf_kernels.h"
-#include "sm100_ptx.cuh"
+#include "rf_attn_common.cuh"
 
 namespace rf {
 
@@ -73,35 +60,7 @@ constexpr int kThreads = 384;
 constexpr int kSlots = 2;
 constexpr int kSlotWarps = 4;                            // softmax warps per slot
 constexpr uint32_t kRegsSoftmax = 216, kRegsControl = 64;
-constexpr int kBoxBytes = RF_BLOCK * 128;                // one TMA box: 128 rows x 128 bytes
 constexpr uint32_t kTmemCols = 512;
-
-constexpr float kRescaleThreshold = 8.0f;                // log2 units
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-
-// Compile-time shape of one precision.
-template <bool kF16_, bool kFp8_>
-struct Cfg {
-  static constexpr bool kF16 = kF16_;                    // 16-bit type: fp16 (else bf16); also the output type
-  static constexpr bool kFp8 = kFp8_;
-  static constexpr int kBoxes = kFp8 ? 1 : 2;            // boxes per 128 x 128 tile
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static constexpr int kKStages = kFp8 ? 2 : 1;
-  static constexpr int kVStages = kFp8 ? 2 : 1;
-  static constexpr int kSteps = kFp8 ? 4 : 8;            // MMAs per product over 128 (K 32 or 16 each)
-  static constexpr int kPCols = kFp8 ? 32 : 64;          // TMEM columns of P
-  // exponent pair i runs the polynomial on the FMA pipe when i % kPolyEvery == kPolyEvery - 1
-  // (the rest on MUFU): measured best split for each path
-  static constexpr int kPolyEvery = kFp8 ? 3 : 4;
-  static constexpr uint32_t kIdescQK =
-      kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, false, !kF16);
-  static constexpr uint32_t kIdescPV =
-      kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, true, !kF16);
-};
-
-struct Item {
-  int bn, qt, ntiles, pad;
-};
 
 // Per-tile factors of the fp8 path, written by the slot's issuer before its
 // arrival on s_full: c = scale * log2(e) * sq * sk (multiplies S), lr =
@@ -136,104 +95,7 @@ struct Smem {
   int abort;
 };
 
-struct AttnParams {
-  rf_plan_t g;       // query geometry (units, dense rows, the output's token order)
-  rf_plan_t gk;      // key/value geometry (KV lists; the same as g unless k and v have their own)
-  int B, S, N, layout;   // S: query sequence length (the output's)
-  int total_items;
-  int n_ptiles;      // query prefix tiles (g.P_pad / 128)
-  int n_ptiles_k;    // key prefix tiles (gk.P_pad / 128)
-  int p_rem_k;       // valid rows of the last key prefix tile when it is partial, else 0
-  float scale_log2;
-  const uint32_t* mask;  // [B*N, g.nb, gk.mask_words]
-  const float* scales;   // fp8: q [B*N, g.n_tiles], then k and v [B*N, gk.n_tiles] block scales
-  const float* vmax;     // fp8: [B*N] largest V block scale of each head
-  int* counter;
-  int* status;
-  void* out;
-  uint64_t wait_limit_ns;   // limit of every device-side wait
-  int skip_first_q;         // test control: the first unit's Q load is never issued
-};
-
-__device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
-  return p.g.dense || qt < p.n_ptiles || (qt - p.n_ptiles) < p.g.ff;
-}
-
-// Bounded wait by one thread.
-template <class C>
-__device__ __forceinline__ bool wait1(Smem<C>& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
-  return rf_wait(bar, parity, &sm.abort, p.status, RF_ERR_TIMEOUT, p.wait_limit_ns);
-}
-// Bounded wait by a whole warp, with a warp-uniform outcome (the warp then
-// runs .sync.aligned tcgen05 instructions together or leaves together).
-template <class C>
-__device__ __forceinline__ bool waitw(Smem<C>& sm, const AttnParams& p, uint64_t* bar, uint32_t parity) {
-  return __all_sync(0xFFFFFFFFu, wait1(sm, p, bar, parity));
-}
-// One arrival per warp, after every lane's preceding work (callers fence first).
-__device__ __forceinline__ void arrive_w(uint64_t* bar) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
-}
-// Parity of completion number n (0-based) of a barrier phase.
-__device__ __forceinline__ uint32_t ph(uint32_t n) { return n & 1u; }
-
-template <uint32_t N>
-__device__ __forceinline__ void regs_increase() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <uint32_t N>
-__device__ __forceinline__ void regs_decrease() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
-
 // ---------------------------------------------------------------- producer
-// Visits the KV tile rows of one unit in order: every prefix tile, then every
-// sparse block (dense unit) or the set bits of its mask row.
-struct KvIter {
-  int base, n_ptiles, nb, words;
-  const uint32_t* mrow;   // nullptr for a dense unit
-  int t, wd;
-  uint32_t bits;
-  __device__ void init(int base_, const AttnParams& p, const uint32_t* mrow_) {
-    base = base_;
-    n_ptiles = p.n_ptiles_k;
-    nb = p.gk.nb;
-    words = p.gk.mask_words;
-    mrow = mrow_;
-    t = 0;
-    wd = 0;
-    bits = 0;
-  }
-  // Row of the next KV tile, or -1 at the end.
-  __device__ int next() {
-    if (t < n_ptiles) return base + (t++) * RF_BLOCK;
-    if (!mrow) {
-      const int j = t - n_ptiles;
-      if (j >= nb) return -1;
-      ++t;
-      return base + (n_ptiles + j) * RF_BLOCK;
-    }
-    while (bits == 0) {
-      if (wd >= words) return -1;
-      bits = mrow[wd++];
-    }
-    const int j = 32 * (wd - 1) + __ffs(bits) - 1;
-    bits &= bits - 1;
-    return base + (n_ptiles + j) * RF_BLOCK;
-  }
-};
-
-// One 128 x 128 tile: one box of 128 bytes per row (fp8) or two boxes of 64
-// 16-bit columns.
-template <class C>
-__device__ __forceinline__ void load_tile(uint8_t* dst, const CUtensorMap* map, uint64_t* bar, int row,
-                                          uint64_t policy) {
-  mbar_arrive_expect_tx(bar, C::kTileBytes);
-#pragma unroll
-  for (int b = 0; b < C::kBoxes; ++b) tma_load_2d(dst + b * kBoxBytes, map, bar, b * 64, row, policy);
-}
-
 // Producer of one slot: takes units from the global counter, loads Q and then
 // the K and V tiles of the KV list into rings of kKStages / kVStages buffers
 // (K of tile t once S of tile t - stages is done, V once P V of tile
@@ -248,26 +110,14 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
   const int BN = p.B * p.N;
   bool ok = true;
   while (ok) {
-    const int w = atomicAdd(p.counter, 1);
+    const int w = atomicAdd(p.list_mode ? &p.redo[0] : p.counter, 1);
     const uint32_t it = c & 1;
-    if (c >= 2 && !wait1(sm, p, &sl.item_empty[it], ph((c >> 1) - 1))) {
+    if (c >= 2 && !wait1(&sm.abort, p, &sl.item_empty[it], ph((c >> 1) - 1))) {
       ok = false;
       break;
     }
-    Item itm{-1, 0, 0, 0};
-    const uint32_t* mrow = nullptr;
-    if (w < p.total_items) {
-      itm.bn = w / p.g.n_tiles;
-      itm.qt = w - itm.bn * p.g.n_tiles;
-      if (is_dense_tile(p, itm.qt)) {
-        itm.ntiles = p.gk.n_tiles;
-      } else {
-        mrow = p.mask + ((size_t)itm.bn * p.g.nb + (itm.qt - p.n_ptiles)) * p.gk.mask_words;
-        int cnt = 0;
-        for (int wd = 0; wd < p.gk.mask_words; ++wd) cnt += __popc(mrow[wd]);
-        itm.ntiles = p.n_ptiles_k + cnt;
-      }
-    }
+    const uint32_t* mrow;
+    const Item itm = make_item(p, unit_of(p, w), mrow);
     sl.items[it] = itm;
     mbar_arrive(&sl.item_full[it]);
     if (itm.bn < 0) break;
@@ -275,7 +125,7 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
     const int base = itm.bn * S_int_k;   // the unit's KV rows
     const float* sc_k = C::kFp8 ? p.scales + (size_t)BN * p.g.n_tiles + (size_t)itm.bn * p.gk.n_tiles : nullptr;
     const float* sc_v = C::kFp8 ? sc_k + (size_t)BN * p.gk.n_tiles : nullptr;
-    if (c >= 1 && !wait1(sm, p, &sl.q_empty, ph(c - 1))) {
+    if (c >= 1 && !wait1(&sm.abort, p, &sl.q_empty, ph(c - 1))) {
       ok = false;
       break;
     }
@@ -288,7 +138,7 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
     kit.init(base, p, mrow);
     for (int row = kit.next(); row >= 0 && ok; row = kit.next()) {
       const uint32_t ks = nk % C::kKStages, ku = nk / C::kKStages;
-      if (ku >= 1 && !wait1(sm, p, &sl.k_empty[ks], ph(ku - 1))) {
+      if (ku >= 1 && !wait1(&sm.abort, p, &sl.k_empty[ks], ph(ku - 1))) {
         ok = false;
         break;
       }
@@ -300,7 +150,7 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
       load_tile<C>(sl.k[ks], tk, &sl.k_full[ks], row, pol_kv);
       ++nk;
       const uint32_t vs = nv % C::kVStages, vu = nv / C::kVStages;
-      if (vu >= 1 && !wait1(sm, p, &sl.v_empty[vs], ph(vu - 1))) {
+      if (vu >= 1 && !wait1(&sm.abort, p, &sl.v_empty[vs], ph(vu - 1))) {
         ok = false;
         break;
       }
@@ -324,40 +174,6 @@ __device__ void producer_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, con
   }
 }
 
-// ---------------------------------------------------------------- MMA issue
-// Descriptor low words of the 128-byte swizzled operands; every descriptor
-// used here shares one high word (stride 1024 B, sm_100 version, swizzle).
-// A K step (16 16-bit or 32 8-bit elements) advances a K-major operand by
-// 32 B (2 in the descriptor's 16-byte units); the second box of a 16-bit
-// tile (columns 64..127) starts 16 KB further.  The issuing warp runs this
-// code together; one elected lane issues.
-template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
-#pragma unroll
-  for (int kk = 0; kk < C::kSteps; ++kk) {
-    const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-    if (C::kFp8)
-      mma_ss_lo_elect_f8(s_tmem, q_lo + off, k_lo + off, hi, C::kIdescQK, kk > 0);
-    else
-      mma_ss_lo_elect(s_tmem, q_lo + off, k_lo + off, hi, C::kIdescQK, kk > 0);
-  }
-}
-// P V: a K step takes the next 8 TMEM columns of P (16 16-bit or 32 8-bit
-// keys).  16-bit V is MN-major: 16 keys are 16 rows of 128 B further.  fp8 V
-// is stored transposed (K-major): 32 keys are 32 B further.
-template <class C>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
-                                         bool accumulate) {
-#pragma unroll
-  for (int kk = 0; kk < C::kSteps; ++kk) {
-    const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
-    if (C::kFp8)
-      mma_ts_lo_elect_f8(o_tmem, p_tmem + kk * 8, v_lo + kk * 2, hi, C::kIdescPV, acc);
-    else
-      mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, C::kIdescPV, acc);
-  }
-}
-
 // Rendezvous of a slot's four warps (named barrier `id`, 128 threads) that
 // also returns whether every thread passed `ok`: the warps of a slot leave
 // together, so none is left waiting at a later rendezvous.
@@ -373,83 +189,6 @@ __device__ __forceinline__ bool slot_vote(int id, bool ok) {
 }
 
 // ---------------------------------------------------------------- softmax of one tile
-// P = 2^(s c + off) for the row's 128 scores s (already in registers), with
-// the tile's sum of P; writes the packed P words.
-template <class C>
-__device__ __forceinline__ float exp_tile(const uint32_t (&s)[4][32], float c, float off, int p_valid,
-                                          uint32_t (&pk)[C::kPCols]) {
-  const uint64_t c2 = f2_pack(c, c);
-  const uint64_t negm = f2_pack(off, off);
-  const bool partial = p_valid < RF_BLOCK;
-  uint64_t sum2[4] = {0, 0, 0, 0};
-  float hold0 = 0.f, hold1 = 0.f;   // fp8: the first pair of a 4-key word
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-    for (int e = 0; e < 32; e += 2) {
-      const int i = 16 * q4 + (e >> 1);     // pair index 0..63
-      const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1])), c2, negm);
-      uint64_t p2;
-      if ((i % C::kPolyEvery) == C::kPolyEvery - 1) {
-        p2 = exp2_poly_x2(x2);
-      } else {
-        float x0, x1;
-        f2_unpack(x2, x0, x1);
-        p2 = f2_pack(ex2_approx(x0), ex2_approx(x1));
-      }
-      if (partial) {
-        float a0, a1;
-        f2_unpack(p2, a0, a1);
-        p2 = f2_pack(2 * i < p_valid ? a0 : 0.f, 2 * i + 1 < p_valid ? a1 : 0.f);
-      }
-      sum2[i & 3] = f2_add(sum2[i & 3], p2);
-      float a0, a1;
-      f2_unpack(p2, a0, a1);
-      if (C::kFp8) {
-        if (i & 1)
-          pk[i >> 1] = pack_e4m3x4(hold0, hold1, a0, a1);
-        else {
-          hold0 = a0;
-          hold1 = a1;
-        }
-      } else {
-        pk[i] = pack_half2<C::kF16>(a0, a1);
-      }
-    }
-  float s0, s1, s2, s3;
-  f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
-  f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);
-  return (s0 + s1) + (s2 + s3);
-}
-
-template <class C>
-__device__ __forceinline__ void load_scores(uint32_t tS, int p_valid, uint32_t (&s)[4][32]) {
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + 32 * q4, s[q4]);
-  tmem_wait_ld();
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4) reg_fence32(s[q4]);
-  if (p_valid < RF_BLOCK) {
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        if (32 * q4 + e >= p_valid) s[q4][e] = __float_as_uint(-CUDART_INF_F);
-  }
-}
-
-__device__ __forceinline__ float row_max(const uint32_t (&s)[4][32]) {
-  float mx8[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) mx8[i] = -CUDART_INF_F;
-#pragma unroll
-  for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-    for (int e = 0; e < 32; e += 2)
-      mx8[(e >> 1) & 7] = max3f(mx8[(e >> 1) & 7], __uint_as_float(s[q4][e]), __uint_as_float(s[q4][e + 1]));
-  return max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
-}
-
 // Thread = query row.  Reads the row's 128 scores from S and writes P =
 // 2^(s c - m_use + lr) over the first columns of S (64 words of two 16-bit
 // values, or (fp8) 32 words of four e4m3 codes), adding the tile's sum of P
@@ -467,24 +206,24 @@ __device__ __forceinline__ void softmax_tile(uint32_t tS, uint32_t tO, bool firs
   constexpr float kSumLimit = C::kFp8 ? 448.f : 65536.f;
   uint32_t s[4][32];
   uint32_t pk[C::kPCols];
-  load_scores<C>(tS, p_valid, s);
+  load_scores<4>(tS, p_valid, s);
   float alpha = 1.f;
   bool rescale = false;
   float tsum;
   if (first) {
-    m_use = row_max(s) * c;
-    tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+    m_use = row_max<4>(s) * c;
+    tsum = exp_scores<C, 4>(s, c, lr - m_use, p_valid, pk);
   } else {
-    tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+    tsum = exp_scores<C, 4>(s, c, lr - m_use, p_valid, pk);
     if (__any_sync(0xFFFFFFFFu, !(tsum <= kSumLimit))) {
-      load_scores<C>(tS, p_valid, s);
-      const float mx_s = row_max(s) * c;
+      load_scores<4>(tS, p_valid, s);
+      const float mx_s = row_max<4>(s) * c;
       if (mx_s > m_use + kRescaleThreshold) {
         alpha = ex2_approx(m_use - mx_s);
         m_use = mx_s;
         rescale = true;
       }
-      tsum = exp_tile<C>(s, c, lr - m_use, p_valid, pk);
+      tsum = exp_scores<C, 4>(s, c, lr - m_use, p_valid, pk);
     }
   }
   l = l * alpha + tsum * ir;
@@ -537,10 +276,10 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
   // ts[tt & 1], and the issuer's arrival on s_full publishes them.
   auto qk = [&](uint32_t tt, bool last_of_unit) -> bool {
     const uint32_t ks = tt % C::kKStages;
-    if (!waitw(sm, p, &sl.k_full[ks], ph(tt / C::kKStages))) return false;
+    if (!waitw(&sm.abort, p, &sl.k_full[ks], ph(tt / C::kKStages))) return false;
     // read before the MMAs: once they finish, the producer may refill the stage
     const float sk = C::kFp8 ? sl.kv_scale[ks][0] : 0.f, sv = C::kFp8 ? sl.kv_scale[ks][1] : 0.f;
-    if (tt >= 1 && !waitw(sm, p, &sl.pv_done, ph(tt - 1))) return false;
+    if (tt >= 1 && !waitw(&sm.abort, p, &sl.pv_done, ph(tt - 1))) return false;
     tc_fence_after();
     issue_qk<C>(s_tmem, q_lo, k_lo0 + ks * (C::kTileBytes >> 4), hi);
     mma_commit_elect(&sl.s_full);
@@ -569,7 +308,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
     // failed carries ok = false to the next one, where all four leave.
     const uint32_t it = c & 1;
     Item itm{-1, 0, 0, 0};
-    if (ok) ok = waitw(sm, p, &sl.item_full[it], ph(c >> 1));
+    if (ok) ok = waitw(&sm.abort, p, &sl.item_full[it], ph(c >> 1));
     if (ok) {
       itm = sl.items[it];
       arrive_w(&sl.item_empty[it]);
@@ -577,7 +316,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
     ok = slot_vote(bar_id, ok);
     if (!ok || itm.bn < 0) break;
     if (issuer) {
-      ok = waitw(sm, p, &sl.q_full, ph(c));
+      ok = waitw(&sm.abort, p, &sl.q_full, ph(c));
       if (C::kFp8 && ok) {
         q_scale = sl.q_scale;
         unit_vmax = p.vmax[itm.bn];
@@ -588,7 +327,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
 
     float m_use = -CUDART_INF_F, l = 0.f;
     for (int j = 0; j < itm.ntiles; ++j, ++t) {
-      if (ok) ok = waitw(sm, p, &sl.s_full, ph(t));
+      if (ok) ok = waitw(&sm.abort, p, &sl.s_full, ph(t));
       if (ok) {
         tc_fence_after();
         const int p_valid = (p.p_rem_k != 0 && j == p.n_ptiles_k - 1) ? p.p_rem_k : RF_BLOCK;
@@ -603,7 +342,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
       if (!ok) break;
       if (issuer) {
         const uint32_t vs = t % C::kVStages;
-        ok = waitw(sm, p, &sl.v_full[vs], ph(t / C::kVStages));
+        ok = waitw(&sm.abort, p, &sl.v_full[vs], ph(t / C::kVStages));
         if (ok) {
           tc_fence_after();
           issue_pv<C>(o_tmem, s_tmem, v_lo0 + vs * (C::kTileBytes >> 4), hi, j > 0);
@@ -614,7 +353,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
       }
     }
     // epilogue: O * out_scale / l of this unit once its last P V is done
-    if (ok) ok = waitw(sm, p, &sl.pv_done, ph(t - 1));
+    if (ok) ok = waitw(&sm.abort, p, &sl.pv_done, ph(t - 1));
     if (ok) {
       tc_fence_after();
       const float rl = out_scale / l;
@@ -657,6 +396,8 @@ template <class C>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  // second pass with nothing listed: leave before any setup
+  if (p.list_mode && p.redo[1] == 0) return;
   extern __shared__ uint8_t smem_raw[];
   Smem<C>& sm = *reinterpret_cast<Smem<C>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -716,74 +457,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult qres;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qres) == cudaSuccess &&
-        qres == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(ptr);
-  }
-  return fn;
-}
-
-// [rows, 128] elements of `elem_bytes` (2: bf16/fp16, 1: e4m3 codes),
-// row-major; boxes of 128 rows x 128 bytes, 128-byte swizzle.
-bool make_tile_map(CUtensorMap* map, const void* base, uint64_t rows, CUtensorMapDataType type, int elem_bytes) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[2] = {RF_HEAD_DIM, rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)RF_HEAD_DIM * elem_bytes};
-  const cuuint32_t box[2] = {(cuuint32_t)(128 / elem_bytes), RF_BLOCK};
-  const cuuint32_t estr[2] = {1, 1};
-  return enc(map, type, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-AttnParams make_params(const uint32_t* mask, int layout, int B, int S, int N, const rf_plan_t& g,
-                       const rf_plan_t& gk, float scale, void* out, int* counter, int* status, const AttnDebug& dbg) {
-  AttnParams p;
-  p.g = g;
-  p.gk = gk;
-  p.B = B;
-  p.S = S;
-  p.N = N;
-  p.layout = layout;
-  p.total_items = B * N * g.n_tiles;
-  p.n_ptiles = g.P_pad / RF_BLOCK;
-  p.n_ptiles_k = gk.P_pad / RF_BLOCK;
-  p.p_rem_k = gk.P % RF_BLOCK;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.mask = mask;
-  p.scales = nullptr;
-  p.vmax = nullptr;
-  p.counter = counter;
-  p.status = status;
-  p.out = out;
-  p.wait_limit_ns = dbg.wait_limit_ns > 0 ? (uint64_t)dbg.wait_limit_ns : kWaitLimitNs;
-  p.skip_first_q = dbg.skip_first_q;
-  return p;
-}
-
 template <class C>
 cudaError_t launch_cfg(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
                        cudaStream_t stream) {
-  int dev = 0, sms = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = 0;
+  cudaError_t e = sm_count(&sms);
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(Smem<C>) + 1024;
   e = cudaFuncSetAttribute(attn_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(p.counter, 0, sizeof(int), stream);
-  if (e != cudaSuccess) return e;
+  if (!p.list_mode) {
+    e = cudaMemsetAsync(p.counter, 0, sizeof(int), stream);
+    if (e != cudaSuccess) return e;
+  }
   const int grid = std::min(sms, p.total_items);
   attn_kernel<C><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
@@ -791,10 +477,10 @@ cudaError_t launch_cfg(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 
 }  // namespace
 
-cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
-                             int dtype, int layout, int B, int S, int N, const rf_plan_t& g, const rf_plan_t& gk,
-                             float scale, void* out, int* counter, int* status, const AttnDebug& dbg,
-                             cudaStream_t stream) {
+cudaError_t launch_attention_slots(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
+                                   int dtype, int layout, int B, int S, int N, const rf_plan_t& g,
+                                   const rf_plan_t& gk, float scale, void* out, int* counter, int* status, int* redo,
+                                   int list_mode, const AttnDebug& dbg, cudaStream_t stream) {
   const uint64_t rows_q = (uint64_t)B * N * g.S_int, rows_k = (uint64_t)B * N * gk.S_int;
   const bool f16 = dtype == RF_F16;
   const CUtensorMapDataType type = f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -802,7 +488,8 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
   if (!make_tile_map(&tq, q_int, rows_q, type, 2) || !make_tile_map(&tk, k_int, rows_k, type, 2) ||
       !make_tile_map(&tv, v_int, rows_k, type, 2))
     return cudaErrorInvalidValue;
-  const AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, dbg);
+  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, redo, dbg);
+  p.list_mode = list_mode;
   return f16 ? launch_cfg<Cfg<true, false>>(tq, tk, tv, p, stream)
              : launch_cfg<Cfg<false, false>>(tq, tk, tv, p, stream);
 }
@@ -817,7 +504,7 @@ cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uin
       !make_tile_map(&tk, k8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
       !make_tile_map(&tv, v8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
     return cudaErrorInvalidValue;
-  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, dbg);
+  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, nullptr, dbg);
   p.scales = scales;
   p.vmax = vmax;
   return dtype == RF_F16 ? launch_cfg<Cfg<true, true>>(tq, tk, tv, p, stream)

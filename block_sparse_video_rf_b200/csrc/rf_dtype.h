@@ -43,4 +43,17 @@ __device__ __forceinline__ void unpack_half8(const uint4& u, float (&f)[8]) {
   }
 }
 
+// The two 16-bit values of one word (low half first) as fp32.
+template <bool kF16>
+__device__ __forceinline__ void unpack_half2(uint32_t w, float& lo, float& hi) {
+  if (kF16) {
+    const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&w));
+    lo = h.x;
+    hi = h.y;
+  } else {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+  }
+}
+
 }  // namespace rf

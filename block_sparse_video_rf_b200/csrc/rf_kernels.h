@@ -30,15 +30,27 @@ cudaError_t launch_mask(const float* pooled_q, const float* pooled_k, int BN, co
 struct AttnDebug {
   long long wait_limit_ns = 0;   // 0: the default limit (2 s)
   int skip_first_q = 0;          // 1: the first unit of every CTA never gets its Q tile
+  int path = 0;                  // 16-bit: 0 chain_kernel then the second pass; 1 attn_kernel over every unit
+  float sum_limit = 0.f;         // chain_kernel: tile sum of P that hands a unit on (0: the P type's headroom)
 };
 
-// K3: block-sparse flash attention over the internal layout, output written
-// straight to the caller's layout (inverse reorder fused in the epilogue).
-// Operands and output in dtype (rf_dtype_t).
+// K3, 16-bit: block-sparse flash attention over the internal layout, output
+// written straight to the caller's layout (inverse reorder fused in the
+// epilogue).  Operands and output in dtype (rf_dtype_t).  chain_kernel runs
+// every unit and lists in `redo` ([0] a work counter, [1] a count, [2 ...]
+// unit ids; 2 + B*N*g.n_tiles ints) those whose P left the type's headroom;
+// attn_kernel then computes the listed units.
 cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
                              int dtype, int layout, int B, int S, int N, const rf_plan_t& g, const rf_plan_t& gk,
-                             float scale, void* out, int* counter, int* status, const AttnDebug& dbg,
+                             float scale, void* out, int* counter, int* status, int* redo, const AttnDebug& dbg,
                              cudaStream_t stream);
+
+// attn_kernel (two query tiles per CTA, running maximum with rescaling) over
+// every unit (list_mode 0) or over the units listed in `redo` (list_mode 1).
+cudaError_t launch_attention_slots(const void* q_int, const void* k_int, const void* v_int, const uint32_t* mask,
+                                   int dtype, int layout, int B, int S, int N, const rf_plan_t& g,
+                                   const rf_plan_t& gk, float scale, void* out, int* counter, int* status, int* redo,
+                                   int list_mode, const AttnDebug& dbg, cudaStream_t stream);
 
 // fp8 quantisation of the reordered q (plan g), k and v (plan gk)
 // (RF_PREC_FP8): per (tensor, head, 128-row block) scale = amax / 448 and

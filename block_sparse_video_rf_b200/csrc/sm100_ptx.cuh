@@ -343,13 +343,15 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
 // f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted here for minimum
 // relative error on [-0.5, 0.5] (max relative error 7.5e-5, far below the
 // bf16 rounding of P); 2^n by adding n to the exponent field.  Inputs are
-// clamped at -125 so the exponent field stays normal: anything below gives
-// 2^-125 (about 2.4e-38) instead of a smaller number; callers that need an
-// exact 0 (masked keys) zero those lanes themselves.
+// clamped to [-125, 128] so n never carries past the exponent field: below,
+// the result is 2^-125 (about 2.4e-38) instead of a smaller number (callers
+// that need an exact 0, masked keys, zero those lanes themselves); above,
+// it is +inf, NaN or at least 2^127.5, never a small or negative number, so
+// a caller's overflow test sees it as MUFU's ex2 would.
 __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
   float a, b;
   f2_unpack(x2, a, b);
-  const uint64_t xc = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t xc = f2_pack(fminf(fmaxf(a, -125.f), 128.f), fminf(fmaxf(b, -125.f), 128.f));
   const uint64_t magic = f2_pack(12582912.f, 12582912.f);
   const uint64_t neg_magic = f2_pack(-12582912.f, -12582912.f);
   const uint64_t minus1 = f2_pack(-1.f, -1.f);

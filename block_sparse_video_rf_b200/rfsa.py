@@ -24,14 +24,14 @@ STATUS = {0: "RF_OK", 1: "RF_ERR_LAYOUT", 2: "RF_ERR_ARG", 3: "RF_ERR_UNSUPPORTE
 PLAN_FIELDS = ["S", "txt_len", "T", "H", "W", "Ha", "Wa", "n_promoted", "n_tail", "P", "P_pad", "nb", "ff", "k",
                "dense", "S_int", "n_tiles", "mask_words"]
 WS_FIELDS = ["q_int", "k_int", "v_int", "pooled_q", "pooled_k", "mask", "kept", "margin", "counter", "status",
-             "q8", "k8", "v8", "scales", "vmax", "total"]
+             "q8", "k8", "v8", "scales", "vmax", "redo", "total"]
 RF_BF16, RF_F16 = 0, 1
 PRECISIONS = {"native": 0, "fp8": 1}
 
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_debug_set_wait", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
+           "rf_debug_set_wait", "rf_debug_set_path", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
            "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv"]
 
 
@@ -71,6 +71,7 @@ def _load():
         "rf_read_status": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(I), P]),
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
+        "rf_debug_set_path": (I, [I, F]),
         "rf_last_error_string": (ctypes.c_char_p, []),
         "rf_plan_kv": (I, [I, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan)]),
         "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan),
@@ -284,6 +285,11 @@ def rf_debug_set_wait(wait_limit_ns: int = 0, skip_first_q: int = 0):
     _check(LIB.rf_debug_set_wait(int(wait_limit_ns), int(skip_first_q)))
 
 
+def rf_debug_set_path(path: int = 0, sum_limit: float = 0.0):
+    """Test control of the 16-bit attention path (see include/rfsa.h)."""
+    _check(LIB.rf_debug_set_path(int(path), float(sum_limit)))
+
+
 def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
     st = ctypes.c_int(0)
     _check(LIB.rf_read_status(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
@@ -329,7 +335,8 @@ def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"
         "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),
         "kept": view(lay.kept, heads * nb, torch.int32, (B, N, nb)),
         "margin": view(lay.margin, heads * nb, torch.float32, (B, N, nb)),
-    }
+    } | ({} if precision == "fp8" else {"redo": view(lay.redo, 2 + heads * plan.n_tiles, torch.int32,
+                                                         (2 + heads * plan.n_tiles,))})
 
 
 def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda", precision: str = "native", S_kv: int = 0,

@@ -105,10 +105,14 @@ typedef struct {
  * [B, N, S_int, 128]; v8: e4m3 codes of V with each 128-row block stored
  * transposed ([B, N, n_tiles, 128 channels, 128 rows]); scales: fp32
  * q [B, N, n_tiles_q], then k and v [B, N, n_tiles_kv]; vmax: fp32 [B, N],
- * the largest V block scale of each head. */
+ * the largest V block scale of each head.
+ * Only with RF_PREC_NATIVE: redo: int32 [2 + B * N * n_tiles_q], the query
+ * tiles the 16-bit attention hands to its second pass ([0] a work counter,
+ * [1] how many, [2 ...] their ids). */
 typedef struct {
   size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status;
   size_t q8, k8, v8, scales, vmax;
+  size_t redo;
   size_t total;
 } rf_ws_layout_t;
 
@@ -231,6 +235,16 @@ rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D
  * output is not valid.  Used by the tests to exercise the timeout path
  * without any fault; call with (0, 0) to restore normal operation. */
 rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q);
+
+/* Test control of the 16-bit attention path, process-wide, read at each
+ * launch.  path 0 (default): the three-chain kernel runs every query tile
+ * and hands the tiles whose P left the type's headroom to the two-tile
+ * kernel; path 1: the two-tile kernel runs every query tile.  sum_limit > 0
+ * replaces the headroom test (a tile sum of P above it hands the tile on;
+ * 0 = the type's own: 2^64 for bf16, 65504 for fp16), so a test can send a
+ * chosen share of the tiles through the second pass.  Returns RF_ERR_ARG on
+ * path outside {0, 1} or sum_limit < 0. */
+rf_status_t rf_debug_set_path(int path, float sum_limit);
 
 /* Size of the library-owned static scratch array of rf_block_mask_noalloc,
  * per device (32 MiB): enough for B * N * nb <= 32768 block rows of pooled Q and K

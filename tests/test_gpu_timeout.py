@@ -12,12 +12,13 @@ from parity_util import assert_close, to_bnsd_np
 
 
 
-
 @pytest.mark.gpu
-def test_wait_timeout_is_reported_and_context_recovers():
+@pytest.mark.parametrize("path", [0, 1], ids=["chain_kernel", "two_tile_kernel"])
+def test_wait_timeout_is_reported_and_context_recovers(path):
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     from block_sparse_video_rf_b200 import rfsa, synth
+    rfsa.rf_debug_set_path(path, 0.0)
     w = synth.workload("tiny")
     q, k, v = (t.cuda() for t in synth.make_inputs(w, device="cpu"))
     sp = np.float32(w.sparsity)
@@ -33,8 +34,11 @@ def test_wait_timeout_is_reported_and_context_recovers():
         rfsa.rf_debug_set_wait(0, 0)
     assert status == 6                                  # RF_ERR_TIMEOUT
     # the context is still usable and the status word was cleared
-    rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws)
-    assert rfsa.rf_read_status(ws, w.B, w.N, 128, plan) == 0
+    try:
+        rfsa.rf_attend(out, w.layout, w.txt_len, w.latent, sp, ws)
+        assert rfsa.rf_read_status(ws, w.B, w.N, 128, plan) == 0
+    finally:
+        rfsa.rf_debug_set_path(0, 0.0)
     ref, _, _, _ = oracle.rf_sparse_attention(q.float().cpu().numpy(), k.float().cpu().numpy(),
                                               v.float().cpu().numpy(), w.layout, w.txt_len, w.latent, float(sp))
     assert_close(out.float().cpu().numpy(), ref, "after timeout")
@@ -49,3 +53,8 @@ def test_debug_control_rejects_bad_values():
     with pytest.raises(rfsa.RfError):
         rfsa.rf_debug_set_wait(0, 2)
     rfsa.rf_debug_set_wait(0, 0)
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_debug_set_path(2, 0.0)
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_debug_set_path(0, -1.0)
+    rfsa.rf_debug_set_path(0, 0.0)
