@@ -233,11 +233,12 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     for (int j = 0; j < itm.ntiles; ++j, ++gq) {
       const int c = j % kSets;
       const uint32_t ks = gq % kRing;
-      if (uses[c] >= 1 && !waitw(&sm.abort, p, &sm.pv_done[c], ph(uses[c] - 1))) {
+      // K lands tiles ahead; the buffer's previous P V is the wait that counts
+      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / kRing))) {
         ok = false;
         break;
       }
-      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / kRing))) {
+      if (uses[c] >= 1 && !waitw(&sm.abort, p, &sm.pv_done[c], ph(uses[c] - 1))) {
         ok = false;
         break;
       }
@@ -277,7 +278,7 @@ __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     for (int j = 0; j < itm.ntiles; ++j, ++gp) {
       const int c = j % kSets;
       const uint32_t vs = gp % kRing;
-      if (!waitw(&sm.abort, p, &sm.p_full[c], ph(uses[c]))) {
+      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / kRing))) {
         ok = false;
         break;
       }
@@ -286,7 +287,7 @@ __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
         ok = false;
         break;
       }
-      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / kRing))) {
+      if (!waitw(&sm.abort, p, &sm.p_full[c], ph(uses[c]))) {
         ok = false;
         break;
       }
