@@ -31,8 +31,8 @@
 //         previous tile is done (P lives in the first 64 columns of S);
 //         owns the tensor memory.
 // Shared memory: Q (32 KB), rings of three K and three V tiles (96 KB each),
-// 128-byte swizzled boxes of 128 rows x 128 bytes; K and V of the CTA's
-// tile g load once the S, respectively the P V, of tile g - 3 is done.
+// 128-byte swizzled boxes of 128 rows x 128 bytes; K of the CTA's tile g
+// loads once the S of tile g - 3 is done, V once the P V of tile g - 3 is.
 // Tensor memory (512 columns): S_c at [128 c, 128 c + 128) for c = 0, 1, 2,
 // O at [384, 512).
 #include "rf_attn_common.cuh"
@@ -43,7 +43,11 @@ namespace {
 
 constexpr int kCThreads = 512;
 constexpr int kSets = 3;                      // S buffers = softmax warp sets
-constexpr int kRing = 3;                      // K tiles and V tiles in flight (each)
+// Shared memory holds 7 tiles: one Q (a second Q buffer, taken from the V
+// ring, measured slower: the bubble at a unit change costs less than a
+// shallower V ring), three K and three V.
+constexpr int kQBufs = 1;
+constexpr int kKRing = 3, kVRing = 3;         // K tiles and V tiles in flight
 constexpr int kItemQ = 8;                     // depth of the unit queue
 constexpr uint32_t kCTmemCols = 512;
 constexpr int kWarpKProd = 12, kWarpVProd = 13, kWarpPV = 14, kWarpQK = 15;
@@ -52,11 +56,11 @@ constexpr int kMaxSmem = 232448;              // 227 KB: the most dynamic shared
 
 template <class C>
 struct __align__(1024) ChainSmem {
-  uint8_t q[C::kTileBytes];
-  uint8_t k[kRing][C::kTileBytes];
-  uint8_t v[kRing][C::kTileBytes];
-  uint64_t q_full, q_empty;
-  uint64_t k_full[kRing], k_empty[kRing], v_full[kRing], v_empty[kRing];
+  uint8_t q[kQBufs][C::kTileBytes];
+  uint8_t k[kKRing][C::kTileBytes];
+  uint8_t v[kVRing][C::kTileBytes];
+  uint64_t q_full[kQBufs], q_empty[kQBufs];
+  uint64_t k_full[kKRing], k_empty[kKRing], v_full[kVRing], v_empty[kVRing];
   uint64_t s_full[kSets];     // S of the set's next tile is in TMEM (MMA commit)
   uint64_t p_full[kSets];     // the set wrote P of its tile (one arrival per warp)
   uint64_t pv_done[kSets];    // P V of the set's tile done (MMA commit)
@@ -119,7 +123,7 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
   uint32_t u = 0, nk = 0;   // units published, K tiles issued
-  bool q_issued = false;    // a Q load of this CTA is in flight or landed
+  uint32_t nq[kQBufs] = {}; // Q loads issued into each buffer
   bool ok = true;
   while (ok) {
     const int w = atomicAdd(p.counter, 1);
@@ -133,19 +137,20 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
     sm.items[qi] = itm;
     mbar_arrive(&sm.item_full[qi]);
     if (itm.bn < 0) break;
-    if (u >= 1 && !wait1(&sm.abort, p, &sm.q_empty, ph(u - 1))) {
+    const uint32_t qb = u % kQBufs;
+    if (u >= (uint32_t)kQBufs && !wait1(&sm.abort, p, &sm.q_empty[qb], ph(u / kQBufs - 1))) {
       ok = false;
       break;
     }
     if (!(p.skip_first_q && u == 0)) {
-      load_tile<C>(sm.q, tq, &sm.q_full, itm.bn * p.g.S_int + itm.qt * RF_BLOCK, pol_q);
-      q_issued = true;
+      load_tile<C>(sm.q[qb], tq, &sm.q_full[qb], itm.bn * p.g.S_int + itm.qt * RF_BLOCK, pol_q);
+      ++nq[qb];
     }
     ++u;
     KvIter kit;
     kit.init(itm.bn * p.gk.S_int, p, mrow);
     for (int row = kit.next(); row >= 0; row = kit.next()) {
-      const uint32_t s = nk % kRing, n = nk / kRing;
+      const uint32_t s = nk % kKRing, n = nk / kKRing;
       if (n >= 1 && !wait1(&sm.abort, p, &sm.k_empty[s], ph(n - 1))) {
         ok = false;
         break;
@@ -158,9 +163,10 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
     // Let the copies already issued land before the CTA may exit (bounded by
     // time, not cut short by the abort flag).
     const uint64_t lim = p.wait_limit_ns / 4;
-    if (q_issued) rf_wait_time(&sm.q_full, ph(u - 1), lim);
-    for (uint32_t st = 0; st < (uint32_t)kRing; ++st) {
-      const uint32_t n = (nk > st) ? (nk - st + kRing - 1) / kRing : 0;
+    for (uint32_t b = 0; b < (uint32_t)kQBufs; ++b)
+      if (nq[b]) rf_wait_time(&sm.q_full[b], ph(nq[b] - 1), lim);
+    for (uint32_t st = 0; st < (uint32_t)kKRing; ++st) {
+      const uint32_t n = (nk > st) ? (nk - st + kKRing - 1) / kKRing : 0;
       if (n) rf_wait_time(&sm.k_full[st], ph(n - 1), lim);
     }
   }
@@ -184,7 +190,7 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
     KvIter kit;
     kit.init(itm.bn * p.gk.S_int, p, mask_row(p, itm));
     for (int row = kit.next(); row >= 0; row = kit.next()) {
-      const uint32_t s = nv % kRing, n = nv / kRing;
+      const uint32_t s = nv % kVRing, n = nv / kVRing;
       if (n >= 1 && !wait1(&sm.abort, p, &sm.v_empty[s], ph(n - 1))) {
         ok = false;
         break;
@@ -195,8 +201,8 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
   }
   if (!ok) {
     const uint64_t lim = p.wait_limit_ns / 4;
-    for (uint32_t st = 0; st < (uint32_t)kRing; ++st) {
-      const uint32_t n = (nv > st) ? (nv - st + kRing - 1) / kRing : 0;
+    for (uint32_t st = 0; st < (uint32_t)kVRing; ++st) {
+      const uint32_t n = (nv > st) ? (nv - st + kVRing - 1) / kVRing : 0;
       if (n) rf_wait_time(&sm.v_full[st], ph(n - 1), lim);
     }
   }
@@ -212,7 +218,7 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
 template <class C>
 __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
-  const uint32_t q_lo = (uint32_t)make_sdesc_sw128(smem_u32(sm.q), 16, 1024);
+  const uint32_t q_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
   const uint32_t k_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
   uint32_t uses[kSets] = {0, 0, 0};   // S tiles issued into each buffer
   uint32_t gq = 0;                    // the CTA's tiles issued (K ring position)
@@ -226,15 +232,17 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     const Item itm = sm.items[qi];
     arrive_w(&sm.item_empty[qi]);
     if (itm.bn < 0) break;
-    if (!waitw(&sm.abort, p, &sm.q_full, ph(u))) {
+    const uint32_t qb = u % kQBufs;
+    const uint32_t q_lo = q_lo0 + qb * (C::kTileBytes >> 4);
+    if (!waitw(&sm.abort, p, &sm.q_full[qb], ph(u / kQBufs))) {
       ok = false;
       break;
     }
     for (int j = 0; j < itm.ntiles; ++j, ++gq) {
       const int c = j % kSets;
-      const uint32_t ks = gq % kRing;
+      const uint32_t ks = gq % kKRing;
       // K lands tiles ahead; the buffer's previous P V is the wait that counts
-      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / kRing))) {
+      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / kKRing))) {
         ok = false;
         break;
       }
@@ -246,7 +254,7 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
       issue_qk<C>(tmem + 128 * c, q_lo, k_lo0 + ks * (C::kTileBytes >> 4), hi);
       mma_commit_elect(&sm.s_full[c]);
       mma_commit_elect(&sm.k_empty[ks]);
-      if (j == itm.ntiles - 1) mma_commit_elect(&sm.q_empty);
+      if (j == itm.ntiles - 1) mma_commit_elect(&sm.q_empty[qb]);
       issued = true;
       ++uses[c];
     }
@@ -277,8 +285,8 @@ __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     if (itm.bn < 0) break;
     for (int j = 0; j < itm.ntiles; ++j, ++gp) {
       const int c = j % kSets;
-      const uint32_t vs = gp % kRing;
-      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / kRing))) {
+      const uint32_t vs = gp % kVRing;
+      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / kVRing))) {
         ok = false;
         break;
       }
@@ -489,11 +497,15 @@ __global__ void __launch_bounds__(kCThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_empty, 1);
-    for (int i = 0; i < kRing; ++i) {
+    for (int i = 0; i < kQBufs; ++i) {
+      mbar_init(&sm.q_full[i], 1);
+      mbar_init(&sm.q_empty[i], 1);
+    }
+    for (int i = 0; i < kKRing; ++i) {
       mbar_init(&sm.k_full[i], 1);
       mbar_init(&sm.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVRing; ++i) {
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
