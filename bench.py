@@ -70,7 +70,7 @@ def _k3_traffic(heads: int):
     digest = h.hexdigest()[:16]
     for line in open(path):
         parts = line.split()
-        if len(parts) >= 3 and not line.startswith("#") and parts[0] == "attn_kernel" and parts[1] == digest:
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == "k3" and parts[1] == digest:
             return int(parts[2]) * heads / 56.0
     return None
 
