@@ -356,9 +356,9 @@ def main():
             "roofline": {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": k3_tflops / peak,
                          "traffic": _k3_traffic(w.N) if default_mode else None, "peak_source": peak_note},
-            # K1, K2 and K3 (fp8: and the quantisation pass; 16-bit: K3 is the chain kernel and its
-            # second pass, which returns at once when no unit was handed to it)
-            "gpu_launches": 4 * args.steps,
+            # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
+            # handed to it); fp8 adds the quantisation pass
+            "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -249,7 +249,7 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
   L.v8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
   L.scales = take(fp8 ? heads * (g->n_tiles + 2 * (size_t)gk->n_tiles) * 4 : 0);
   L.vmax = take(fp8 ? heads * 4 : 0);
-  L.redo = take(fp8 ? 0 : (2 + heads * g->n_tiles) * 4);
+  L.redo = take((2 + heads * g->n_tiles) * 4);
   L.total = off;
   *lay = L;
   return ok();
@@ -330,7 +330,7 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
     e = rf::launch_attention_fp8(at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
                                  at<float>(ws, L.scales), at<float>(ws, L.vmax), at<uint32_t>(ws, L.mask), dtype,
                                  layout, B, S, N, g, gk, resolve_scale(scale, D), out, at<int>(ws, L.counter),
-                                 at<int>(ws, L.status), debug_settings(), s);
+                                 at<int>(ws, L.status), at<int>(ws, L.redo), debug_settings(), s);
   else
     e = rf::launch_attention(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int),
                              at<uint32_t>(ws, L.mask), dtype, layout, B, S, N, g, gk, resolve_scale(scale, D), out,

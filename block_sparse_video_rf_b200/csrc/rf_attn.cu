@@ -62,14 +62,6 @@ constexpr int kSlotWarps = 4;                            // softmax warps per sl
 constexpr uint32_t kRegsSoftmax = 216, kRegsControl = 64;
 constexpr uint32_t kTmemCols = 512;
 
-// Per-tile factors of the fp8 path, written by the slot's issuer before its
-// arrival on s_full: c = scale * log2(e) * sq * sk (multiplies S), lr =
-// log2(sv / vmax) (added to P's exponent), ir = vmax / sv (l adds P's sum
-// times ir).
-struct TileScale {
-  float c, lr, ir, pad;
-};
-
 // One slot: buffers and barriers of one unit in flight.
 template <class C>
 struct __align__(1024) Slot {
@@ -287,16 +279,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
     if (last_of_unit) mma_commit_elect(&sl.q_empty);
     issued = true;
     if ((threadIdx.x & 31) == 0) {
-      if (C::kFp8) {
-        const float vmax = unit_vmax;
-        TileScale f;
-        f.c = p.scale_log2 * q_scale * sk;
-        const bool use_r = sv > 0.f && vmax > 0.f;   // an all-zero V block adds nothing whatever P is
-        f.lr = use_r ? __log2f(sv / vmax) : 0.f;
-        f.ir = use_r ? vmax / sv : 1.f;
-        f.pad = 0.f;
-        sl.ts[tt & 1] = f;
-      }
+      if (C::kFp8) sl.ts[tt & 1] = tile_scale(p, q_scale, sk, sv, unit_vmax);
       mbar_arrive(&sl.s_full);
     }
     __syncwarp();
@@ -307,7 +290,7 @@ __device__ void slot_loop(Smem<C>& sm, Slot<C>& sl, const AttnParams& p, uint32_
     // Every warp of the slot reaches every rendezvous: a warp whose wait
     // failed carries ok = false to the next one, where all four leave.
     const uint32_t it = c & 1;
-    Item itm{-1, 0, 0, 0};
+    Item itm{-1, 0, 0, -1};
     if (ok) ok = waitw(&sm.abort, p, &sl.item_full[it], ph(c >> 1));
     if (ok) {
       itm = sl.items[it];
@@ -494,19 +477,21 @@ cudaError_t launch_attention_slots(const void* q_int, const void* k_int, const v
              : launch_cfg<Cfg<false, false>>(tq, tk, tv, p, stream);
 }
 
-cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
-                                 const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
-                                 const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out, int* counter,
-                                 int* status, const AttnDebug& dbg, cudaStream_t stream) {
+cudaError_t launch_attention_fp8_slots(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
+                                       const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S,
+                                       int N, const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out,
+                                       int* counter, int* status, int* redo, int list_mode, const AttnDebug& dbg,
+                                       cudaStream_t stream) {
   const uint64_t rows_q = (uint64_t)B * N * g.S_int, rows_k = (uint64_t)B * N * gk.S_int;
   CUtensorMap tq, tk, tv;
   if (!make_tile_map(&tq, q8, rows_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
       !make_tile_map(&tk, k8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
       !make_tile_map(&tv, v8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
     return cudaErrorInvalidValue;
-  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, nullptr, dbg);
+  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, redo, dbg);
   p.scales = scales;
   p.vmax = vmax;
+  p.list_mode = list_mode;
   return dtype == RF_F16 ? launch_cfg<Cfg<true, true>>(tq, tk, tv, p, stream)
                          : launch_cfg<Cfg<false, true>>(tq, tk, tv, p, stream);
 }

@@ -35,6 +35,8 @@
 // loads once the S of tile g - 3 is done, V once the P V of tile g - 3 is.
 // Tensor memory (512 columns): S_c at [128 c, 128 c + 128) for c = 0, 1, 2,
 // O at [384, 512).
+#include <cstring>
+
 #include "rf_attn_common.cuh"
 
 namespace rf {
@@ -43,25 +45,31 @@ namespace {
 
 constexpr int kCThreads = 512;
 constexpr int kSets = 3;                      // S buffers = softmax warp sets
-// Shared memory holds 7 tiles: one Q (a second Q buffer, taken from the V
-// ring, measured slower: the bubble at a unit change costs less than a
-// shallower V ring), three K and three V.
-constexpr int kQBufs = 1;
-constexpr int kKRing = 3, kVRing = 3;         // K tiles and V tiles in flight
+// Q buffers and K / V tiles in flight.  16-bit (32 KB tiles): shared memory
+// holds 7 tiles, one Q, three K and three V (a second Q buffer, taken from
+// the V ring, measured slower: the bubble at a unit change costs less than a
+// shallower V ring).  fp8 (16 KB tiles): two Q, four K and four V.
+template <class C>
+struct ChainShape {
+  static constexpr int kQBufs = C::kFp8 ? 2 : 1;
+  static constexpr int kKRing = C::kFp8 ? 4 : 3;
+  static constexpr int kVRing = C::kFp8 ? 4 : 3;
+};
 constexpr int kItemQ = 8;                     // depth of the unit queue
 constexpr uint32_t kCTmemCols = 512;
 constexpr int kWarpKProd = 12, kWarpVProd = 13, kWarpPV = 14, kWarpQK = 15;
 constexpr int kItemReaders = 3 + 4 * kSets;   // V producer, the two MMA warps, softmax warps
 constexpr int kMaxSmem = 232448;              // 227 KB: the most dynamic shared memory a CTA may have
 
-template <class C>
+template <class C, class CS = ChainShape<C>>
 struct __align__(1024) ChainSmem {
-  uint8_t q[kQBufs][C::kTileBytes];
-  uint8_t k[kKRing][C::kTileBytes];
-  uint8_t v[kVRing][C::kTileBytes];
-  uint64_t q_full[kQBufs], q_empty[kQBufs];
-  uint64_t k_full[kKRing], k_empty[kKRing], v_full[kVRing], v_empty[kVRing];
-  uint64_t s_full[kSets];     // S of the set's next tile is in TMEM (MMA commit)
+  uint8_t q[CS::kQBufs][C::kTileBytes];
+  uint8_t k[CS::kKRing][C::kTileBytes];
+  uint8_t v[CS::kVRing][C::kTileBytes];
+  uint64_t q_full[CS::kQBufs], q_empty[CS::kQBufs];
+  uint64_t k_full[CS::kKRing], k_empty[CS::kKRing], v_full[CS::kVRing], v_empty[CS::kVRing];
+  uint64_t s_full[kSets];     // S of the set's next tile is in TMEM (MMA commit; fp8: and the S warp's
+                              // arrival once the tile's factors are in ts)
   uint64_t p_full[kSets];     // the set wrote P of its tile (one arrival per warp)
   uint64_t pv_done[kSets];    // P V of the set's tile done (MMA commit)
   uint64_t o_full;            // the last P V of a unit done (MMA commit)
@@ -73,17 +81,21 @@ struct __align__(1024) ChainSmem {
   Item items[kItemQ];
   float m_sh[RF_BLOCK];
   float l_sh[kSets][RF_BLOCK];
+  float kv_scale[CS::kKRing][2];   // fp8: {sk, sv} of the tile in each K slot (K producer, with k_full)
+  TileScale ts[kSets];             // fp8: factors of each buffer's tile (S warp, with s_full)
   uint32_t tmem_base;
   int abort;
 };
 static_assert(sizeof(ChainSmem<Cfg<false, false>>) <= kMaxSmem, "shared memory of the chain kernel");
+static_assert(sizeof(ChainSmem<Cfg<false, true>>) <= kMaxSmem, "shared memory of the chain kernel");
 
 // Sum of P above which a tile's unit goes to the second pass: P must stay
-// finite in its 16-bit type (bf16 to 2^127: the limit 2^64 keeps O and l far
-// from fp32 overflow; fp16 to 65504, and every P is at most the sum).
+// finite in its type (bf16 to 2^127: the limit 2^64 keeps O and l far from
+// fp32 overflow; fp16 to 65504; e4m3 to 448 before it saturates), and every
+// P is at most the sum.
 template <class C>
 __device__ __forceinline__ float sum_limit(const AttnParams& p) {
-  return p.sum_limit > 0.f ? p.sum_limit : (C::kF16 ? 65504.f : 18446744073709551616.f);
+  return p.sum_limit > 0.f ? p.sum_limit : (C::kFp8 ? 448.f : C::kF16 ? 65504.f : 18446744073709551616.f);
 }
 
 __device__ __forceinline__ const uint32_t* mask_row(const AttnParams& p, const Item& itm) {
@@ -120,10 +132,12 @@ __device__ __forceinline__ bool set_or(int set, bool v) {
 // its K tiles into the ring.
 template <class C>
 __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk) {
+  using CS = ChainShape<C>;
+  const int BN = p.B * p.N;
   const uint64_t pol_q = l2_policy_evict_first();
   const uint64_t pol_kv = l2_policy_evict_last();
   uint32_t u = 0, nk = 0;   // units published, K tiles issued
-  uint32_t nq[kQBufs] = {}; // Q loads issued into each buffer
+  uint32_t nq[CS::kQBufs] = {};   // Q loads issued into each buffer
   bool ok = true;
   while (ok) {
     const int w = atomicAdd(p.counter, 1);
@@ -133,12 +147,14 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
       break;
     }
     const uint32_t* mrow;
-    const Item itm = make_item(p, unit_of(p, w), mrow);
+    Item itm = make_item(p, unit_of(p, w), mrow);
+    const int own = own_tile(p, itm, mrow);
+    itm.partial = partial_place(p, own);
     sm.items[qi] = itm;
     mbar_arrive(&sm.item_full[qi]);
     if (itm.bn < 0) break;
-    const uint32_t qb = u % kQBufs;
-    if (u >= (uint32_t)kQBufs && !wait1(&sm.abort, p, &sm.q_empty[qb], ph(u / kQBufs - 1))) {
+    const uint32_t qb = u % CS::kQBufs;
+    if (u >= (uint32_t)CS::kQBufs && !wait1(&sm.abort, p, &sm.q_empty[qb], ph(u / CS::kQBufs - 1))) {
       ok = false;
       break;
     }
@@ -147,13 +163,21 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
       ++nq[qb];
     }
     ++u;
+    const int base = itm.bn * p.gk.S_int;   // the unit's KV rows
+    const float* sc_k = C::kFp8 ? p.scales + (size_t)BN * p.g.n_tiles + (size_t)itm.bn * p.gk.n_tiles : nullptr;
+    const float* sc_v = C::kFp8 ? sc_k + (size_t)BN * p.gk.n_tiles : nullptr;
     KvIter kit;
-    kit.init(itm.bn * p.gk.S_int, p, mrow);
+    kit.init(base, p, mrow, own);
     for (int row = kit.next(); row >= 0; row = kit.next()) {
-      const uint32_t s = nk % kKRing, n = nk / kKRing;
+      const uint32_t s = nk % CS::kKRing, n = nk / CS::kKRing;
       if (n >= 1 && !wait1(&sm.abort, p, &sm.k_empty[s], ph(n - 1))) {
         ok = false;
         break;
+      }
+      if (C::kFp8) {   // published by the arrival in load_tile, read under k_full
+        const int tile = (row - base) / RF_BLOCK;
+        sm.kv_scale[s][0] = sc_k[tile];
+        sm.kv_scale[s][1] = sc_v[tile];
       }
       load_tile<C>(sm.k[s], tk, &sm.k_full[s], row, pol_kv);
       ++nk;
@@ -163,10 +187,10 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
     // Let the copies already issued land before the CTA may exit (bounded by
     // time, not cut short by the abort flag).
     const uint64_t lim = p.wait_limit_ns / 4;
-    for (uint32_t b = 0; b < (uint32_t)kQBufs; ++b)
+    for (uint32_t b = 0; b < (uint32_t)CS::kQBufs; ++b)
       if (nq[b]) rf_wait_time(&sm.q_full[b], ph(nq[b] - 1), lim);
-    for (uint32_t st = 0; st < (uint32_t)kKRing; ++st) {
-      const uint32_t n = (nk > st) ? (nk - st + kKRing - 1) / kKRing : 0;
+    for (uint32_t st = 0; st < (uint32_t)CS::kKRing; ++st) {
+      const uint32_t n = (nk > st) ? (nk - st + CS::kKRing - 1) / CS::kKRing : 0;
       if (n) rf_wait_time(&sm.k_full[st], ph(n - 1), lim);
     }
   }
@@ -175,6 +199,7 @@ __device__ void kprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
 // V: follows the unit queue and loads the V tiles into their ring.
 template <class C>
 __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensorMap* tv) {
+  using CS = ChainShape<C>;
   const uint64_t pol_kv = l2_policy_evict_last();
   uint32_t nv = 0;
   bool ok = true;
@@ -188,9 +213,10 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
     mbar_arrive(&sm.item_empty[qi]);
     if (itm.bn < 0) break;
     KvIter kit;
-    kit.init(itm.bn * p.gk.S_int, p, mask_row(p, itm));
+    const uint32_t* mrow = mask_row(p, itm);
+    kit.init(itm.bn * p.gk.S_int, p, mrow, own_tile(p, itm, mrow));
     for (int row = kit.next(); row >= 0; row = kit.next()) {
-      const uint32_t s = nv % kVRing, n = nv / kVRing;
+      const uint32_t s = nv % CS::kVRing, n = nv / CS::kVRing;
       if (n >= 1 && !wait1(&sm.abort, p, &sm.v_empty[s], ph(n - 1))) {
         ok = false;
         break;
@@ -201,8 +227,8 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
   }
   if (!ok) {
     const uint64_t lim = p.wait_limit_ns / 4;
-    for (uint32_t st = 0; st < (uint32_t)kVRing; ++st) {
-      const uint32_t n = (nv > st) ? (nv - st + kVRing - 1) / kVRing : 0;
+    for (uint32_t st = 0; st < (uint32_t)CS::kVRing; ++st) {
+      const uint32_t n = (nv > st) ? (nv - st + CS::kVRing - 1) / CS::kVRing : 0;
       if (n) rf_wait_time(&sm.v_full[st], ph(n - 1), lim);
     }
   }
@@ -217,6 +243,7 @@ __device__ void vprod_loop(ChainSmem<C>& sm, const AttnParams& p, const CUtensor
 // MMAs.  On an abort each waits (bounded) for its MMAs before leaving.
 template <class C>
 __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
+  using CS = ChainShape<C>;
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
   const uint32_t q_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
   const uint32_t k_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.k[0]), 16, 1024);
@@ -232,20 +259,25 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     const Item itm = sm.items[qi];
     arrive_w(&sm.item_empty[qi]);
     if (itm.bn < 0) break;
-    const uint32_t qb = u % kQBufs;
+    const uint32_t qb = u % CS::kQBufs;
     const uint32_t q_lo = q_lo0 + qb * (C::kTileBytes >> 4);
-    if (!waitw(&sm.abort, p, &sm.q_full[qb], ph(u / kQBufs))) {
+    if (!waitw(&sm.abort, p, &sm.q_full[qb], ph(u / CS::kQBufs))) {
       ok = false;
       break;
     }
+    // fp8: the unit's Q block scale and the head's largest V block scale
+    const float sq = C::kFp8 ? p.scales[(size_t)itm.bn * p.g.n_tiles + itm.qt] : 0.f;
+    const float vmax = C::kFp8 ? p.vmax[itm.bn] : 0.f;
     for (int j = 0; j < itm.ntiles; ++j, ++gq) {
       const int c = j % kSets;
-      const uint32_t ks = gq % kKRing;
+      const uint32_t ks = gq % CS::kKRing;
       // K lands tiles ahead; the buffer's previous P V is the wait that counts
-      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / kKRing))) {
+      if (!waitw(&sm.abort, p, &sm.k_full[ks], ph(gq / CS::kKRing))) {
         ok = false;
         break;
       }
+      // read before the MMAs: once they finish, the producer may refill the slot
+      const float sk = C::kFp8 ? sm.kv_scale[ks][0] : 0.f, sv = C::kFp8 ? sm.kv_scale[ks][1] : 0.f;
       if (uses[c] >= 1 && !waitw(&sm.abort, p, &sm.pv_done[c], ph(uses[c] - 1))) {
         ok = false;
         break;
@@ -257,6 +289,15 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
       if (j == itm.ntiles - 1) mma_commit_elect(&sm.q_empty[qb]);
       issued = true;
       ++uses[c];
+      if (C::kFp8) {
+        // the set of buffer c read the previous tile's factors before its P,
+        // which came before that tile's P V
+        if ((threadIdx.x & 31) == 0) {
+          sm.ts[c] = tile_scale(p, sq, sk, sv, vmax);
+          mbar_arrive(&sm.s_full[c]);
+        }
+        __syncwarp();
+      }
     }
   }
   if (!ok && issued) {
@@ -268,8 +309,9 @@ __device__ void qk_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
 
 template <class C>
 __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
+  using CS = ChainShape<C>;
   const uint32_t hi = (uint32_t)(make_sdesc_sw128(0, 16, 1024) >> 32);
-  const uint32_t v_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.v[0]), kBoxBytes, 1024);
+  const uint32_t v_lo0 = (uint32_t)make_sdesc_sw128(smem_u32(sm.v[0]), C::kFp8 ? 16 : kBoxBytes, 1024);
   const uint32_t o_tmem = tmem + 384;
   uint32_t uses[kSets] = {0, 0, 0};   // P V tiles issued from each buffer
   uint32_t gp = 0;                    // the CTA's tiles issued (V ring position)
@@ -285,8 +327,8 @@ __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
     if (itm.bn < 0) break;
     for (int j = 0; j < itm.ntiles; ++j, ++gp) {
       const int c = j % kSets;
-      const uint32_t vs = gp % kVRing;
-      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / kVRing))) {
+      const uint32_t vs = gp % CS::kVRing;
+      if (!waitw(&sm.abort, p, &sm.v_full[vs], ph(gp / CS::kVRing))) {
         ok = false;
         break;
       }
@@ -328,8 +370,10 @@ __device__ __forceinline__ float tile_max(uint32_t tS, int p_valid) {
   return mx;
 }
 
-// P = 2^(s c + off) of the row's 128 scores, in two halves of 64 (P of half
-// h goes to columns [32 h, 32 h + 32), already read); returns the sum of P.
+// P = 2^(s c + off) of the row's 128 scores, in two halves of 64; P of half
+// h goes to columns [32 h, 32 h + 32) (16-bit, two per column) or
+// [16 h, 16 h + 16) (e4m3, four per column), which are already read.
+// Returns the sum of P.
 template <class C>
 __device__ __forceinline__ float tile_softmax(uint32_t tS, int p_valid, float c, float off) {
   float tsum = 0.f;
@@ -337,9 +381,15 @@ __device__ __forceinline__ float tile_softmax(uint32_t tS, int p_valid, float c,
   for (int h = 0; h < 2; ++h) {
     uint32_t s[2][32];
     load_scores<2>(tS + 64 * h, p_valid - 64 * h, s);
-    uint32_t pk[32];
-    tsum += exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
-    tmem_st32(tS + 32 * h, pk);
+    if constexpr (C::kFp8) {
+      uint32_t pk[16];
+      tsum += exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
+      tmem_st16(tS + 16 * h, pk);
+    } else {
+      uint32_t pk[32];
+      tsum += exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
+      tmem_st32(tS + 32 * h, pk);
+    }
   }
   tmem_wait_st();
   return tsum;
@@ -357,13 +407,12 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
   const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
   const uint32_t lanes = (uint32_t)(quad * 32) << 16;
   const uint32_t tS = tmem + 128 * set + lanes, tO = tmem + 384 + lanes;
-  const float c = p.scale_log2;
   const float limit = sum_limit<C>(p);
   uint32_t mine = 0;   // tiles this set has taken (completions of s_full / p_full)
   bool ok = true;
   for (uint32_t u = 0;; ++u) {
     const uint32_t qi = u % kItemQ;
-    Item itm{-1, 0, 0, 0};
+    Item itm{-1, 0, 0, -1};
     if (ok) ok = waitw(&sm.abort, p, &sm.item_full[qi], ph(u / kItemQ));
     if (ok) {
       itm = sm.items[qi];
@@ -376,7 +425,18 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
     const int last = (n - 1) % kSets;             // set of the unit's last tile
     float m_use = 0.f, l = 0.f;
     bool row_bad = false;
-    auto p_valid_of = [&](int j) { return (p.p_rem_k != 0 && j == p.n_ptiles_k - 1) ? p.p_rem_k : RF_BLOCK; };
+    // The tile's factors: 16-bit, S c with c = scale log2(e); fp8, the S
+    // warp's TileScale of the buffer (published with s_full).
+    auto factors = [&]() -> TileScale {
+      if (C::kFp8) return sm.ts[set];
+      TileScale f;
+      f.c = p.scale_log2;
+      f.lr = 0.f;
+      f.ir = 1.f;
+      f.pad = 0.f;
+      return f;
+    };
+    auto p_valid_of = [&](int j) { return j == itm.partial ? p.p_rem_k : RF_BLOCK; };
     // S of the set's next tile: the set's first warp waits on the barrier,
     // the other three at the set's named barrier, where they take no issue
     // slots; every warp reaches it, carrying the outcome.
@@ -389,9 +449,10 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
       wait_s();
       if (ok) {
         tc_fence_after();
-        const float ts = tile_softmax<C>(tS, p_valid_of(j), c, -m_use);
+        const TileScale f = factors();
+        const float ts = tile_softmax<C>(tS, p_valid_of(j), f.c, f.lr - m_use);
         row_bad |= !(ts <= limit);
-        l += ts;
+        l += ts * f.ir;
         tc_fence_before();
         arrive_w(&sm.p_full[set]);
       }
@@ -400,9 +461,11 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
     if (set == owner) {
       // the unit's maximum: the row maximum of its first tile
       wait_s();
+      TileScale f0{};
       if (ok) {
         tc_fence_after();
-        m_use = tile_max(tS, p_valid_of(0)) * c;
+        f0 = factors();
+        m_use = tile_max(tS, p_valid_of(0)) * f0.c;
       }
       if (ok && u >= 1) ok = waitw(&sm.abort, p, &sm.m_empty, ph(u - 1));
       if (ok) {
@@ -411,9 +474,9 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
         arrive_w(&sm.m_full);
         arrive_w(&sm.m_empty);
         // the first tile's P (its S is still in place)
-        const float ts = tile_softmax<C>(tS, p_valid_of(0), c, -m_use);
+        const float ts = tile_softmax<C>(tS, p_valid_of(0), f0.c, f0.lr - m_use);
         row_bad |= !(ts <= limit);
-        l += ts;
+        l += ts * f0.ir;
         tc_fence_before();
         arrive_w(&sm.p_full[set]);
       }
@@ -437,7 +500,7 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
     if (!ok) break;
     if (set != last) continue;
 
-    // output of the unit: O / (l_0 + l_1 + l_2)
+    // output of the unit: O / (l_0 + l_1 + l_2) (fp8: times the head's largest V scale)
     float lt = 0.f;
     ok = waitw(&sm.abort, p, &sm.l_full, ph(u));
     if (ok) {
@@ -450,7 +513,7 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
     ok = waitw(&sm.abort, p, &sm.o_full, ph(u));
     if (ok) {
       tc_fence_after();
-      const float rl = 1.f / lt;
+      const float rl = (C::kFp8 ? p.vmax[itm.bn] : 1.f) / lt;
       uint16_t* dst = unit_bad ? nullptr : out_row<C>(p, itm.bn, itm.qt, row);
 #pragma unroll 1
       for (int q4 = 0; q4 < 4; ++q4) {
@@ -497,20 +560,21 @@ __global__ void __launch_bounds__(kCThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kQBufs; ++i) {
+    using CS = ChainShape<C>;
+    for (int i = 0; i < CS::kQBufs; ++i) {
       mbar_init(&sm.q_full[i], 1);
       mbar_init(&sm.q_empty[i], 1);
     }
-    for (int i = 0; i < kKRing; ++i) {
+    for (int i = 0; i < CS::kKRing; ++i) {
       mbar_init(&sm.k_full[i], 1);
       mbar_init(&sm.k_empty[i], 1);
     }
-    for (int i = 0; i < kVRing; ++i) {
+    for (int i = 0; i < CS::kVRing; ++i) {
       mbar_init(&sm.v_full[i], 1);
       mbar_init(&sm.v_empty[i], 1);
     }
     for (int i = 0; i < kSets; ++i) {
-      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_full[i], C::kFp8 ? 2 : 1);
       mbar_init(&sm.p_full[i], 4);
       mbar_init(&sm.pv_done[i], 1);
     }
@@ -561,6 +625,9 @@ __global__ void __launch_bounds__(kCThreads, 1)
   if (warp == kWarpQK) tmem_dealloc(tmem, kCTmemCols);
 }
 
+// Keys and values follow the query plan (no geometry of their own).
+int same_plan(const rf_plan_t& g, const rf_plan_t& gk) { return std::memcmp(&g, &gk, sizeof(rf_plan_t)) == 0; }
+
 template <class C>
 cudaError_t launch_chain_cfg(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const AttnParams& p, cudaStream_t stream) {
@@ -597,6 +664,7 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
       !make_tile_map(&tv, v_int, rows_k, type, 2))
     return cudaErrorInvalidValue;
   AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, redo, dbg);
+  p.own_first = same_plan(g, gk);
   e = f16 ? launch_chain_cfg<Cfg<true, false>>(tq, tk, tv, p, stream)
           : launch_chain_cfg<Cfg<false, false>>(tq, tk, tv, p, stream);
   if (e != cudaSuccess) return e;
@@ -604,6 +672,34 @@ cudaError_t launch_attention(const void* q_int, const void* k_int, const void* v
   second.skip_first_q = 0;
   return launch_attention_slots(q_int, k_int, v_int, mask, dtype, layout, B, S, N, g, gk, scale, out, counter, status,
                                 redo, 1, second, stream);
+}
+
+cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
+                                 const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
+                                 const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out, int* counter,
+                                 int* status, int* redo, const AttnDebug& dbg, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(redo, 0, 2 * sizeof(int), stream);
+  if (e != cudaSuccess) return e;
+  if (dbg.path == 1)
+    return launch_attention_fp8_slots(q8, k8, v8, scales, vmax, mask, dtype, layout, B, S, N, g, gk, scale, out,
+                                      counter, status, redo, 0, dbg, stream);
+  const uint64_t rows_q = (uint64_t)B * N * g.S_int, rows_k = (uint64_t)B * N * gk.S_int;
+  CUtensorMap tq, tk, tv;
+  if (!make_tile_map(&tq, q8, rows_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tk, k8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1) ||
+      !make_tile_map(&tv, v8, rows_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1))
+    return cudaErrorInvalidValue;
+  AttnParams p = make_params(mask, layout, B, S, N, g, gk, scale, out, counter, status, redo, dbg);
+  p.scales = scales;
+  p.vmax = vmax;
+  p.own_first = same_plan(g, gk);
+  e = dtype == RF_F16 ? launch_chain_cfg<Cfg<true, true>>(tq, tk, tv, p, stream)
+                      : launch_chain_cfg<Cfg<false, true>>(tq, tk, tv, p, stream);
+  if (e != cudaSuccess) return e;
+  AttnDebug second = dbg;
+  second.skip_first_q = 0;
+  return launch_attention_fp8_slots(q8, k8, v8, scales, vmax, mask, dtype, layout, B, S, N, g, gk, scale, out,
+                                    counter, status, redo, 1, second, stream);
 }
 
 }  // namespace rf

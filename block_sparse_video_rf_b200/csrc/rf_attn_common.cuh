@@ -53,7 +53,16 @@ struct Cfg {
 };
 
 struct Item {
-  int bn, qt, ntiles, pad;
+  int bn, qt, ntiles;
+  int partial;   // chain_kernel: place of the partial key prefix tile in the unit's tile order (-1: none)
+};
+
+// Per-tile factors of the fp8 path, written by the slot's issuer before its
+// arrival on s_full: c = scale * log2(e) * sq * sk (multiplies S), lr =
+// log2(sv / vmax) (added to P's exponent), ir = vmax / sv (l adds P's sum
+// times ir).
+struct TileScale {
+  float c, lr, ir, pad;
 };
 
 struct AttnParams {
@@ -75,10 +84,23 @@ struct AttnParams {
   // counter, [1] the number of units listed (-1: every unit), [2 ...] their ids.
   int* redo;
   int list_mode;            // attn_kernel: take units from `redo` instead of all of them
+  int own_first;            // chain_kernel: keys share the query plan, so a unit starts with its own key tile
   float sum_limit;          // chain_kernel: tile sum of P that sends a unit to the second pass (0: the type's)
   uint64_t wait_limit_ns;   // limit of every device-side wait
   int skip_first_q;         // test control: the first unit's Q load is never issued
 };
+
+// The fp8 factors of one tile from the unit's Q block scale sq, the tile's
+// K and V block scales sk, sv and the head's largest V block scale vmax.
+__device__ __forceinline__ TileScale tile_scale(const AttnParams& p, float sq, float sk, float sv, float vmax) {
+  TileScale f;
+  f.c = p.scale_log2 * sq * sk;
+  const bool use_r = sv > 0.f && vmax > 0.f;   // an all-zero V block adds nothing whatever P is
+  f.lr = use_r ? __log2f(sv / vmax) : 0.f;
+  f.ir = use_r ? vmax / sv : 1.f;
+  f.pad = 0.f;
+  return f;
+}
 
 __device__ __forceinline__ bool is_dense_tile(const AttnParams& p, int qt) {
   return p.g.dense || qt < p.n_ptiles || (qt - p.n_ptiles) < p.g.ff;
@@ -95,7 +117,7 @@ __device__ __forceinline__ int unit_of(const AttnParams& p, int w) {
 // The unit of work item w: its (head, query tile) and KV tile count; `mrow`
 // is its mask row (nullptr for a dense tile).
 __device__ __forceinline__ Item make_item(const AttnParams& p, int unit, const uint32_t*& mrow) {
-  Item itm{-1, 0, 0, 0};
+  Item itm{-1, 0, 0, -1};
   mrow = nullptr;
   if (unit < 0) return itm;
   itm.bn = unit / p.g.n_tiles;
@@ -138,13 +160,17 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // Visits the KV tile rows of one unit in order: every prefix tile, then every
-// sparse block (dense unit) or the set bits of its mask row.
+// sparse block (dense unit) or the set bits of its mask row.  With own >= 0
+// (a key tile index: prefix tile, or n_ptiles + block) that tile comes
+// first and the rest follow in that order.
 struct KvIter {
   int base, n_ptiles, nb, words;
   const uint32_t* mrow;   // nullptr for a dense unit
   int t, wd;
   uint32_t bits;
-  __device__ void init(int base_, const AttnParams& p, const uint32_t* mrow_) {
+  int own;                // the tile visited first, or -1
+  bool own_done;
+  __device__ void init(int base_, const AttnParams& p, const uint32_t* mrow_, int own_ = -1) {
     base = base_;
     n_ptiles = p.n_ptiles_k;
     nb = p.gk.nb;
@@ -153,9 +179,22 @@ struct KvIter {
     t = 0;
     wd = 0;
     bits = 0;
+    own = own_;
+    own_done = own_ < 0;
   }
   // Row of the next KV tile, or -1 at the end.
   __device__ int next() {
+    if (!own_done) {
+      own_done = true;
+      return base + own * RF_BLOCK;
+    }
+    int r;
+    do {
+      r = next_natural();
+    } while (own >= 0 && r == base + own * RF_BLOCK);
+    return r;
+  }
+  __device__ int next_natural() {
     if (t < n_ptiles) return base + (t++) * RF_BLOCK;
     if (!mrow) {
       const int j = t - n_ptiles;
@@ -172,6 +211,25 @@ struct KvIter {
     return base + (n_ptiles + j) * RF_BLOCK;
   }
 };
+
+// The key tile of a unit's own rows (same index as its query tile) when keys
+// share the query plan and the unit reads that tile, else -1.  Attention is
+// strongest near the query in video, so the unit's reference maximum is best
+// taken there.
+__device__ __forceinline__ int own_tile(const AttnParams& p, const Item& itm, const uint32_t* mrow) {
+  if (!p.own_first || itm.bn < 0) return -1;
+  if (itm.qt < p.n_ptiles || !mrow) return itm.qt;
+  const int b = itm.qt - p.n_ptiles;
+  return ((mrow[b >> 5] >> (b & 31)) & 1u) ? itm.qt : -1;
+}
+// Place of the partial key prefix tile (index n_ptiles_k - 1) in the order
+// KvIter gives with `own` first; -1 when the prefix has no partial tile.
+__device__ __forceinline__ int partial_place(const AttnParams& p, int own) {
+  if (p.p_rem_k == 0) return -1;
+  const int part = p.n_ptiles_k - 1;
+  if (own < 0 || own < part) return part;
+  return own == part ? 0 : part + 1;
+}
 
 // One 128 x 128 tile: one box of 128 bytes per row (fp8) or two boxes of 64
 // 16-bit columns.
@@ -379,6 +437,7 @@ inline AttnParams make_params(const uint32_t* mask, int layout, int B, int S, in
   p.out = out;
   p.redo = redo;
   p.list_mode = 0;
+  p.own_first = 0;
   p.sum_limit = dbg.sum_limit;
   p.wait_limit_ns = dbg.wait_limit_ns > 0 ? (uint64_t)dbg.wait_limit_ns : kWaitLimitNs;
   p.skip_first_q = dbg.skip_first_q;

@@ -60,11 +60,19 @@ cudaError_t launch_quantize_fp8(const void* q_int, const void* k_int, const void
                                 const rf_plan_t& g, const rf_plan_t& gk, uint8_t* q8, uint8_t* k8, uint8_t* v8,
                                 float* scales, float* vmax, cudaStream_t stream);
 
-// K3 on the e4m3 tensors of launch_quantize_fp8; output in dtype.
+// K3 on the e4m3 tensors of launch_quantize_fp8; output in dtype.  As
+// launch_attention: chain_kernel, then attn_kernel over the units it lists
+// (P above e4m3's 448).
 cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
                                  const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S, int N,
                                  const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out, int* counter,
-                                 int* status, const AttnDebug& dbg, cudaStream_t stream);
+                                 int* status, int* redo, const AttnDebug& dbg, cudaStream_t stream);
+// attn_kernel's fp8 form over every unit (list_mode 0) or the units listed in redo (list_mode 1).
+cudaError_t launch_attention_fp8_slots(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,
+                                       const float* vmax, const uint32_t* mask, int dtype, int layout, int B, int S,
+                                       int N, const rf_plan_t& g, const rf_plan_t& gk, float scale, void* out,
+                                       int* counter, int* status, int* redo, int list_mode, const AttnDebug& dbg,
+                                       cudaStream_t stream);
 
 // Block mask with the pooled means in the library's static scratch array
 // (no device allocation); see rf_block_mask_noalloc.

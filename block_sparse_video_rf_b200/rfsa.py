@@ -335,8 +335,7 @@ def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"
         "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),
         "kept": view(lay.kept, heads * nb, torch.int32, (B, N, nb)),
         "margin": view(lay.margin, heads * nb, torch.float32, (B, N, nb)),
-    } | ({} if precision == "fp8" else {"redo": view(lay.redo, 2 + heads * plan.n_tiles, torch.int32,
-                                                         (2 + heads * plan.n_tiles,))})
+    } | {"redo": view(lay.redo, 2 + heads * plan.n_tiles, torch.int32, (2 + heads * plan.n_tiles,))}
 
 
 def alloc_workspace(B, S, N, D, txt_len, latent, device="cuda", precision: str = "native", S_kv: int = 0,

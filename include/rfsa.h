@@ -106,9 +106,8 @@ typedef struct {
  * transposed ([B, N, n_tiles, 128 channels, 128 rows]); scales: fp32
  * q [B, N, n_tiles_q], then k and v [B, N, n_tiles_kv]; vmax: fp32 [B, N],
  * the largest V block scale of each head.
- * Only with RF_PREC_NATIVE: redo: int32 [2 + B * N * n_tiles_q], the query
- * tiles the 16-bit attention hands to its second pass ([0] a work counter,
- * [1] how many, [2 ...] their ids). */
+ * redo: int32 [2 + B * N * n_tiles_q], the query tiles the attention hands
+ * to its second pass ([0] a work counter, [1] how many, [2 ...] their ids). */
 typedef struct {
   size_t q_int, k_int, v_int, pooled_q, pooled_k, mask, kept, margin, counter, status;
   size_t q8, k8, v8, scales, vmax;

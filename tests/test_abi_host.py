@@ -161,12 +161,12 @@ def test_fp8_workspace_layout(rfsa):
     codes = 56 * 62848 * 128
     assert _regions_disjoint(lay, {"q_int": 2 * codes, "v_int": 2 * codes, "q8": codes, "k8": codes, "v8": codes,
                                    "scales": 3 * 56 * p.n_tiles * 4, "vmax": 56 * 4})
-    # the native layout is the same up to the fp8 regions, which it leaves empty; it ends with the
-    # redo list of the 16-bit attention (two counters and one id per query tile), which fp8 leaves empty
+    # the native layout is the same up to the fp8 regions, which it leaves empty; both end with the
+    # attention's redo list (two counters and one id per query tile)
     assert [getattr(nat, f) for f in rfsa.WS_FIELDS[:10]] == offs[:10]
     assert nat.q8 == nat.k8 == nat.v8 == nat.scales == nat.vmax == nat.redo
-    assert nat.total - nat.redo >= (2 + 56 * p.n_tiles) * 4
-    assert lay.redo == lay.total
+    for L in (nat, lay):
+        assert L.total - L.redo >= (2 + 56 * p.n_tiles) * 4
     assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42), precision="fp8") == lay.total
 
 

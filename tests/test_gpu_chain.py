@@ -114,3 +114,49 @@ def test_scores_beyond_headroom(rfsa, dtype, gain):
     assert redo[1] > 0
     ref = _oracle(w, q.to(torch.float32), k.to(torch.float32), v.to(torch.float32))
     assert_close(to_np(out), ref, f"beyond headroom {dtype}")
+
+
+def _fp8_check(w, q, k, v, out, what):
+    from oracle import fp8
+    from parity_util import assert_close_fp8, to_bnsd_np
+    ref, _, _, g = fp8.rf_sparse_attention_fp8(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent,
+                                               float(np.float32(w.sparsity)))
+    ob, rb, vb = to_bnsd_np(out, w.layout), oracle.to_bnsd(ref, w.layout), to_bnsd_np(v, w.layout)
+    for b in range(w.B):
+        for n in range(w.N):
+            vd = fp8.quantize_head(vb[b, n], g)[0]
+            assert_close_fp8(ob[b, n], rb[b, n], vd, f"{what} b{b} n{n}")
+
+
+@pytest.mark.parametrize("case", ["tiny", "ragged", "batch2"])
+@pytest.mark.parametrize("path,limit", [(0, 0.0), (1, 0.0), (0, 3.0)], ids=["chain", "two_tile", "handover"])
+def test_fp8_paths_against_oracle(rfsa, case, path, limit):
+    # e4m3 operands: the chain kernel (fp8 form), the two-tile kernel alone, and
+    # a lowered limit that hands a share of the units from one to the other
+    name, over = CASES[case]
+    w, q, k, v = _inputs(name, **over)
+    rfsa.rf_debug_set_path(path, limit)
+    try:
+        out = rfsa.rf_sparse_attention(q, k, v, w.layout, w.txt_len, w.latent, np.float32(w.sparsity),
+                                       precision="fp8")
+        torch.cuda.synchronize()
+    finally:
+        rfsa.rf_debug_set_path(0, 0.0)
+    _fp8_check(w, q, k, v, out, f"fp8 {case} path {path} limit {limit}")
+
+
+def test_fp8_scores_beyond_headroom(rfsa):
+    # later tiles' P would pass e4m3's 448 against the first tile's maximum:
+    # those units go to the second pass, which rescales
+    w, q, k, v = _inputs("tiny", txt_len=128, latent=(4, 32, 32), N=2, seed=31)
+    k = k.clone()
+    k[:, w.txt_len:] *= 6.0
+    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent, precision="fp8")
+    out = torch.empty_like(q)
+    rfsa.rf_sparse_attention_ws(q, k, v, w.layout, w.txt_len, w.latent, np.float32(w.sparsity), ws, out=out,
+                                precision="fp8")
+    torch.cuda.synchronize()
+    plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, np.float32(w.sparsity))
+    redo = rfsa.workspace_views(ws, w.B, w.N, plan, precision="fp8")["redo"].cpu().numpy()
+    assert redo[1] > 0
+    _fp8_check(w, q, k, v, out, "fp8 beyond headroom")
