@@ -119,6 +119,39 @@ rf_status_t cached_buffer(WsCache& c, size_t need, void** out) {
   return RF_OK;
 }
 
+// Copy streams and events of rf_sparse_attention_host, one set per device,
+// created on first use (non-blocking streams, so a caller on the legacy
+// default stream still overlaps with them).
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t loaded[2] = {}, comp[2] = {}, stored[2] = {};
+};
+std::mutex g_pipe_mu;
+HostPipe g_pipe[64];
+bool g_pipe_ready[64] = {};
+
+rf_status_t host_pipe(HostPipe** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(RF_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& p = g_pipe[dev];
+  if (!g_pipe_ready[dev]) {
+    e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking);
+    for (int z = 0; z < 2 && e == cudaSuccess; ++z) {
+      e = cudaEventCreateWithFlags(&p.loaded[z], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.comp[z], cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.stored[z], cudaEventDisableTiming);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "creating the host-buffer pipeline's streams and events");
+    g_pipe_ready[dev] = true;
+  }
+  *out = &p;
+  return RF_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -407,29 +440,73 @@ rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void*
   if (!qh || !kh || !vh || !out_h) return fail(RF_ERR_ARG, "host buffers must not be NULL");
   rf_plan_t g;
   if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
+  // Heads are independent: the call runs on chunks of c heads of one batch
+  // entry, each a [1, S, c, D] (BSND) or [1, c, S, D] (BNSD) problem, in two
+  // device slots.  While chunk i computes on the caller's stream, chunk i + 1
+  // is copied in on one stream and chunk i - 1 copied out on another.
+  const size_t head_bytes = (size_t)S * D * 2;
+  const int c = std::max(1, std::min(N, (int)(((size_t)192 << 20) / (3 * head_bytes))));
+  const size_t chunk = align256((size_t)c * head_bytes);
   rf_ws_layout_t L;
-  if ((st = rf_workspace_layout(B, N, D, &g, &L)) != RF_OK) return st;
-  const size_t tensor = (size_t)B * S * N * D * 2;
-  const size_t t_al = align256(tensor);
+  if ((st = rf_workspace_layout(1, c, D, &g, &L)) != RF_OK) return st;
+  const size_t ws_slot = align256(L.total);
   void* io = nullptr;
   void* ws = nullptr;
-  if ((st = cached_buffer(g_io, 4 * t_al, &io)) != RF_OK) return st;
-  if ((st = cached_buffer(g_ws, L.total, &ws)) != RF_OK) return st;
-  char* d = static_cast<char*>(io);
+  if ((st = cached_buffer(g_io, 2 * 4 * chunk, &io)) != RF_OK) return st;
+  if ((st = cached_buffer(g_ws, 2 * ws_slot, &ws)) != RF_OK) return st;
+  HostPipe* hp = nullptr;
+  if ((st = host_pipe(&hp)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  const void* srcs[3] = {qh, kh, vh};
-  for (int i = 0; i < 3; ++i) {
-    e = cudaMemcpyAsync(d + i * t_al, srcs[i], tensor, cudaMemcpyHostToDevice, s);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (host to device)");
+  const bool bsnd = layout == RF_BSND;
+  const size_t row = (size_t)N * D * 2;   // BSND: one token's heads
+  auto copy = [&](void* dst, const void* src, int heads, cudaMemcpyKind kind, bool to_dev, cudaStream_t cs) {
+    if (!bsnd) return cudaMemcpyAsync(dst, src, (size_t)heads * head_bytes, kind, cs);
+    const size_t w = (size_t)heads * D * 2;
+    return to_dev ? cudaMemcpy2DAsync(dst, w, src, row, w, S, kind, cs)
+                  : cudaMemcpy2DAsync(dst, row, src, w, w, S, kind, cs);
+  };
+  const char* srcs[3] = {static_cast<const char*>(qh), static_cast<const char*>(kh), static_cast<const char*>(vh)};
+  char* outh = static_cast<char*>(out_h);
+  int i = 0;
+  cudaError_t e = cudaSuccess;
+  for (int b = 0; b < B; ++b) {
+    for (int n0 = 0; n0 < N; n0 += c, ++i) {
+      const int heads = std::min(c, N - n0);
+      const int z = i & 1;
+      char* d = static_cast<char*>(io) + (size_t)z * 4 * chunk;
+      // host offset of the chunk's first element
+      const size_t off = bsnd ? ((size_t)b * S * N + n0) * D * 2 : ((size_t)b * N + n0) * head_bytes;
+      // copy in once the slot's previous chunk has been computed
+      if (i >= 2 && (e = cudaStreamWaitEvent(hp->in, hp->comp[z], 0)) != cudaSuccess) break;
+      for (int t = 0; t < 3 && e == cudaSuccess; ++t)
+        e = copy(d + t * chunk, srcs[t] + off, heads, cudaMemcpyHostToDevice, true, hp->in);
+      if (e != cudaSuccess || (e = cudaEventRecord(hp->loaded[z], hp->in)) != cudaSuccess) break;
+      // compute once it is in and the slot's previous output has left
+      if ((e = cudaStreamWaitEvent(s, hp->loaded[z], 0)) != cudaSuccess) break;
+      if (i >= 2 && (e = cudaStreamWaitEvent(s, hp->stored[z], 0)) != cudaSuccess) break;
+      st = rf_sparse_attention_ws(d, d + chunk, d + 2 * chunk, layout, 1, S, heads, D, txt_len, T, H, W, block_size,
+                                  sparsity, scale, d + 3 * chunk, static_cast<char*>(ws) + (size_t)z * ws_slot,
+                                  ws_slot, stream);
+      if (st != RF_OK) {
+        // no copy of the caller's buffers may still run when this returns
+        cudaStreamSynchronize(hp->in);
+        cudaStreamSynchronize(hp->out);
+        cudaStreamSynchronize(s);
+        return st;
+      }
+      if ((e = cudaEventRecord(hp->comp[z], s)) != cudaSuccess) break;
+      // copy out
+      if ((e = cudaStreamWaitEvent(hp->out, hp->comp[z], 0)) != cudaSuccess) break;
+      if ((e = copy(outh + off, d + 3 * chunk, heads, cudaMemcpyDeviceToHost, false, hp->out)) != cudaSuccess) break;
+      if ((e = cudaEventRecord(hp->stored[z], hp->out)) != cudaSuccess) break;
+    }
+    if (e != cudaSuccess) break;
   }
-  st = rf_sparse_attention_ws(d, d + t_al, d + 2 * t_al, layout, B, S, N, D, txt_len, T, H, W, block_size, sparsity,
-                              scale, d + 3 * t_al, ws, L.total, stream);
-  if (st != RF_OK) return st;
-  e = cudaMemcpyAsync(out_h, d + 3 * t_al, tensor, cudaMemcpyDeviceToHost, s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpyAsync (device to host)");
-  e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  const cudaError_t e_in = cudaStreamSynchronize(hp->in);
+  const cudaError_t e_out = cudaStreamSynchronize(hp->out);
+  const cudaError_t e_s = cudaStreamSynchronize(s);
+  if (e == cudaSuccess) e = e_in != cudaSuccess ? e_in : e_out != cudaSuccess ? e_out : e_s;
+  if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline (copies, events or synchronisation)");
   return ok();
 }
 

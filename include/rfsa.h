@@ -209,9 +209,14 @@ rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, in
                          int latent_t, int latent_h, int latent_w, void* out, void* stream);
 
 /* End-to-end through HOST buffers (bf16, caller layout): copies q, k, v to
- * the device, runs the call with the cached workspace, copies the result
- * back to out_host and synchronises `stream`.  Host buffers should be pinned
- * for full copy bandwidth. */
+ * the device, runs the call, copies the result back to out_host and
+ * synchronises.  The heads are independent, so the call runs on chunks of
+ * heads (about 192 MiB of q, k and v each) in two device slots: chunk i + 1
+ * is copied in and chunk i - 1 copied out, on two library-owned streams,
+ * while chunk i computes on `stream`.  Buffers are cached by the library per
+ * device.  Host buffers should be pinned: pageable ones still give the right
+ * result, with the copies no longer overlapping the compute.  On return no
+ * copy of the caller's buffers is in flight, also after an error. */
 rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, const void* v_host, rf_layout_t layout,
                                      int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
                                      int latent_w, int block_size, float sparsity, float scale, void* out_host,
