@@ -52,6 +52,26 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs):
+    """Per-stage times with the HBM-bound stage's algorithmic bytes: K1 reads q, k, v in the caller's layout and
+    writes the internal copies plus the fp32 block means of q and k, K2 reads the block means and writes the
+    mask, kept counts and margins; fp8 adds the quantisation pass (reads the internal copies, writes e4m3 codes
+    and one fp32 scale per 128-row block)."""
+    heads = w.B * w.N
+    row = 128 * 2                                          # one token's head vector, bytes
+    pooled = 2 * plan.nb * 128 * 4                         # q and k block means, bytes per head
+    words = (plan.nb + 31) // 32
+    k1 = heads * (3 * w.S * row + 3 * plan.S_int * row + pooled)
+    k2 = heads * (pooled + plan.nb * (words * 4 + 8))
+    kq = heads * (3 * plan.S_int * row + 3 * plan.S_int * 128 + 3 * plan.n_tiles * 4) if prec == "fp8" else 0
+    moved = k1 + k2 + kq
+    gbs = moved / (ms_prepare * 1e-3) / 1e9
+    return {"prepare": {"kernels": "K1 reorder + block means, K2 block scores + top-k" +
+                        (", Kq e4m3 quantisation" if prec == "fp8" else ""),
+                        "ms": ms_prepare, "algorithmic_bytes": moved, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs},
+            "attention": {"kernels": "K3", "ms": ms_attention, "tflops": k3_tflops}}
+
+
 # The attention kernels' sources, hashed together to tie a traffic capture to the code it measured.
 K3_SOURCES = ("rf_attn_common.cuh", "rf_attn_chain.cu", "rf_attn.cu")
 
@@ -359,6 +379,7 @@ def main():
             # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
             # handed to it); fp8 adds the quantisation pass
             "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
+            "stages": _stages(w, plan, prec, statistics.mean(k1k2), k3_ms, k3_tflops, peaks["hbm_gbs"]),
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -14,6 +14,7 @@
 #include <cstdio>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "rf_geometry.h"
 #include "rf_kernels.h"
@@ -526,6 +527,52 @@ rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the status word");
   *status = h;
+  return ok();
+}
+
+rf_status_t rf_read_stats(void* ws, size_t ws_bytes, int B, int N, int D, const rf_plan_t* g, rf_stats_t* stats,
+                          void* stream) {
+  if (!stats) return fail(RF_ERR_ARG, "stats pointer is NULL");
+  rf_ws_layout_t L;
+  rf_status_t st = rf_workspace_layout(B, N, D, g, &L);
+  if (st != RF_OK) return st;
+  if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
+  const size_t heads = (size_t)B * N, rows = heads * g->nb;
+  std::vector<int> kept(rows);
+  std::vector<float> margin(rows);
+  int redo[2] = {0, 0}, status = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaSuccess;
+  if (rows) {
+    e = cudaMemcpyAsync(kept.data(), at<int>(ws, L.kept), rows * sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(margin.data(), at<float>(ws, L.margin), rows * sizeof(float), cudaMemcpyDeviceToHost, s);
+  }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(redo, at<int>(ws, L.redo), sizeof(redo), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&status, at<int>(ws, L.status), sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the workspace statistics");
+  rf_stats_t r{};
+  const double S = g->S;
+  if (g->dense) {
+    r.kept_pairs = (double)heads * S * S;
+  } else {
+    const double dense_rows = (double)g->P + 128.0 * g->ff;
+    double sparse_keys = 0;
+    for (size_t h = 0; h < heads; ++h)
+      for (int i = g->ff; i < g->nb; ++i) {
+        const size_t j = h * g->nb + i;
+        r.kept_blocks += kept[j];
+        sparse_keys += 128.0 * kept[j] + g->P;
+        if (margin[j] < 1e-5f) ++r.near_ties;
+      }
+    r.query_blocks = (long long)heads * (g->nb - g->ff);
+    r.kept_pairs = (double)heads * dense_rows * S + 128.0 * sparse_keys;
+  }
+  r.density = r.kept_pairs / ((double)heads * S * S);
+  r.redo_tiles = redo[1] < 0 ? (int)(heads * g->n_tiles) : redo[1];
+  r.status = status;
+  *stats = r;
   return ok();
 }
 

@@ -31,7 +31,7 @@ PRECISIONS = {"native": 0, "fp8": 1}
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_debug_set_wait", "rf_debug_set_path", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
+           "rf_debug_set_wait", "rf_debug_set_path", "rf_read_stats", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
            "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv"]
 
 
@@ -44,6 +44,15 @@ class RfPlan(ctypes.Structure):
 
 class RfWsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in WS_FIELDS]
+
+
+class RfStats(ctypes.Structure):
+    _fields_ = [("kept_blocks", ctypes.c_longlong), ("query_blocks", ctypes.c_longlong),
+                ("kept_pairs", ctypes.c_double), ("density", ctypes.c_double), ("near_ties", ctypes.c_int),
+                ("redo_tiles", ctypes.c_int), ("status", ctypes.c_int)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
 
 
 class RfError(RuntimeError):
@@ -72,6 +81,7 @@ def _load():
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "rf_debug_set_path": (I, [I, F]),
+        "rf_read_stats": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfStats), P]),
         "rf_last_error_string": (ctypes.c_char_p, []),
         "rf_plan_kv": (I, [I, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan)]),
         "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan),
@@ -295,6 +305,14 @@ def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
     _check(LIB.rf_read_status(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
                               ctypes.byref(plan), ctypes.byref(st), _stream(workspace, stream)))
     return st.value
+
+
+def rf_read_stats(workspace, B, N, D, plan, stream=None) -> dict:
+    """Statistics of the last call on a workspace (see include/rfsa.h)."""
+    st = RfStats()
+    _check(LIB.rf_read_stats(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
+                             ctypes.byref(plan), ctypes.byref(st), _stream(workspace, stream)))
+    return st.as_dict()
 
 
 def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native", plan_kv=None):

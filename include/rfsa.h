@@ -115,6 +115,18 @@ typedef struct {
   size_t total;
 } rf_ws_layout_t;
 
+/* Statistics of the last call on a workspace (rf_read_stats). */
+typedef struct {
+  long long kept_blocks;   /* key blocks kept over all sparse query blocks (top-k plus forced first-frame columns) */
+  long long query_blocks;  /* sparse query blocks that select (B * N * (nb - ff)) */
+  double kept_pairs;       /* (query row, key) pairs attended: dense rows read all S keys, a sparse block's rows
+                            * the P prefix keys plus 128 per kept block; 4 * D * kept_pairs is the kept-block work */
+  double density;          /* kept_pairs / (B * N * S * S) */
+  int near_ties;           /* sparse query blocks whose k-th and (k+1)-th block scores are within 1e-5 (relative) */
+  int redo_tiles;          /* query tiles the attention handed to its second pass (P beyond its type's headroom) */
+  int status;              /* the workspace status word (not cleared) */
+} rf_stats_t;
+
 /* Host-only: validate a geometry and fill *plan.  No CUDA call. */
 rf_status_t rf_plan(int S, int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
                     rf_plan_t* plan);
@@ -229,6 +241,16 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
  * Returns RF_OK, RF_ERR_ARG, RF_ERR_WORKSPACE or RF_ERR_CUDA. */
 rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                            int* status, void* stream);
+
+/* Synchronises `stream` and reads *stats from a workspace after rf_prepare +
+ * rf_attend (or rf_sparse_attention_ws) with keys in the query's geometry
+ * and native precision: the kept counts and k-th-score margins of the mask,
+ * the redo list and the status word (copied, not cleared).  The debug view of
+ * a call: how much of the sequence it kept, how many selections sat on a
+ * near-tie (R7), how many tiles took the second pass.
+ * Returns RF_OK, RF_ERR_ARG, RF_ERR_WORKSPACE or RF_ERR_CUDA. */
+rf_status_t rf_read_stats(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
+                          rf_stats_t* stats, void* stream);
 
 /* Test control of the device-side waits of the attention kernel, process-wide,
  * read at each launch.  wait_limit_ns: limit of every wait (0 = the default,

@@ -198,3 +198,15 @@ def test_key_geometry_workspace(rfsa):
     n2 = rfsa.rf_workspace_size(1, 7 + 768, 1, 128, 7, (3, 16, 16), "native", 7 + 6400, (5, 32, 40))
     n3 = rfsa.rf_workspace_size(1, 7 + 768, 1, 128, 7, (3, 16, 16), "native", 7 + 6400, (0, 0, 0))
     assert n2 == n3 > 0
+
+
+def test_read_stats_validates_before_any_cuda_call(rfsa):
+    import ctypes
+    L = rfsa.LIB
+    p = rfsa.rf_plan(4096, 0, (4, 32, 32), 0.5)
+    st = rfsa.RfStats()
+    P = ctypes.c_void_p
+    assert L.rf_read_stats(P(0x1000), 1 << 30, 1, 2, 128, ctypes.byref(p), None, None) == 2      # NULL stats
+    assert L.rf_read_stats(None, 1 << 30, 1, 2, 128, ctypes.byref(p), ctypes.byref(st), None) == 5   # NULL workspace
+    assert L.rf_read_stats(P(0x1000), 16, 1, 2, 128, ctypes.byref(p), ctypes.byref(st), None) == 5   # too small
+    assert L.rf_read_stats(P(0x1000), 1 << 30, 1, 2, 64, ctypes.byref(p), ctypes.byref(st), None) == 3  # D != 128

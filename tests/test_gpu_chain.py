@@ -160,3 +160,30 @@ def test_fp8_scores_beyond_headroom(rfsa):
     redo = rfsa.workspace_views(ws, w.B, w.N, plan, precision="fp8")["redo"].cpu().numpy()
     assert redo[1] > 0
     _fp8_check(w, q, k, v, out, "fp8 beyond headroom")
+
+
+def test_read_stats_after_a_call(rfsa):
+    # rf_read_stats: the mask's kept blocks, density and near-ties as the
+    # workspace holds them, and the number of tiles that took the second pass
+    w, q, k, v = _inputs("tiny", N=2, txt_len=64, latent=(6, 32, 32), sparsity=0.6, seed=21)
+    plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, np.float32(w.sparsity))
+    ws = rfsa.alloc_workspace(w.B, w.S, w.N, w.D, w.txt_len, w.latent)
+    out = torch.empty_like(q)
+    rfsa.rf_sparse_attention_ws(q, k, v, w.layout, w.txt_len, w.latent, np.float32(w.sparsity), ws, out=out)
+    st = rfsa.rf_read_stats(ws, w.B, w.N, w.D, plan)
+    views = rfsa.workspace_views(ws, w.B, w.N, plan)
+    kept, margin = views["kept"].cpu(), views["margin"].cpu()
+    assert st["kept_blocks"] == int(kept[..., plan.ff:].sum())
+    assert st["query_blocks"] == w.B * w.N * (plan.nb - plan.ff)
+    assert st["near_ties"] == int((margin[..., plan.ff:] < 1e-5).sum())
+    flops = rfsa.kept_block_flops(plan, kept, w.B, w.N, w.D)
+    assert abs(st["kept_pairs"] * 4 * w.D - flops) <= 1e-9 * flops
+    assert abs(st["density"] - st["kept_pairs"] / (w.B * w.N * w.S * w.S)) < 1e-12
+    assert 0 < st["density"] < 1 and st["redo_tiles"] == 0 and st["status"] == 0
+    rfsa.rf_debug_set_path(0, 4.0)
+    try:
+        rfsa.rf_sparse_attention_ws(q, k, v, w.layout, w.txt_len, w.latent, np.float32(w.sparsity), ws, out=out)
+        st2 = rfsa.rf_read_stats(ws, w.B, w.N, w.D, plan)
+    finally:
+        rfsa.rf_debug_set_path(0, 0.0)
+    assert st2["redo_tiles"] == int(views["redo"][1].item()) > 0
