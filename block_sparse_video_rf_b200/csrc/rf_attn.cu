@@ -1,6 +1,8 @@
 // Block-sparse flash attention on sm_100a tensor cores (K3), two query
-// tiles per CTA: the fp8 path, and the second pass of the 16-bit path (the
-// units chain_kernel hands back, see rf_attn_chain.cu).
+// tiles per CTA, with a running maximum that is raised (and O and l
+// rescaled) when a tile needs it: the second pass of every precision (the
+// units chain_kernel hands back, see rf_attn_chain.cu), and the whole of K3
+// when a test selects it (rf_debug_set_path).
 //
 // vllm-omni "RainFusion Attention", intro: prefix rows and first-frame
 // blocks stay dense; every other query block attends to its highest-scoring
