@@ -58,6 +58,10 @@ CASES = {
     "dense": ("tiny", {"sparsity": 0.0, "seed": 13}),
     "batch2": ("tiny", {"B": 2, "N": 2, "txt_len": 37, "latent": (6, 24, 40), "sparsity": 0.6, "seed": 41}),
     "short_units": ("tiny", {"txt_len": 0, "latent": (3, 16, 16), "sparsity": 0.9, "seed": 14}),
+    # one first-frame block and k = 0 / 1: every sparse unit reads 1 / 2 key tiles, so sets 1 and 2 (and set
+    # 2) have no tile in it and the S buffers are reused back to back
+    "one_tile_units": ("tiny", {"txt_len": 0, "latent": (32, 8, 16), "sparsity": 1.0, "seed": 15}),
+    "two_tile_units": ("tiny", {"txt_len": 0, "latent": (32, 8, 16), "sparsity": 0.97, "seed": 16}),
 }
 
 
@@ -128,7 +132,7 @@ def _fp8_check(w, q, k, v, out, what):
             assert_close_fp8(ob[b, n], rb[b, n], vd, f"{what} b{b} n{n}")
 
 
-@pytest.mark.parametrize("case", ["tiny", "ragged", "batch2"])
+@pytest.mark.parametrize("case", ["tiny", "ragged", "batch2", "one_tile_units"])
 @pytest.mark.parametrize("path,limit", [(0, 0.0), (1, 0.0), (0, 3.0)], ids=["chain", "two_tile", "handover"])
 def test_fp8_paths_against_oracle(rfsa, case, path, limit):
     # e4m3 operands: the chain kernel (fp8 form), the two-tile kernel alone, and
