@@ -153,7 +153,11 @@ size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D
                             int latent_h, int latent_w, int S_kv, int kv_t, int kv_h, int kv_w);
 
 /* The whole rf_v2 call, with a workspace cached by the library per device
- * (grown with cudaMalloc on first use of a larger shape; never shrunk). */
+ * (grown with cudaMalloc on first use of a larger shape; never shrunk).  The
+ * cached buffers are shared by rf_sparse_attention, rf_sparse_attention_ex
+ * (NULL workspace) and rf_sparse_attention_host on a device: calls from
+ * several host threads to the same device must be serialised by the caller,
+ * and device calls must be ordered on one stream. */
 rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
                                 int D, int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
                                 float sparsity, float scale, void* out, void* stream);
