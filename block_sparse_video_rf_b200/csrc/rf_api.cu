@@ -445,8 +445,13 @@ rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void*
   // entry, each a [1, S, c, D] (BSND) or [1, c, S, D] (BNSD) problem, in two
   // device slots.  While chunk i computes on the caller's stream, chunk i + 1
   // is copied in on one stream and chunk i - 1 copied out on another.
+  // About 96 MiB of q, k and v per chunk (2 heads at MiniMax-H3): a shorter
+  // pipeline tail than 192 MiB (52.3 vs 53.4 ms per call there).  At least 2
+  // heads when BSND: a chunk of 1 head copies 256-byte rows, and the strided
+  // copy then runs far below the link's rate (81.6 ms).
   const size_t head_bytes = (size_t)S * D * 2;
-  const int c = std::max(1, std::min(N, (int)(((size_t)192 << 20) / (3 * head_bytes))));
+  int c = std::max(1, std::min(N, (int)(((size_t)96 << 20) / (3 * head_bytes))));
+  if (layout == RF_BSND && c < 2) c = std::min(N, 2);
   const size_t chunk = align256((size_t)c * head_bytes);
   rf_ws_layout_t L;
   if ((st = rf_workspace_layout(1, c, D, &g, &L)) != RF_OK) return st;

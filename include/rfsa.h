@@ -227,7 +227,8 @@ rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, in
 /* End-to-end through HOST buffers (bf16, caller layout): copies q, k, v to
  * the device, runs the call, copies the result back to out_host and
  * synchronises.  The heads are independent, so the call runs on chunks of
- * heads (about 192 MiB of q, k and v each) in two device slots: chunk i + 1
+ * heads (about 96 MiB of q, k and v each, and at least two heads in BSND) in
+ * two device slots: chunk i + 1
  * is copied in and chunk i - 1 copied out, on two library-owned streams,
  * while chunk i computes on `stream`.  Buffers are cached by the library per
  * device.  Host buffers should be pinned: pageable ones still give the right

@@ -3,8 +3,8 @@ call on chunks of heads with the copies of neighbouring chunks overlapping
 the compute.  Heads are independent and every kernel's result for a head is
 the same whichever launch computes it, so the output must equal the device
 call on the whole tensors bit for bit.  At the MiniMax-H3 sequence length a
-chunk holds 4 heads: 7 heads and B = 2 give four chunks, a partial one among
-them, and reuse both device slots."""
+chunk holds 2 heads: 7 heads and B = 2 give eight chunks, a partial one
+among them, and reuse both device slots."""
 
 import numpy as np
 import pytest
