@@ -104,54 +104,102 @@ def _describe(w, dtype="bf16", precision="native") -> str:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
+    """SM clock, power and throttle reasons sampled every 20 ms while the
+    timed region runs (NVML in a thread of this process; nvidia-smi at 200 ms
+    where NVML cannot be loaded).  Only samples taken inside the region count,
+    so the median is the clock under load."""
+    PERIOD_S = 0.02
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index: int):
-        self.proc = None
-        self.lines = []
         self.device_index = device_index
+        self.samples = []           # (sm_mhz, max_mhz, watts, reason names)
+        self.source = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            pr = torch.cuda.get_device_properties(self.device_index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.device_index)
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
+            nv, h = self._nvml_handle()
+        except Exception:
+            nv = None
+        if nv is not None:
+            bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": nv.nvmlClocksEventReasonSwPowerCap}
+            self._stop = threading.Event()
+
+            def run():
+                while not self._stop.is_set():
+                    try:
+                        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+                        watts = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((float(sm), float(mx), watts, [n for n, b in bits.items() if r & b]))
+                    except Exception:
+                        pass
+                    self._stop.wait(self.PERIOD_S)
+
+            self.source = "nvml"
+            self._thread = threading.Thread(target=run, daemon=True)
+            self._thread.start()
+            return self
+        try:
+            self._proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "200",
                  "-i", str(self.device_index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.source = "nvidia-smi"
         except OSError:
-            self.proc = None
-        time.sleep(0.3)
+            self._proc = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            time.sleep(0.25)
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                out, _ = self._proc.communicate(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
+                self._proc.kill()
+                out, _ = self._proc.communicate()
+            for line in out.splitlines():
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm, mx, watts = float(parts[1]), float(parts[2]), float(parts[3])
+                except ValueError:
+                    continue
+                self.samples.append((sm, mx, watts, [n for n, v in zip(self.NAMES, parts[5:9])
+                                                     if v.lower().startswith("active")]))
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx = float(parts[2])
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
+        if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        reasons = sorted({n for smp in self.samples for n in smp[3]})
+        return {"sm_mhz": statistics.median(smp[0] for smp in self.samples), "sm_max_mhz": self.samples[-1][1],
+                "reasons": reasons, "samples": len(self.samples),
+                "power_w_median": round(statistics.median(smp[2] for smp in self.samples), 1),
+                "source": self.source}
 
 
 # ---------------------------------------------------------------- multi-rank aggregation

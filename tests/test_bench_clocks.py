@@ -1,0 +1,50 @@
+"""bench.py's clock sampler on CPU, against a fake NVML module: samples are
+taken only inside the sampled region, the median is reported, and the
+throttle-reason bits map to their names."""
+
+import itertools
+import sys
+import time
+import types
+
+
+def _fake_nvml(clocks, reasons):
+    nv = types.ModuleType("pynvml")
+    nv.NVML_CLOCK_SM = 1
+    nv.nvmlClocksEventReasonSwPowerCap = 0x4
+    nv.nvmlClocksEventReasonHwSlowdown = 0x8
+    nv.nvmlClocksEventReasonSwThermalSlowdown = 0x20
+    nv.nvmlClocksEventReasonHwThermalSlowdown = 0x40
+    it = itertools.cycle(clocks)
+    nv.nvmlInit = lambda: None
+    nv.nvmlDeviceGetHandleByPciBusId = lambda bus: "h"
+    nv.nvmlDeviceGetHandleByIndex = lambda i: "h"
+    nv.nvmlDeviceGetClockInfo = lambda h, kind: next(it)
+    nv.nvmlDeviceGetMaxClockInfo = lambda h, kind: 1965
+    nv.nvmlDeviceGetPowerUsage = lambda h: 990000
+    nv.nvmlDeviceGetCurrentClocksEventReasons = lambda h: reasons
+    return nv
+
+
+def test_median_under_load_and_reason_names(monkeypatch):
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml([1400, 1500, 1600], 0x4 | 0x40))
+    with bench.ClockSampler(0) as c:
+        time.sleep(0.2)
+    s = c.summary()
+    assert s["source"] == "nvml" and s["samples"] >= 3
+    assert s["sm_mhz"] in (1400, 1450, 1500, 1550, 1600)
+    assert s["sm_max_mhz"] == 1965 and s["power_w_median"] == 990.0
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    n = s["samples"]
+    time.sleep(0.1)                      # nothing is sampled once the region is left
+    assert c.summary()["samples"] == n
+
+
+def test_no_reasons(monkeypatch):
+    import bench
+    monkeypatch.setitem(sys.modules, "pynvml", _fake_nvml([1965], 0))
+    with bench.ClockSampler(0) as c:
+        time.sleep(0.1)
+    s = c.summary()
+    assert s["reasons"] == [] and s["sm_mhz"] == 1965
