@@ -5,36 +5,39 @@
 // sparse_attention, rf_v2 pipeline; vllm-omni "RainFusion Attention",
 // intro).  A CTA (one per SM, persistent) runs one unit at a time, but its
 // key tiles run in three chains: tile j of a unit has its scores S in
-// tensor-memory buffer j % 3 and its softmax done by warp set j % 3, so
-// three softmaxes and the MMAs of the other tiles overlap.  All three add
+// tensor-memory buffer j % 3, and three warp sets share the softmaxes (fp8:
+// set j % 3 takes tile j; 16-bit: two sets take a tile's two halves of 64
+// keys at once), so softmaxes and the MMAs of the other tiles overlap.  All three add
 // into one O, so they share one running maximum: the row maximum of the
 // unit's first tile (log2 units), published through shared memory.  P is
 // 2^(s c - m) with that m throughout the unit (no per-tile maximum, no
 // rescale); a tile whose sum of P passes the headroom of the P type (2^64
 // for bf16, 65504 for fp16) marks its rows, and the whole unit is handed to
 // the second pass (attn_kernel in list mode, which rescales as it goes)
-// instead of being written.  Each set keeps the sum l of its own tiles; the
-// set of the unit's last tile adds the three sums in a fixed order and
-// writes O / l to the caller's layout.  Which set takes which tile depends
-// on the tile's place in its unit only, so results do not depend on which
+// instead of being written.  Each set keeps the sum l of its own tasks; the
+// set of the unit's last task adds the three sums in a fixed order and
+// writes O / l to the caller's layout.  Which set takes which task depends
+// on the task's place in its unit only, so results do not depend on which
 // CTA ran the unit.
 //
 // Warps (512 threads):
 //   0-11  softmax sets 0, 1, 2 (four warps each, thread = query row = TMEM
-//         lane); the set of a unit's last tile also writes the unit's output.
+//         lane); the set of a unit's last task also writes the unit's output.
 //   12    TMA producer of Q and K (one thread): takes units from the global
 //         counter and publishes them to the other roles through a queue.
 //   13    TMA producer of V (one thread).
 //   14    P V issuer (one elected lane): O += P V of each tile once P is
 //         written.
 //   15    S issuer: S = Q K^T of each tile once the P V of the buffer's
-//         previous tile is done (P lives in the first 64 columns of S);
-//         owns the tensor memory.
+//         previous tile is done (P lives in the S columns); owns the tensor
+//         memory.
 // Shared memory: Q (32 KB), rings of three K and three V tiles (96 KB each),
 // 128-byte swizzled boxes of 128 rows x 128 bytes; K of the CTA's tile g
 // loads once the S of tile g - 3 is done, V once the P V of tile g - 3 is.
 // Tensor memory (512 columns): S_c at [128 c, 128 c + 128) for c = 0, 1, 2,
-// O at [384, 512).
+// O at [384, 512).  P of a tile's keys 64 h .. 64 h + 63 overwrites S
+// columns already read: 16-bit, the first 32 of those keys' own columns
+// (from 128 c + 64 h); e4m3, 16 columns from 128 c + 16 h.
 #include <cstring>
 
 #include "rf_attn_common.cuh"
@@ -56,6 +59,15 @@ struct ChainShape {
   static constexpr int kVRing = C::kFp8 ? 4 : 3;
 };
 constexpr int kItemQ = 8;                     // depth of the unit queue
+// Softmax tasks per key tile after a unit's first: 16-bit tiles are split
+// into two halves of 64 keys done by two sets at once, fp8 tiles are not.
+template <class C>
+constexpr int kTaskSplit = C::kFp8 ? 1 : 2;
+// Column of P of a tile's keys 64..127 within its buffer.  Split tiles keep
+// each half's P inside the half's own S columns, so the two sets never touch
+// each other's scores; whole tiles pack P into the first columns.
+template <class C>
+constexpr uint32_t kPHalfCol = kTaskSplit<C> == 2 ? 64u : (C::kFp8 ? 16u : 32u);
 constexpr uint32_t kCTmemCols = 512;
 constexpr int kWarpKProd = 12, kWarpVProd = 13, kWarpPV = 14, kWarpQK = 15;
 constexpr int kItemReaders = 3 + 4 * kSets;   // V producer, the two MMA warps, softmax warps
@@ -70,7 +82,7 @@ struct __align__(1024) ChainSmem {
   uint64_t k_full[CS::kKRing], k_empty[CS::kKRing], v_full[CS::kVRing], v_empty[CS::kVRing];
   uint64_t s_full[kSets];     // S of the set's next tile is in TMEM (MMA commit; fp8: and the S warp's
                               // arrival once the tile's factors are in ts)
-  uint64_t p_full[kSets];     // the set wrote P of its tile (one arrival per warp)
+  uint64_t p_full[kSets];     // P of the buffer's tile written (one arrival per warp and task)
   uint64_t pv_done[kSets];    // P V of the set's tile done (MMA commit)
   uint64_t o_full;            // the last P V of a unit done (MMA commit)
   uint64_t o_free;            // the unit's output has been read out of O (4 warps)
@@ -342,7 +354,7 @@ __device__ void pv_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem) {
         break;
       }
       tc_fence_after();
-      issue_pv<C>(o_tmem, tmem + 128 * c, v_lo0 + vs * (C::kTileBytes >> 4), hi, j > 0);
+      issue_pv<C>(o_tmem, tmem + 128 * c, v_lo0 + vs * (C::kTileBytes >> 4), hi, j > 0, kPHalfCol<C>);
       mma_commit_elect(&sm.pv_done[c]);
       mma_commit_elect(&sm.v_empty[vs]);
       if (j == itm.ntiles - 1) mma_commit_elect(&sm.o_full);
@@ -370,45 +382,60 @@ __device__ __forceinline__ float tile_max(uint32_t tS, int p_valid) {
   return mx;
 }
 
-// P = 2^(s c + off) of the row's 128 scores, in two halves of 64; P of half
-// h goes to columns [32 h, 32 h + 32) (16-bit, two per column) or
-// [16 h, 16 h + 16) (e4m3, four per column), which are already read.
-// Returns the sum of P.
+// P = 2^(s c + off) of half h (keys 64 h .. 64 h + 63) of a tile's row.  P
+// goes to the 32 (16-bit, two per column) or 16 (e4m3, four per column)
+// columns from kPHalfCol h of the tile's buffer, which are read already.
+// Returns the half's sum of P; the caller waits for the store.
+template <class C>
+__device__ __forceinline__ float half_softmax(uint32_t tS, int h, int p_valid, float c, float off) {
+  uint32_t s[2][32];
+  load_scores<2>(tS + 64 * h, p_valid - 64 * h, s);
+  float sum;
+  if constexpr (C::kFp8) {
+    uint32_t pk[16];
+    sum = exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
+    tmem_st16(tS + kPHalfCol<C> * h, pk);
+  } else {
+    uint32_t pk[32];
+    sum = exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
+    tmem_st32(tS + kPHalfCol<C> * h, pk);
+  }
+  return sum;
+}
+// Both halves of a tile's row, one after the other.  Returns the sum of P.
 template <class C>
 __device__ __forceinline__ float tile_softmax(uint32_t tS, int p_valid, float c, float off) {
   float tsum = 0.f;
 #pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    uint32_t s[2][32];
-    load_scores<2>(tS + 64 * h, p_valid - 64 * h, s);
-    if constexpr (C::kFp8) {
-      uint32_t pk[16];
-      tsum += exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
-      tmem_st16(tS + 16 * h, pk);
-    } else {
-      uint32_t pk[32];
-      tsum += exp_scores<C, 2>(s, c, off, p_valid - 64 * h, pk);
-      tmem_st32(tS + 32 * h, pk);
-    }
-  }
+  for (int h = 0; h < 2; ++h) tsum += half_softmax<C>(tS, h, p_valid, c, off);
   tmem_wait_st();
   return tsum;
 }
 
-// Set `set` (warps 4 set .. 4 set + 3): for every unit, its share of the
-// tiles (tile j of a unit whose first tile is the CTA's tile g0 when
-// (g0 + j) % 3 == set), the row sum of those tiles, and the output when the
-// unit's last tile is the set's.  The set's four warps meet at a named
-// barrier once per unit and carry any failed wait to it, so they leave
-// together.
+// Set `set` (warps 4 set .. 4 set + 3).  Tile j of a unit has its scores in
+// buffer j % 3.  Set 0 takes the unit's first tile whole: its row maximum
+// becomes the unit's, published through shared memory, then its P.  16-bit:
+// every later tile is two tasks, its halves of 64 keys, so that two sets work
+// on one tile at once and a tile's P is ready sooner (the tile's chain of
+// S, softmax, P V and the next S into its buffer is what paces the kernel);
+// task t = 2 (j - 1) + h goes to set (t + 1) % 3.  fp8, whose softmax costs
+// more issue slots per key, gains nothing from the shorter chain and loses
+// the second rendezvous: every later tile is one task, t = j - 1, so tile j
+// goes to set j % 3.  Each set takes its tasks in order.  A set keeps the sum l of its tasks' P; the
+// set of the unit's last task adds the three sums in a fixed order and
+// writes the output.  Which set takes which task depends on the task's
+// place in its unit only, so results do not depend on which CTA ran a unit.
+// The set's four warps meet at a named barrier once per task and carry any
+// failed wait to it, so they leave together.
 template <class C>
 __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, int set) {
   const int quad = (threadIdx.x >> 5) & 3;
   const int row = quad * 32 + (threadIdx.x & 31);   // query row == TMEM lane
   const uint32_t lanes = (uint32_t)(quad * 32) << 16;
-  const uint32_t tS = tmem + 128 * set + lanes, tO = tmem + 384 + lanes;
+  const uint32_t tO = tmem + 384 + lanes;
   const float limit = sum_limit<C>(p);
-  uint32_t mine = 0;   // tiles this set has taken (completions of s_full / p_full)
+  uint32_t base0 = 0, base1 = 0, base2 = 0;   // split tiles: tiles of the CTA's earlier units in each buffer
+  uint32_t mine = 0;                          // whole tiles: tiles this set has taken
   bool ok = true;
   for (uint32_t u = 0;; ++u) {
     const uint32_t qi = u % kItemQ;
@@ -421,14 +448,14 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
     ok = set_and(set, ok);
     if (!ok || itm.bn < 0) break;
     const int n = itm.ntiles;
-    const int owner = 0;                          // set of the unit's first tile
-    const int last = (n - 1) % kSets;             // set of the unit's last tile
+    const int tasks = kTaskSplit<C> * (n - 1);    // tasks after the first tile
+    const int last = n == 1 ? 0 : tasks % kSets;  // set of the unit's last task
     float m_use = 0.f, l = 0.f;
     bool row_bad = false;
     // The tile's factors: 16-bit, S c with c = scale log2(e); fp8, the S
     // warp's TileScale of the buffer (published with s_full).
-    auto factors = [&]() -> TileScale {
-      if (C::kFp8) return sm.ts[set];
+    auto factors = [&](int c) -> TileScale {
+      if (C::kFp8) return sm.ts[c];
       TileScale f;
       f.c = p.scale_log2;
       f.lr = 0.f;
@@ -437,35 +464,54 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
       return f;
     };
     auto p_valid_of = [&](int j) { return j == itm.partial ? p.p_rem_k : RF_BLOCK; };
-    // S of the set's next tile: the set's first warp waits on the barrier,
-    // the other three at the set's named barrier, where they take no issue
-    // slots; every warp reaches it, carrying the outcome.
-    auto wait_s = [&]() {
+    // S of tile j: the set's first warp waits on the buffer's barrier (the
+    // tile is the buffer's (base + j / 3)-th), the other three at the set's
+    // named barrier, where they take no issue slots; every warp reaches it,
+    // carrying the outcome.
+    // (Whole tiles: a set only ever takes tiles of its own buffer, and its
+    // count of them gives the phase.)
+    auto buf_of = [&](int j) { return kTaskSplit<C> == 1 ? set : j % kSets; };
+    auto wait_s = [&](int j) {
+      const int c = buf_of(j);
+      uint32_t prev;
+      if (kTaskSplit<C> == 1) {
+        prev = mine++;
+      } else {
+        prev = (c == 0 ? base0 : c == 1 ? base1 : base2) + j / kSets;
+      }
       bool got = ok;
-      if (got && quad == 0) got = waitw(&sm.abort, p, &sm.s_full[set], ph(mine));
+      if (got && quad == 0) got = waitw(&sm.abort, p, &sm.s_full[c], ph(prev));
       ok = set_and(set, got);
     };
-    auto do_tile = [&](int j) {
-      wait_s();
+    auto do_task = [&](int j, int h) {
+      wait_s(j);
       if (ok) {
+        const int c = buf_of(j);
+        const uint32_t tS = tmem + 128 * c + lanes;
         tc_fence_after();
-        const TileScale f = factors();
-        const float ts = tile_softmax<C>(tS, p_valid_of(j), f.c, f.lr - m_use);
-        row_bad |= !(ts <= limit);
-        l += ts * f.ir;
+        const TileScale f = factors(c);
+        float hs;
+        if (kTaskSplit<C> == 2) {
+          hs = half_softmax<C>(tS, h, p_valid_of(j), f.c, f.lr - m_use);
+          tmem_wait_st();
+        } else {
+          hs = tile_softmax<C>(tS, p_valid_of(j), f.c, f.lr - m_use);
+        }
+        row_bad |= !(hs <= limit);
+        l += hs * f.ir;
         tc_fence_before();
-        arrive_w(&sm.p_full[set]);
+        arrive_w(&sm.p_full[c]);
       }
-      ++mine;
     };
-    if (set == owner) {
+    if (set == 0) {
       // the unit's maximum: the row maximum of its first tile
-      wait_s();
+      const uint32_t tS0 = tmem + lanes;
+      wait_s(0);
       TileScale f0{};
       if (ok) {
         tc_fence_after();
-        f0 = factors();
-        m_use = tile_max(tS, p_valid_of(0)) * f0.c;
+        f0 = factors(0);
+        m_use = tile_max(tS0, p_valid_of(0)) * f0.c;
       }
       if (ok && u >= 1) ok = waitw(&sm.abort, p, &sm.m_empty, ph(u - 1));
       if (ok) {
@@ -473,14 +519,14 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
         __threadfence_block();
         arrive_w(&sm.m_full);
         arrive_w(&sm.m_empty);
-        // the first tile's P (its S is still in place)
-        const float ts = tile_softmax<C>(tS, p_valid_of(0), f0.c, f0.lr - m_use);
+        // the first tile's P (its S is still in place); it stands for all
+        // of the tile's tasks' arrivals
+        const float ts = tile_softmax<C>(tS0, p_valid_of(0), f0.c, f0.lr - m_use);
         row_bad |= !(ts <= limit);
         l += ts * f0.ir;
         tc_fence_before();
-        arrive_w(&sm.p_full[set]);
+        for (int a = 0; a < kTaskSplit<C>; ++a) arrive_w(&sm.p_full[0]);
       }
-      ++mine;
     } else {
       if (ok) ok = waitw(&sm.abort, p, &sm.m_full, ph(u));
       if (ok) {
@@ -488,7 +534,11 @@ __device__ void set_loop(ChainSmem<C>& sm, const AttnParams& p, uint32_t tmem, i
         arrive_w(&sm.m_empty);
       }
     }
-    for (int j = (set == owner) ? kSets : set; j < n; j += kSets) do_tile(j);
+    for (int t = (set + kSets - 1) % kSets; t < tasks; t += kSets)
+      do_task(1 + t / kTaskSplit<C>, t % kTaskSplit<C>);
+    base0 += (n + 2) / 3;
+    base1 += (n + 1) / 3;
+    base2 += n / 3;
     // post this set's row sums (NaN marks a row that needs the second pass)
     if (ok && u >= 1) ok = waitw(&sm.abort, p, &sm.l_empty, ph(u - 1));
     if (ok) {
@@ -575,7 +625,7 @@ __global__ void __launch_bounds__(kCThreads, 1)
     }
     for (int i = 0; i < kSets; ++i) {
       mbar_init(&sm.s_full[i], C::kFp8 ? 2 : 1);
-      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.p_full[i], 4 * kTaskSplit<C>);
       mbar_init(&sm.pv_done[i], 1);
     }
     mbar_init(&sm.o_full, 1);

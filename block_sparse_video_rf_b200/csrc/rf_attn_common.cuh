@@ -44,8 +44,8 @@ struct Cfg {
   static constexpr int kSteps = kFp8 ? 4 : 8;            // MMAs per product over 128 (K 32 or 16 each)
   static constexpr int kPCols = kFp8 ? 32 : 64;          // TMEM columns of P
   // exponent pair i runs the polynomial on the FMA pipe when i % kPolyEvery == kPolyEvery - 1
-  // (the rest on MUFU): measured best split for each path
-  static constexpr int kPolyEvery = kFp8 ? 3 : 4;
+  // (the rest on MUFU): measured best split for each path (16-bit, under the power cap)
+  static constexpr int kPolyEvery = kFp8 ? 3 : 8;
   static constexpr uint32_t kIdescQK =
       kFp8 ? make_idesc_e4m3(128, 128, false) : make_idesc_f16kind(128, 128, false, !kF16);
   static constexpr uint32_t kIdescPV =
@@ -260,18 +260,21 @@ __device__ __forceinline__ void issue_qk(uint32_t s_tmem, uint32_t q_lo, uint32_
   }
 }
 // P V: a K step takes the next 8 TMEM columns of P (16 16-bit or 32 8-bit
-// keys).  16-bit V is MN-major: 16 keys are 16 rows of 128 B further.  fp8 V
-// is stored transposed (K-major): 32 keys are 32 B further.
+// keys).  P of keys 64..127 starts `half_col` columns after P of keys 0..63
+// (contiguous when half_col is 8 kSteps / 2).  16-bit V is MN-major: 16 keys
+// are 16 rows of 128 B further.  fp8 V is stored transposed (K-major): 32
+// keys are 32 B further.
 template <class C>
 __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_lo, uint32_t hi,
-                                         bool accumulate) {
+                                         bool accumulate, uint32_t half_col = 8 * (C::kSteps / 2)) {
 #pragma unroll
   for (int kk = 0; kk < C::kSteps; ++kk) {
     const uint32_t acc = (accumulate || kk > 0) ? 1u : 0u;
+    const uint32_t pc = kk < C::kSteps / 2 ? kk * 8 : half_col + (kk - C::kSteps / 2) * 8;
     if (C::kFp8)
-      mma_ts_lo_elect_f8(o_tmem, p_tmem + kk * 8, v_lo + kk * 2, hi, C::kIdescPV, acc);
+      mma_ts_lo_elect_f8(o_tmem, p_tmem + pc, v_lo + kk * 2, hi, C::kIdescPV, acc);
     else
-      mma_ts_lo_elect(o_tmem, p_tmem + kk * 8, v_lo + kk * (2048 >> 4), hi, C::kIdescPV, acc);
+      mma_ts_lo_elect(o_tmem, p_tmem + pc, v_lo + kk * (2048 >> 4), hi, C::kIdescPV, acc);
   }
 }
 
@@ -290,7 +293,8 @@ __device__ __forceinline__ float exp_scores_(const uint32_t (&s)[kQ][32], float 
   const uint64_t c2 = f2_pack(c, c);
   const uint64_t negm = f2_pack(off, off);
   constexpr bool partial = kPartial;
-  uint64_t sum2[4] = {0, 0, 0, 0};
+  uint64_t sum2[4] = {0, 0, 0, 0};  // fp8: four packed partial sums
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // 16-bit: the same eight sums unpacked
   float hold0 = 0.f, hold1 = 0.f;   // fp8: the first pair of a 4-key word
 #pragma unroll
   for (int q4 = 0; q4 < kQ; ++q4)
@@ -324,11 +328,13 @@ __device__ __forceinline__ float exp_scores_(const uint32_t (&s)[kQ][32], float 
       } else {
         const uint32_t wd = pack_half2<C::kF16>(a0, a1);
         pk[i] = wd;
-        float r0, r1;
-        unpack_half2<C::kF16>(wd, r0, r1);
-        sum2[i & 3] = f2_add(sum2[i & 3], f2_pack(r0, r1));
+        add_half2_to<C::kF16>(wd, acc[2 * (i & 3)], acc[2 * (i & 3) + 1]);
       }
     }
+  if (!C::kFp8) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) sum2[k] = f2_pack(acc[2 * k], acc[2 * k + 1]);
+  }
   float s0, s1, s2, s3;
   f2_unpack(f2_add(sum2[0], sum2[1]), s0, s1);
   f2_unpack(f2_add(sum2[2], sum2[3]), s2, s3);

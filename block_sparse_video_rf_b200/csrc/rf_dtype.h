@@ -43,17 +43,19 @@ __device__ __forceinline__ void unpack_half8(const uint4& u, float (&f)[8]) {
   }
 }
 
-// The two 16-bit values of one word (low half first) as fp32.
+// lo += low half of w, hi += high half, each 16-bit value widened exactly to
+// fp32 and the sum rounded to nearest (the sm_100 mixed-precision add, one
+// instruction per value instead of an unpack and an add).
 template <bool kF16>
-__device__ __forceinline__ void unpack_half2(uint32_t w, float& lo, float& hi) {
-  if (kF16) {
-    const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&w));
-    lo = h.x;
-    hi = h.y;
-  } else {
-    lo = __uint_as_float(w << 16);
-    hi = __uint_as_float(w & 0xFFFF0000u);
-  }
+__device__ __forceinline__ void add_half2_to(uint32_t w, float& lo, float& hi) {
+  if (kF16)
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tadd.rn.f32.f16 %0, l, %0;\n\tadd.rn.f32.f16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w));
+  else
+    asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\tadd.rn.f32.bf16 %0, l, %0;\n\tadd.rn.f32.bf16 %1, h, %1;\n\t}"
+        : "+f"(lo), "+f"(hi)
+        : "r"(w));
 }
 
 }  // namespace rf

@@ -90,7 +90,7 @@ def test_redo_list(rfsa):
     # pass takes all of them, and the result is the oracle's whatever the split
     mixed = False
     try:
-        for limit in (4.0, 16.0, 64.0, 256.0, 1024.0):
+        for limit in (4.0, 16.0, 24.0, 32.0, 48.0, 64.0, 256.0, 1024.0):
             rfsa.rf_debug_set_path(0, limit)
             out2, redo2, _ = _call_ws(rfsa, w, q, k, v)
             n = int(redo2[1])
