@@ -52,11 +52,12 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs):
-    """Per-stage times with the HBM-bound stage's algorithmic bytes: K1 reads q, k, v in the caller's layout and
+def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs, ms_k1=None):
+    """Per-stage times with the HBM-bound stages' algorithmic bytes: K1 reads q, k, v in the caller's layout and
     writes the internal copies plus the fp32 block means of q and k, K2 reads the block means and writes the
     mask, kept counts and margins; fp8 adds the quantisation pass (reads the internal copies, writes e4m3 codes
-    and one fp32 scale per 128-row block)."""
+    and one fp32 scale per 128-row block).  ``ms_k1`` (K1 alone, from the library's stage event) splits the
+    prepare stage into K1 and the kernels after it."""
     heads = w.B * w.N
     row = 128 * 2                                          # one token's head vector, bytes
     pooled = 2 * plan.nb * 128 * 4                         # q and k block means, bytes per head
@@ -66,10 +67,19 @@ def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs):
     kq = heads * (3 * plan.S_int * row + 3 * plan.S_int * 128 + 3 * plan.n_tiles * 4) if prec == "fp8" else 0
     moved = k1 + k2 + kq
     gbs = moved / (ms_prepare * 1e-3) / 1e9
-    return {"prepare": {"kernels": "K1 reorder + block means, K2 block scores + top-k" +
-                        (", Kq e4m3 quantisation" if prec == "fp8" else ""),
-                        "ms": ms_prepare, "algorithmic_bytes": moved, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs},
-            "attention": {"kernels": "K3", "ms": ms_attention, "tflops": k3_tflops}}
+    out = {"prepare": {"kernels": "K1 reorder + block means, K2 block scores + top-k" +
+                       (", Kq e4m3 quantisation" if prec == "fp8" else ""),
+                       "ms": ms_prepare, "algorithmic_bytes": moved, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs}}
+    if ms_k1 is not None and 0 < ms_k1 < ms_prepare:
+        g1 = k1 / (ms_k1 * 1e-3) / 1e9
+        rest = ms_prepare - ms_k1
+        g2 = (k2 + kq) / (rest * 1e-3) / 1e9
+        out["permute_pool"] = {"kernels": "K1 reorder + block means", "ms": ms_k1, "algorithmic_bytes": k1,
+                               "gbs": g1, "frac_of_hbm": g1 / hbm_gbs}
+        out["after_permute_pool"] = {"kernels": "K2" + (" + Kq" if prec == "fp8" else ""), "ms": rest,
+                                     "algorithmic_bytes": k2 + kq, "gbs": g2, "frac_of_hbm": g2 / hbm_gbs}
+    out["attention"] = {"kernels": "K3", "ms": ms_attention, "tflops": k3_tflops}
+    return out
 
 
 # The attention kernels' sources, hashed together to tie a traffic capture to the code it measured.
@@ -333,6 +343,7 @@ def main():
     def step(ev=None):
         if ev is not None:
             ev[0].record(stream)
+            rfsa.rf_debug_set_stage_event(ev[3])       # the library records it after K1
         rfsa.rf_prepare(q, k, v, w.layout, w.txt_len, w.latent, sp, ws, precision=prec)
         if ev is not None:
             ev[1].record(stream)
@@ -348,7 +359,9 @@ def main():
         raise RuntimeError(f"device status {status} after warm-up")
     flops = rfsa.kept_block_flops(plan, views["kept"], w.B, w.N, w.D)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e in evs:
+        e[3].record(stream)                            # creates the CUDA event the library records
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist is not None:
         dist.barrier()
@@ -359,9 +372,11 @@ def main():
             step(evs[i])
         t_end.record(stream)
         torch.cuda.synchronize(dev)
+    rfsa.rf_debug_set_stage_event(None)
     if dist is not None:
         dist.barrier()
     ms_total = t_start.elapsed_time(t_end)
+    k1 = [e[0].elapsed_time(e[3]) for e in evs]
     k1k2 = [e[0].elapsed_time(e[1]) for e in evs]
     k3 = [e[1].elapsed_time(e[2]) for e in evs]
     status = rfsa.rf_read_status(ws, w.B, w.N, w.D, plan)
@@ -427,7 +442,8 @@ def main():
             # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
             # handed to it); fp8 adds the quantisation pass
             "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
-            "stages": _stages(w, plan, prec, statistics.mean(k1k2), k3_ms, k3_tflops, peaks["hbm_gbs"]),
+            "stages": _stages(w, plan, prec, statistics.mean(k1k2), k3_ms, k3_tflops, peaks["hbm_gbs"],
+                              statistics.mean(k1)),
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -27,6 +27,7 @@ thread_local std::string g_last_error;
 // Process-wide test controls of the attention kernel (rf_debug_set_wait).
 std::mutex g_debug_mu;
 rf::AttnDebug g_debug;
+cudaEvent_t g_stage_event = nullptr;   // rf_debug_set_stage_event
 
 rf::AttnDebug debug_settings() {
   std::lock_guard<std::mutex> lock(g_debug_mu);
@@ -325,6 +326,12 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
                                           at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
                                           at<float>(ws, L.pooled_k), s);
   if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
+  cudaEvent_t stage_event;
+  {
+    std::lock_guard<std::mutex> lock(g_debug_mu);
+    stage_event = g_stage_event;
+  }
+  if (stage_event && (e = cudaEventRecord(stage_event, s)) != cudaSuccess) return cuda_fail(e, "stage event record");
   e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, gk, at<uint32_t>(ws, L.mask),
                       at<int>(ws, L.kept), at<float>(ws, L.margin), s);
   if (e != cudaSuccess) return cuda_fail(e, "mask launch");
@@ -617,6 +624,12 @@ rf_status_t rf_debug_set_path(int path, float sum_limit) {
   std::lock_guard<std::mutex> lock(g_debug_mu);
   g_debug.path = path;
   g_debug.sum_limit = sum_limit;
+  return ok();
+}
+
+rf_status_t rf_debug_set_stage_event(void* event) {
+  std::lock_guard<std::mutex> lock(g_debug_mu);
+  g_stage_event = static_cast<cudaEvent_t>(event);
   return ok();
 }
 

@@ -31,7 +31,8 @@ PRECISIONS = {"native": 0, "fp8": 1}
 # Every symbol include/rfsa.h declares.
 EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_attention", "rf_sparse_attention_ws",
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
-           "rf_debug_set_wait", "rf_debug_set_path", "rf_read_stats", "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
+           "rf_debug_set_wait", "rf_debug_set_path", "rf_debug_set_stage_event", "rf_read_stats",
+           "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
            "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv"]
 
 
@@ -81,6 +82,7 @@ def _load():
         "rf_block_mask_noalloc": (I, [P, P] + geo + [I, I, F, P, P, P, P]),
         "rf_debug_set_wait": (I, [ctypes.c_longlong, I]),
         "rf_debug_set_path": (I, [I, F]),
+        "rf_debug_set_stage_event": (I, [P]),
         "rf_read_stats": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfStats), P]),
         "rf_last_error_string": (ctypes.c_char_p, []),
         "rf_plan_kv": (I, [I, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan)]),
@@ -296,8 +298,21 @@ def rf_debug_set_wait(wait_limit_ns: int = 0, skip_first_q: int = 0):
 
 
 def rf_debug_set_path(path: int = 0, sum_limit: float = 0.0):
-    """Test control of the 16-bit attention path (see include/rfsa.h)."""
+    """Test control of the attention path (see include/rfsa.h)."""
     _check(LIB.rf_debug_set_path(int(path), float(sum_limit)))
+
+
+def rf_debug_set_stage_event(event=None):
+    """While set, rf_prepare records ``event`` (a torch.cuda.Event that has been
+    recorded once, so that its CUDA event exists) between K1 and the kernels
+    after it; None clears the hook.  The caller keeps the event alive while it
+    is set (see include/rfsa.h)."""
+    handle = None
+    if event is not None:
+        handle = int(event.cuda_event)
+        if not handle:
+            raise ValueError("the event has no CUDA event yet: record it once first")
+    _check(LIB.rf_debug_set_stage_event(ctypes.c_void_p(handle)))
 
 
 def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:

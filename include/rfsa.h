@@ -267,15 +267,26 @@ rf_status_t rf_read_stats(void* workspace, size_t ws_bytes, int B, int N, int D,
  * without any fault; call with (0, 0) to restore normal operation. */
 rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q);
 
-/* Test control of the 16-bit attention path, process-wide, read at each
- * launch.  path 0 (default): the three-chain kernel runs every query tile
- * and hands the tiles whose P left the type's headroom to the two-tile
- * kernel; path 1: the two-tile kernel runs every query tile.  sum_limit > 0
- * replaces the headroom test (a tile sum of P above it hands the tile on;
- * 0 = the type's own: 2^64 for bf16, 65504 for fp16), so a test can send a
- * chosen share of the tiles through the second pass.  Returns RF_ERR_ARG on
- * path outside {0, 1} or sum_limit < 0. */
+/* Test control of the attention path, process-wide, read at each launch.
+ * path 0 (default): the three-chain kernel runs every query tile and hands
+ * the tiles whose P left the type's headroom to the two-tile kernel; path 1:
+ * the two-tile kernel runs every query tile.  sum_limit > 0 replaces the
+ * headroom test (a sum of P above it over one softmax task of the chain
+ * kernel -- a unit's first tile, then half tiles of 64 keys in 16-bit and
+ * whole tiles in fp8 -- hands the query tile on; 0 = the type's own: 2^64
+ * for bf16, 65504 for fp16, 448 for e4m3), so a test can send a chosen share
+ * of the tiles through the second pass.  Returns RF_ERR_ARG on path outside
+ * {0, 1} or sum_limit < 0. */
 rf_status_t rf_debug_set_path(int path, float sum_limit);
+
+/* Measurement hook, process-wide: while `event` is not NULL, rf_prepare /
+ * rf_prepare_ex record it (cudaEventRecord) on their stream between the
+ * reorder + block-mean kernel (K1) and the kernels after it (block scores +
+ * top-k, fp8 quantisation), so a caller's CUDA events around the call can
+ * time K1 alone.  `event` is a cudaEvent_t the caller created and keeps
+ * alive while it is set; NULL clears the hook.  The library never destroys
+ * it.  A failed record is returned by the prepare call as RF_ERR_CUDA. */
+rf_status_t rf_debug_set_stage_event(void* event);
 
 /* Size of the library-owned static scratch array of rf_block_mask_noalloc,
  * per device (32 MiB): enough for B * N * nb <= 32768 block rows of pooled Q and K

@@ -210,3 +210,16 @@ def test_read_stats_validates_before_any_cuda_call(rfsa):
     assert L.rf_read_stats(None, 1 << 30, 1, 2, 128, ctypes.byref(p), ctypes.byref(st), None) == 5   # NULL workspace
     assert L.rf_read_stats(P(0x1000), 16, 1, 2, 128, ctypes.byref(p), ctypes.byref(st), None) == 5   # too small
     assert L.rf_read_stats(P(0x1000), 1 << 30, 1, 2, 64, ctypes.byref(p), ctypes.byref(st), None) == 3  # D != 128
+
+
+def test_stage_event_hook_sets_and_clears_without_cuda(rfsa):
+    # storing or clearing the hook touches no CUDA state; an event that was
+    # never created is refused by the binding
+    rfsa.rf_debug_set_stage_event(None)
+
+    class NoEvent:
+        cuda_event = 0
+
+    with pytest.raises(ValueError):
+        rfsa.rf_debug_set_stage_event(NoEvent())
+    rfsa.rf_debug_set_stage_event(None)
