@@ -7,6 +7,7 @@
 // in [0, 1]; 128-token blocks; fewer than 32 video blocks or no geometry is
 // dense attention).
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -28,6 +29,16 @@ thread_local std::string g_last_error;
 std::mutex g_debug_mu;
 rf::AttnDebug g_debug;
 cudaEvent_t g_stage_event = nullptr;   // rf_debug_set_stage_event
+
+// NVTX range around a stage's launches (host side: it marks when the work
+// is enqueued).  Header-only NVTX: without a tool attached a push or pop is a
+// check of one pointer.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 rf::AttnDebug debug_settings() {
   std::lock_guard<std::mutex> lock(g_debug_mu);
@@ -322,6 +333,7 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
   if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L)) != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  NvtxRange range("rf prepare: K1 reorder + block means, K2 scores + top-k");
   cudaError_t e = rf::launch_permute_pool(q, k, v, dtype, layout, B, S, gk.S, N, g, gk, at<void>(ws, L.q_int),
                                           at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
                                           at<float>(ws, L.pooled_k), s);
@@ -365,6 +377,7 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
   if ((st = rf_workspace_layout_ex(precision, B, N, D, &g, &gk, &L)) != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  NvtxRange range("rf attend: K3 block-sparse attention");
   cudaError_t e = cudaMemsetAsync(at<int>(ws, L.status), 0, sizeof(int), s);
   if (e != cudaSuccess) return cuda_fail(e, "clearing the status word");
   if (precision == RF_PREC_FP8)

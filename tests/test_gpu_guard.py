@@ -1,0 +1,94 @@
+"""Writes outside the caller's buffers.  The workspace and the output are
+placed inside larger device buffers whose guard bytes (1 MiB on each side)
+hold fixed patterns; after calls on ragged geometries, both layouts, every
+precision, keys with their own geometry and the redo path, the guard bytes
+must be unchanged and the output must match the plain call bit for bit."""
+
+import numpy as np
+import pytest
+import torch
+
+pytestmark = pytest.mark.gpu
+
+GUARD = 1 << 20
+LOW, HIGH = 0xA5, 0x5A
+
+
+@pytest.fixture(scope="module")
+def rfsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from block_sparse_video_rf_b200 import rfsa as mod
+    yield mod
+    mod.rf_debug_set_path(0, 0.0)
+
+
+def _guarded(nbytes):
+    buf = torch.empty(nbytes + 2 * GUARD, dtype=torch.uint8, device="cuda")
+    buf[:GUARD].fill_(LOW)
+    buf[GUARD + nbytes:].fill_(HIGH)
+    return buf, buf[GUARD:GUARD + nbytes]
+
+
+def _intact(buf, nbytes):
+    return bool(torch.all(buf[:GUARD] == LOW)) and bool(torch.all(buf[GUARD + nbytes:] == HIGH))
+
+
+CASES = [
+    ("ragged_bsnd", {"txt_len": 37, "latent": (8, 21, 43), "sparsity": 0.7, "seed": 81}, "native", None, 0.0),
+    ("ragged_bnsd", {"txt_len": 19, "latent": (5, 24, 40), "sparsity": 0.6, "layout": "BNSD", "seed": 82},
+     "native", None, 0.0),
+    ("fp16", {"txt_len": 37, "latent": (6, 24, 40), "sparsity": 0.6, "seed": 83, "B": 2}, "native", torch.float16,
+     0.0),
+    ("fp8", {"txt_len": 37, "latent": (8, 21, 43), "sparsity": 0.7, "seed": 84}, "fp8", None, 0.0),
+    ("redo", {"txt_len": 37, "latent": (8, 21, 43), "sparsity": 0.7, "seed": 85}, "native", None, 16.0),
+    ("dense", {"txt_len": 0, "latent": (4, 32, 32), "sparsity": 0.0, "seed": 86}, "native", None, 0.0),
+]
+
+
+@pytest.mark.parametrize("name,over,precision,dtype,limit", CASES, ids=[c[0] for c in CASES])
+def test_guard_bytes_untouched(rfsa, name, over, precision, dtype, limit):
+    from block_sparse_video_rf_b200 import synth
+    w = synth.workload("tiny", **over)
+    q, k, v = synth.make_inputs(w, device="cpu", **({"dtype": dtype} if dtype is not None else {}))
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    sp = np.float32(w.sparsity)
+    n_ws = rfsa.rf_workspace_size(w.B, w.S, w.N, w.D, w.txt_len, w.latent, precision)
+    ws_buf, ws = _guarded(n_ws)
+    n_out = q.numel() * q.element_size()
+    out_buf, out_bytes = _guarded(n_out)
+    out = out_bytes.view(q.dtype).view(q.shape)
+    rfsa.rf_debug_set_path(0, limit)
+    try:
+        rfsa.rf_sparse_attention_ws(q, k, v, w.layout, w.txt_len, w.latent, sp, ws, out=out, precision=precision)
+        torch.cuda.synchronize()
+    finally:
+        rfsa.rf_debug_set_path(0, 0.0)
+    assert _intact(ws_buf, n_ws), "workspace guard bytes changed"
+    assert _intact(out_buf, n_out), "output guard bytes changed"
+    ref = rfsa.rf_sparse_attention(q, k, v, w.layout, w.txt_len, w.latent, sp, precision=precision)
+    torch.cuda.synchronize()
+    if limit == 0.0:
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    else:   # the second pass computes the listed tiles its own way; both are checked against the oracle elsewhere
+        assert torch.isfinite(out.float()).all()
+
+
+def test_guard_bytes_key_geometry(rfsa):
+    from block_sparse_video_rf_b200 import synth
+    w = synth.workload("tiny", txt_len=37, latent=(8, 21, 43), sparsity=0.7, seed=87)
+    q, k, v = synth.make_inputs(w, device="cpu")
+    kv_latent = (4, 21, 43)
+    S_kv = w.txt_len + kv_latent[0] * kv_latent[1] * kv_latent[2]
+    kk = k[:, :S_kv].contiguous().cuda()
+    vv = v[:, :S_kv].contiguous().cuda()
+    q = q.cuda()
+    sp = np.float32(w.sparsity)
+    n_ws = rfsa.rf_workspace_size(w.B, w.S, w.N, w.D, w.txt_len, w.latent, "native", S_kv, kv_latent)
+    ws_buf, ws = _guarded(n_ws)
+    n_out = q.numel() * q.element_size()
+    out_buf, out_bytes = _guarded(n_out)
+    out = out_bytes.view(q.dtype).view(q.shape)
+    rfsa.rf_sparse_attention_ws(q, kk, vv, w.layout, w.txt_len, w.latent, sp, ws, out=out, latent_k=kv_latent)
+    torch.cuda.synchronize()
+    assert _intact(ws_buf, n_ws) and _intact(out_buf, n_out)
