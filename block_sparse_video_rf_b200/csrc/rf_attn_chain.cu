@@ -416,15 +416,16 @@ __device__ __forceinline__ float tile_softmax(uint32_t tS, int p_valid, float c,
 // buffer j % 3.  Set 0 takes the unit's first tile whole: its row maximum
 // becomes the unit's, published through shared memory, then its P.  16-bit:
 // every later tile is two tasks, its halves of 64 keys, so that two sets work
-// on one tile at once and a tile's P is ready sooner (the tile's chain of
-// S, softmax, P V and the next S into its buffer is what paces the kernel);
-// task t = 2 (j - 1) + h goes to set (t + 1) % 3.  fp8, whose softmax costs
-// more issue slots per key, gains nothing from the shorter chain and loses
-// the second rendezvous: every later tile is one task, t = j - 1, so tile j
-// goes to set j % 3.  Each set takes its tasks in order.  A set keeps the
-// sum l of its tasks' P; the set of the unit's last task adds the three sums
-// in a fixed order and writes the output.  Which set takes which task depends on the task's
-// place in its unit only, so results do not depend on which CTA ran a unit.
+// on one tile at once and a tile's P is ready sooner, which shortens the
+// chain of S, softmax, P V and the next S into the tile's buffer; task
+// t = 2 (j - 1) + h goes to set (t + 1) % 3.  fp8, whose softmax costs more
+// issue slots per key, gains nothing from the shorter chain and loses the
+// second rendezvous: every later tile is one task, t = j - 1, so tile j goes
+// to set j % 3.  Each set takes its tasks in order.  A set keeps the sum l
+// of its tasks' P; the set of the unit's last task adds the three sums in a
+// fixed order and writes the output.  Which set takes which task depends on
+// the task's place in its unit only, so results do not depend on which CTA
+// ran a unit.
 // The set's four warps meet at a named barrier once per task and carry any
 // failed wait to it, so they leave together.
 template <class C>
