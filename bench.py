@@ -82,6 +82,18 @@ def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs, ms_k1=N
     return out
 
 
+def _kv_stream(flops, prec, ms_attention, sm_mhz, sms):
+    """K and V brought from L2 into the SMs by K3: each (query row, kept key) pair costs 4 bytes (a 128 x 128
+    tile pair of 64 KB serves 128 x 128 pairs; e4m3: 2 bytes) and 4 D = 512 FLOPs.  Per SM cycle at the median
+    SM clock sampled in the timed region, against the ~50 bytes per SM cycle a streaming probe reached."""
+    pairs = flops / (4 * 128)
+    nbytes = pairs * (2 if prec == "fp8" else 4)
+    out = {"bytes": nbytes, "tbs": nbytes / (ms_attention * 1e-3) / 1e12}
+    if sm_mhz:
+        out["bytes_per_sm_cycle"] = nbytes / (ms_attention * 1e-3 * sms * sm_mhz * 1e6)
+    return out
+
+
 # The attention kernels' sources, hashed together to tie a traffic capture to the code it measured.
 K3_SOURCES = ("rf_attn_common.cuh", "rf_attn_chain.cu", "rf_attn.cu")
 
@@ -446,6 +458,8 @@ def main():
                               statistics.mean(k1)),
             "clocks": clocks.summary(),
         }
+        line["stages"]["attention"]["kv_stream"] = _kv_stream(flops, prec, k3_ms, line["clocks"].get("sm_mhz"),
+                                                              torch.cuda.get_device_properties(dev).multi_processor_count)
         if world == 1 and not args.no_cpu_baseline:
             val, threads, desc = oracle_sample(q, k, v, w)
             line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}

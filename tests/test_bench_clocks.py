@@ -48,3 +48,13 @@ def test_no_reasons(monkeypatch):
         time.sleep(0.1)
     s = c.summary()
     assert s["reasons"] == [] and s["sm_mhz"] == 1965
+
+
+def test_kv_stream_bytes_per_pair():
+    import bench
+    flops = 512.0 * 1e9                      # 1e9 (row, key) pairs at 4 D = 512 FLOPs each
+    bf = bench._kv_stream(flops, "native", 10.0, 1500.0, 148)
+    assert bf["bytes"] == 4e9 and abs(bf["tbs"] - 0.4) < 1e-12
+    assert abs(bf["bytes_per_sm_cycle"] - 4e9 / (10e-3 * 148 * 1.5e9)) < 1e-9
+    f8 = bench._kv_stream(flops, "fp8", 10.0, None, 148)
+    assert f8["bytes"] == 2e9 and "bytes_per_sm_cycle" not in f8
