@@ -223,3 +223,14 @@ def test_stage_event_hook_sets_and_clears_without_cuda(rfsa):
     with pytest.raises(ValueError):
         rfsa.rf_debug_set_stage_event(NoEvent())
     rfsa.rf_debug_set_stage_event(None)
+
+
+@pytest.mark.parametrize("B,S,N", [(0, 4096, 2), (1, 4096, 0), (1, 0, 2), (-1, 4096, 2), (1, -5, 2)])
+def test_empty_or_negative_sizes_are_argument_errors(rfsa, B, S, N):
+    # nothing to compute is refused up front, before any CUDA call
+    L = rfsa.LIB
+    P = ctypes.c_void_p
+    fake = P(0x1000)
+    st = L.rf_sparse_attention(fake, fake, fake, 0, B, S, N, 128, 0, 4, 32, 32, 128, 0.5, 0.0, P(0x2000), None)
+    assert st == 2, st
+    assert L.rf_last_error_string()
