@@ -252,3 +252,16 @@ def test_sparsity_one_keeps_prefix_and_first_frame(rfsa):
     ref, mask, _, g = oracle.rf_sparse_attention(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent, 1.0)
     assert (mask[0, :, g.ff:].sum(-1) == g.ff).all()
     assert_close(to_np(out), ref, "s=1")
+
+
+@pytest.mark.parametrize("S", [1, 2, 127, 129])
+def test_tiny_sequences_without_video_geometry(rfsa, S):
+    # one query tile with 1..127 valid rows, or a second tile holding one row: a unit of one or two key tiles,
+    # the rest of the tile masked
+    g = torch.Generator().manual_seed(100 + S)
+    q, k, v = (torch.randn((1, S, 3, 128), generator=g).to(torch.bfloat16).cuda() for _ in range(3))
+    out = rfsa.rf_sparse_attention(q, k, v, "BSND", 0, (0, 0, 0), 0.5)
+    torch.cuda.synchronize()
+    qb, kb, vb = (to_bnsd_np(t, "BSND") for t in (q, k, v))
+    for n in range(3):
+        assert_close(to_bnsd_np(out, "BSND")[0, n], oracle.dense_attention(qb[0, n], kb[0, n], vb[0, n], 128 ** -0.5))
