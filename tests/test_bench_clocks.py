@@ -58,3 +58,23 @@ def test_kv_stream_bytes_per_pair():
     assert abs(bf["bytes_per_sm_cycle"] - 4e9 / (10e-3 * 148 * 1.5e9)) < 1e-9
     f8 = bench._kv_stream(flops, "fp8", 10.0, None, 148)
     assert f8["bytes"] == 2e9 and "bytes_per_sm_cycle" not in f8
+
+
+def test_reference_arm_line_on_cpu():
+    # the reference arm (the oracle on the host cores) prints one JSON line with the contract's keys
+    import json
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "0",
+                        "--ref-budget", "0.3"], cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads(r.stdout.strip().splitlines()[-1])
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] == 0
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["unit"] == "TFLOP/s"
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["e2e"]["d2h_bytes_per_step"] == 0
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["config"]["workload"].startswith("minimax")
