@@ -18,9 +18,11 @@ CUDA library takes the same one; the two share no code):
       e4m3_value(code) * scale.  The block mask is computed from the
       unquantised inputs, exactly as at native precision.
   R15 The fp8 attention output is the oracle's attention (fp64) over the
-      dequantised Q, K and V.  The tensor-core path also rounds P to e4m3
-      before P V; that rounding is not modelled here and is covered by the
-      fp8 tolerance of the tests.
+      dequantised Q, K and V.  An fp8 tensor-core path must also round the
+      softmax weights P to e4m3 before P V; the oracle does not apply that
+      rounding, but ``p_rounding_model`` states what it can change: per
+      output element a worst-case bound and an error scale, both computed
+      from the oracle's own weights (see there for the derivation).
 
 The e4m3 format (OCP 8-bit floating point, E4M3): 1 sign bit, 4 exponent
 bits with bias 7, 3 mantissa bits; exponent field 0 holds subnormals
@@ -29,7 +31,10 @@ finite value is 1.75 * 2^8 = 448.
 
 Parity: the value table and the rounding are pinned against torch's
 float8_e4m3fn conversion and against a brute-force nearest-value search in
-``tests/test_oracle_fp8.py``.
+``tests/test_oracle_fp8.py``; the quantised attention equals the plain
+oracle exactly on operands that e4m3 represents exactly; the error model of
+the P rounding is checked against an explicit e4m3 rounding of P on random
+rows (flat, peaked, and with the reference maximum far below the row's).
 """
 
 from __future__ import annotations
@@ -160,3 +165,115 @@ def rf_sparse_attention_fp8(q, k, v, layout: str, txt_len: int, latent, sparsity
             kd, vd = (quantize_head(x[b, n], gkv, dense)[0] for x in (kb, vb))
             out[b, n] = rf_v2.attention_rows(qd, kd, vd, g, None if dense else mask[b, n], scale, gk=gk)
     return rf_v2.from_bnsd(out, layout), mask, margin, (g if gk is None else (g, gk))
+
+
+# ---------------------------------------------------------------------------
+# The rounding of P to e4m3 (R15): what it can change in the output
+# ---------------------------------------------------------------------------
+
+P_REL = 2.0 ** -4        # e4m3 normals: 3 mantissa bits, round to nearest -> |p~ - p| <= 2^-4 p
+P_MIN_NORMAL = 2.0 ** -6  # below it the spacing is 2^-9 ...
+P_ABS = 2.0 ** -10       # ... so |p~ - p| <= min(p, 2^-10) (values under 2^-10 round to 0)
+ARITH_REL = 2.0 ** -9    # room for the fp32 scores and sums and the approximate exponentials
+OUT_REL = 2.0 ** -8      # the 16-bit output's own rounding (bf16: at most 2^-9 |o|), with room
+
+
+def token_scales(g: rf_v2.Geometry, scales: np.ndarray, dense: bool | None = None) -> np.ndarray:
+    """[S] the block scale of each token's internal tile (``scales`` as
+    returned by ``quantize_head`` for the same geometry)."""
+    out = np.zeros(g.S, dtype=np.float64)
+    for t, rows in enumerate(internal_tiles(g, dense)):
+        valid = rows >= 0
+        out[rows[valid]] = float(scales[t])
+    return out
+
+
+def p_rounding_model(e: np.ndarray, v: np.ndarray, sv_tok: np.ndarray, vmax: float):
+    """Output rows and the error the e4m3 rounding of P may add to them.
+
+    ``e`` [R, K]: exp(scale q.k - M) of each row over its key set, with M the
+    row's largest scaled score (the oracle's own softmax numerators, fp64);
+    ``v`` [K, D]: the dequantised values of those keys; ``sv_tok`` [K]: the
+    block scale of each key's V tile; ``vmax``: the head's largest V block
+    scale.  Returns (o, bound, sigma), each [R, D].
+
+    Derivation.  Let w_j = e_j / L_M with L_M = sum_j e_j, so o = sum_j w_j v_j.
+    An fp8 path takes a reference maximum of its choosing, m <= M (a
+    maximum over part of the row is at most the row's), writes the weights
+    as P'_j = 2^D e_j sv_j / vmax with D = M - m >= 0 (so that P' times V's
+    own codes, v_j = sv_j code_j, carries the one factor vmax), keeps them
+    at most 448 (so none saturates), rounds them to e4m3 (RNE), P~'_j =
+    P'_j + d_j, and divides by the sum of the unrounded weights, L = 2^D L_M.
+    The output is then o + sum_j d_j (vmax / sv_j) v_j / L, and
+      * if e_j sv_j / vmax >= 2^-6, P'_j is a normal e4m3 value whatever D
+        is, |d_j| <= 2^-4 P'_j, and the key's term is at most 2^-4 w_j |v_j|;
+      * otherwise P'_j may lie in the subnormal range, where
+        |d_j| <= min(P'_j, 2^-10) (or 2^-4 P'_j if it is normal after all);
+        dividing by L = 2^D L_M, the term is at most
+        max(2^-4 w_j, min(w_j, 2^-10 vmax / (sv_j L_M))) |v_j| for every D >= 0.
+    With c_j those coefficients, the worst case is sum_j c_j |v_j|.  The
+    approximate exponentials and the fp32 scores and sums change P'_j and
+    L together by relative amounts far below 2^-9, which moves o by at most
+    2^-9 sum_j w_j |v_j - o| <= 2^-9 (sum_j w_j |v_j| + |o|); the 16-bit
+    output adds at most 2^-9 |o| (bf16), taken as 2^-8 |o|.
+    The rounding errors of different keys are independent and (up to the
+    truncation of the smallest values to 0) of zero mean; the term of key j
+    lies in [-c_j |v_j|, c_j |v_j|], whose uniform distribution has variance
+    (c_j v_j)^2 / 3, and RNE's error is no wider.  The error of an element
+    therefore has a standard deviation of at most
+    sigma = sqrt(sum_j (c_j v_j)^2 / 3 + (2^-9 o)^2 / 3), the second term
+    for the output's rounding.
+    """
+    e = np.asarray(e, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    sv = np.asarray(sv_tok, dtype=np.float64)
+    L = e.sum(axis=1, keepdims=True)
+    w = e / L
+    o = w @ v
+    av = np.abs(v)
+    c = P_REL * w
+    if vmax > 0:
+        ratio = np.where(sv > 0, sv / vmax, 0.0)                  # sv_j / vmax in [0, 1]
+        sub = e * ratio[None, :] < P_MIN_NORMAL                    # may be subnormal for some reference
+        with np.errstate(divide="ignore"):
+            cap = np.where(ratio > 0, P_ABS / np.where(ratio > 0, ratio, 1.0), np.inf)[None, :] / L
+        c = np.where(sub, np.maximum(c, np.minimum(w, cap)), c)
+    wav = w @ av
+    bound = (c @ av) * (1.0 + 2.0 ** -6) + ARITH_REL * (wav + np.abs(o)) + OUT_REL * np.abs(o) + 2.0 ** -24
+    sigma = np.sqrt(((c * c) @ (v * v)) / 3.0 + (2.0 ** -9 * o) ** 2 / 3.0 + (2.0 ** -24) ** 2)
+    return o, bound, sigma
+
+
+def attention_rows_fp8(qd, kd, vd, sv_tok, vmax: float, g: rf_v2.Geometry, mask_bn, scale: float, rows=None,
+                       chunk: int = 128, gk: rf_v2.Geometry | None = None):
+    """R15 for one (b, head): the attention of ``rows`` (default all) over
+    the dequantised operands, as ``rf_v2.attention_rows`` computes it, with
+    the per-element bound and error scale of ``p_rounding_model``.
+
+    ``sv_tok`` [S_kv]: the V block scale of each key token (``token_scales``);
+    ``vmax``: the head's largest V block scale.  Returns (o, bound, sigma),
+    each [len(rows), D] in fp64.
+    """
+    q64, k64, v64 = (np.asarray(a, dtype=np.float64) for a in (qd, kd, vd))
+    S, D = q64.shape
+    rows = np.arange(S) if rows is None else np.asarray(rows, dtype=np.int64)
+    out = np.empty((len(rows), D))
+    bound = np.empty((len(rows), D))
+    sigma = np.empty((len(rows), D))
+    dense = rf_v2.is_dense(g, gk)
+    block_of = np.full(S, -1, dtype=np.int64)
+    if not dense:
+        block_of[g.blocks.ravel()] = np.repeat(np.arange(g.nb), rf_v2.BLOCK)
+    groups: dict[int, list[int]] = {}
+    for pos, r in enumerate(rows):
+        groups.setdefault(int(block_of[r]), []).append(pos)
+    for blk, positions in groups.items():
+        keys = rf_v2.key_set(g, mask_bn, None if blk < 0 else blk, gk)
+        kk, vv, sv = k64[keys], v64[keys], np.asarray(sv_tok, dtype=np.float64)[keys]
+        positions = np.asarray(positions)
+        for c0 in range(0, len(positions), chunk):
+            p = positions[c0:c0 + chunk]
+            s = (q64[rows[p]] @ kk.T) * scale
+            e = np.exp(s - s.max(axis=1, keepdims=True))
+            out[p], bound[p], sigma[p] = p_rounding_model(e, vv, sv, vmax)
+    return out, bound, sigma

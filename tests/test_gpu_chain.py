@@ -121,15 +121,15 @@ def test_scores_beyond_headroom(rfsa, dtype, gain):
 
 
 def _fp8_check(w, q, k, v, out, what):
-    from oracle import fp8
-    from parity_util import assert_close_fp8, to_bnsd_np
-    ref, _, _, g = fp8.rf_sparse_attention_fp8(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent,
-                                               float(np.float32(w.sparsity)))
-    ob, rb, vb = to_bnsd_np(out, w.layout), oracle.to_bnsd(ref, w.layout), to_bnsd_np(v, w.layout)
+    from parity_util import assert_close_fp8, fp8_reference, to_bnsd_np
+    qb, kb, vb = (to_bnsd_np(t, w.layout) for t in (q, k, v))
+    g = oracle.geometry(w.S, w.txt_len, *w.latent)
+    mask, _ = oracle.build_mask(qb, kb, g, float(np.float32(w.sparsity)))
+    ob = to_bnsd_np(out, w.layout)
     for b in range(w.B):
         for n in range(w.N):
-            vd = fp8.quantize_head(vb[b, n], g)[0]
-            assert_close_fp8(ob[b, n], rb[b, n], vd, f"{what} b{b} n{n}")
+            ref, bound, sigma = fp8_reference(qb[b, n], kb[b, n], vb[b, n], g, mask[b, n], w.D ** -0.5)
+            assert_close_fp8(ob[b, n], ref, bound, sigma, f"{what} b{b} n{n}")
 
 
 @pytest.mark.parametrize("case", ["tiny", "ragged", "batch2", "one_tile_units"])

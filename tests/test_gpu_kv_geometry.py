@@ -10,7 +10,8 @@ import torch
 
 import oracle
 from oracle import fp8
-from parity_util import assert_close, assert_close_fp8, mask_mismatch, pack_mask, to_bnsd_np, to_np
+from parity_util import (assert_close, assert_close_fp8, fp8_reference, mask_mismatch, pack_mask, to_bnsd_np,
+                         to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -77,10 +78,9 @@ def test_mask_and_attention(rfsa, case, precision):
     got = to_bnsd_np(out, w.layout).astype(np.float64)
     for n in range(w.N):
         if precision == "fp8":
-            qd = fp8.quantize_head(qb[0, n], gq, dense)[0]
-            kd, vd = (fp8.quantize_head(x[0, n], gk, dense)[0] for x in (kb, vb))
-            ref = oracle.attention_rows(qd, kd, vd, gq, None if dense else mask[0, n], w.D ** -0.5, gk=gk)
-            assert_close_fp8(got[0, n], ref, vd, f"{case} fp8 n{n}")
+            ref, bound, sigma = fp8_reference(qb[0, n], kb[0, n], vb[0, n], gq, None if dense else mask[0, n],
+                                              w.D ** -0.5, gk=gk, dense=dense)
+            assert_close_fp8(got[0, n], ref, bound, sigma, f"{case} fp8 n{n}")
         else:
             ref = oracle.attention_rows(qb[0, n], kb[0, n], vb[0, n], gq, None if dense else mask[0, n],
                                         w.D ** -0.5, gk=gk)

@@ -202,8 +202,7 @@ def test_running_max_that_grows_after_the_first_tile(rfsa, precision):
     # The text prefix tile comes first and holds small scores; the video keys are
     # scaled up, so later tiles exceed the first tile's maximum by far and the
     # kernel must raise its running max (and rescale O and l) mid-row.
-    from oracle import fp8
-    from parity_util import assert_close_fp8
+    from parity_util import assert_close_fp8, fp8_reference
     w, q, k, v = _inputs("tiny", txt_len=128, latent=(4, 32, 32), N=2, seed=31)
     k = k.clone()
     k[:, w.txt_len:] *= 6.0
@@ -215,13 +214,12 @@ def test_running_max_that_grows_after_the_first_tile(rfsa, precision):
                                                   float(np.float32(w.sparsity)))
         assert_close(to_np(out), ref, "growing max")
     else:
-        ref, _, _, g = fp8.rf_sparse_attention_fp8(to_np(q), to_np(k), to_np(v), w.layout, w.txt_len, w.latent,
-                                                   float(np.float32(w.sparsity)))
-        vb = to_bnsd_np(v, w.layout)
+        qb, kb, vb = (to_bnsd_np(t, w.layout) for t in (q, k, v))
+        g = oracle.geometry(w.S, w.txt_len, *w.latent)
+        mask, _ = oracle.build_mask(qb, kb, g, float(np.float32(w.sparsity)))
         for n in range(w.N):
-            vd = fp8.quantize_head(vb[0, n], g)[0]
-            assert_close_fp8(to_bnsd_np(out, w.layout)[0, n], oracle.to_bnsd(ref, w.layout)[0, n], vd,
-                             f"growing max fp8 n{n}")
+            ref, bound, sigma = fp8_reference(qb[0, n], kb[0, n], vb[0, n], g, mask[0, n], w.D ** -0.5)
+            assert_close_fp8(to_bnsd_np(out, w.layout)[0, n], ref, bound, sigma, f"growing max fp8 n{n}")
 
 
 @pytest.mark.parametrize("layout", ["BSND", "BNSD"])
