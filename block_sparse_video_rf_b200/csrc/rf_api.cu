@@ -78,6 +78,13 @@ rf_status_t check_common(rf_layout_t layout, int B, int S, int N, int D) {
   return RF_OK;
 }
 
+// The kernels read and write 16-byte vectors of a token's head vector, so
+// every tensor must start on a 16-byte boundary (rows are 256 bytes long).
+rf_status_t check_aligned16(const void* p, const char* name) {
+  if (reinterpret_cast<uintptr_t>(p) & 15) return fail(RF_ERR_ARG, "%s is not 16-byte aligned", name);
+  return RF_OK;
+}
+
 rf_status_t check_types(rf_dtype_t dtype, rf_precision_t precision) {
   if (dtype != RF_BF16 && dtype != RF_F16) return fail(RF_ERR_ARG, "dtype must be RF_BF16 (0) or RF_F16 (1)");
   if (precision != RF_PREC_NATIVE && precision != RF_PREC_FP8)
@@ -326,6 +333,9 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
   if (st != RF_OK) return st;
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!q || !k || !v) return fail(RF_ERR_ARG, "q, k and v must be device pointers");
+  if ((st = check_aligned16(q, "q")) != RF_OK || (st = check_aligned16(k, "k")) != RF_OK ||
+      (st = check_aligned16(v, "v")) != RF_OK)
+    return st;
   rf_plan_t g, gk;
   if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
     return st;
@@ -370,6 +380,7 @@ rf_status_t rf_attend_ex(rf_dtype_t dtype, rf_precision_t precision, rf_layout_t
   if (st != RF_OK) return st;
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!out) return fail(RF_ERR_ARG, "out must be a device pointer");
+  if ((st = check_aligned16(out, "out")) != RF_OK) return st;
   rf_plan_t g, gk;
   if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
     return st;
@@ -410,6 +421,9 @@ rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, 
   if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!q || !k || !v || !out) return fail(RF_ERR_ARG, "q, k, v and out must be device pointers");
   if (out == q || out == k || out == v) return fail(RF_ERR_ARG, "out must not alias q, k or v");
+  if ((st = check_aligned16(q, "q")) != RF_OK || (st = check_aligned16(k, "k")) != RF_OK ||
+      (st = check_aligned16(v, "v")) != RF_OK || (st = check_aligned16(out, "out")) != RF_OK)
+    return st;
   if (!ws) {
     rf_plan_t g, gk;
     if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
@@ -446,6 +460,7 @@ rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, in
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
   if (!o_int || !out) return fail(RF_ERR_ARG, "o_int and out must be device pointers");
+  if ((st = check_aligned16(o_int, "o_int")) != RF_OK || (st = check_aligned16(out, "out")) != RF_OK) return st;
   rf_plan_t g;
   if ((st = rf_plan(S, txt_len, T, H, W, RF_BLOCK, 0.f, &g)) != RF_OK) return st;
   cudaError_t e = rf::launch_unpermute(o_int, layout, B, S, N, g, out, static_cast<cudaStream_t>(stream));
@@ -555,11 +570,13 @@ rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const
   return ok();
 }
 
-rf_status_t rf_read_stats(void* ws, size_t ws_bytes, int B, int N, int D, const rf_plan_t* g, rf_stats_t* stats,
-                          void* stream) {
+rf_status_t rf_read_stats_ex(rf_precision_t precision, void* ws, size_t ws_bytes, int B, int N, int D,
+                             const rf_plan_t* g, const rf_plan_t* gk, rf_stats_t* stats, void* stream) {
   if (!stats) return fail(RF_ERR_ARG, "stats pointer is NULL");
+  if (!g) return fail(RF_ERR_ARG, "plan pointer is NULL");
+  if (!gk) gk = g;
   rf_ws_layout_t L;
-  rf_status_t st = rf_workspace_layout(B, N, D, g, &L);
+  rf_status_t st = rf_workspace_layout_ex(precision, B, N, D, g, gk, &L);
   if (st != RF_OK) return st;
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   const size_t heads = (size_t)B * N, rows = heads * g->nb;
@@ -578,27 +595,34 @@ rf_status_t rf_read_stats(void* ws, size_t ws_bytes, int B, int N, int D, const 
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e, "reading the workspace statistics");
   rf_stats_t r{};
-  const double S = g->S;
+  const double S = g->S, S_kv = gk->S;
   if (g->dense) {
-    r.kept_pairs = (double)heads * S * S;
+    r.kept_pairs = (double)heads * S * S_kv;
   } else {
+    // dense query rows (prefix, first-frame blocks) read every key; a sparse
+    // block's rows read the key prefix and 128 keys per kept key block
     const double dense_rows = (double)g->P + 128.0 * g->ff;
     double sparse_keys = 0;
     for (size_t h = 0; h < heads; ++h)
       for (int i = g->ff; i < g->nb; ++i) {
         const size_t j = h * g->nb + i;
         r.kept_blocks += kept[j];
-        sparse_keys += 128.0 * kept[j] + g->P;
+        sparse_keys += 128.0 * kept[j] + gk->P;
         if (margin[j] < 1e-5f) ++r.near_ties;
       }
     r.query_blocks = (long long)heads * (g->nb - g->ff);
-    r.kept_pairs = (double)heads * dense_rows * S + 128.0 * sparse_keys;
+    r.kept_pairs = (double)heads * dense_rows * S_kv + 128.0 * sparse_keys;
   }
-  r.density = r.kept_pairs / ((double)heads * S * S);
+  r.density = r.kept_pairs / ((double)heads * S * S_kv);
   r.redo_tiles = redo[1] < 0 ? (int)(heads * g->n_tiles) : redo[1];
   r.status = status;
   *stats = r;
   return ok();
+}
+
+rf_status_t rf_read_stats(void* ws, size_t ws_bytes, int B, int N, int D, const rf_plan_t* g, rf_stats_t* stats,
+                          void* stream) {
+  return rf_read_stats_ex(RF_PREC_NATIVE, ws, ws_bytes, B, N, D, g, nullptr, stats, stream);
 }
 
 rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layout, int B, int S, int N, int D,
@@ -607,10 +631,13 @@ rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layo
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
   if (!q || !k) return fail(RF_ERR_ARG, "q and k must be device pointers");
+  if ((st = check_aligned16(q, "q")) != RF_OK || (st = check_aligned16(k, "k")) != RF_OK) return st;
   rf_plan_t g;
   if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
   if (g.nb == 0) return ok();
   if (!mask || !kept || !margin) return fail(RF_ERR_ARG, "mask, kept and margin must be device pointers");
+  if ((reinterpret_cast<uintptr_t>(mask) | reinterpret_cast<uintptr_t>(kept) | reinterpret_cast<uintptr_t>(margin)) & 3)
+    return fail(RF_ERR_ARG, "mask, kept and margin must be 4-byte aligned");
   const size_t need = (size_t)B * N * g.nb * RF_HEAD_DIM * sizeof(float) * 2;
   if (need > RF_NOALLOC_SCRATCH_BYTES)
     return fail(RF_ERR_UNSUPPORTED,
@@ -643,6 +670,16 @@ rf_status_t rf_debug_set_path(int path, float sum_limit) {
 rf_status_t rf_debug_set_stage_event(void* event) {
   std::lock_guard<std::mutex> lock(g_debug_mu);
   g_stage_event = static_cast<cudaEvent_t>(event);
+  return ok();
+}
+
+rf_status_t rf_debug_exp2_poly(const float* x, float* y, int n, void* stream) {
+  if (n < 0) return fail(RF_ERR_ARG, "n must be >= 0");
+  if (n > 0 && (!x || !y)) return fail(RF_ERR_ARG, "x and y must be device pointers");
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 3)
+    return fail(RF_ERR_ARG, "x and y must be 4-byte aligned");
+  cudaError_t e = rf::launch_debug_exp2_poly(x, y, n, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "exp2 polynomial launch");
   return ok();
 }
 

@@ -80,4 +80,8 @@ cudaError_t launch_block_mask_noalloc(const void* q, const void* k, int dtype, i
                                       const rf_plan_t& g, uint32_t* mask, int* kept, float* margin,
                                       cudaStream_t stream);
 
+// Debug: the attention's FMA-pipe exponential (exp2_poly_x2) on n fp32
+// values, y[i] = 2^x[i] as the softmax computes it.
+cudaError_t launch_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
+
 }  // namespace rf

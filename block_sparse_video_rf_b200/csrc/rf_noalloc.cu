@@ -16,6 +16,7 @@
 // must be ordered by the caller.  Each call overwrites every element it later
 // reads, so nothing has to start at zero and the previous call's contents do
 // not matter.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -73,10 +74,45 @@ __global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const uint16_t* _
   *dst = s * (1.0f / RF_BLOCK);
 }
 
-// Device address of the static scratch array, resolved once per device.
+// Device address of the static scratch array, resolved once per device and
+// CUDA context: a device reset, or a primary context released and made
+// again, loads the module anew and may move the array, so the address is
+// looked up again whenever the current context is not the one it was taken in.
 constexpr int kMaxDevices = 64;
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* ptr;
+};
 std::mutex g_addr_mu;
-void* g_addr[kMaxDevices] = {};
+ScratchAddr g_addr[kMaxDevices] = {};
+
+// Id of the current context (false when there is none yet).  The driver's
+// functions are reached through the runtime's entry-point query, so the
+// library does not link against the driver library and still loads where
+// there is none.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+bool current_ctx_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess || !a)
+      return false;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess || !b)
+      return false;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
+  }
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
 
 }  // namespace
 
@@ -86,15 +122,21 @@ cudaError_t noalloc_scratch(void** ptr) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_addr_mu);
-  if (!g_addr[dev]) {
-    // In host code g_noalloc_scratch names a host-side stand-in; the kernel
-    // needs the device address of this device's copy.
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_addr[dev] = p;
+  unsigned long long id = 0;
+  if (g_addr[dev].ptr && current_ctx_id(&id) && id == g_addr[dev].ctx_id) {
+    *ptr = g_addr[dev].ptr;
+    return cudaSuccess;
   }
-  *ptr = g_addr[dev];
+  // In host code g_noalloc_scratch names a host-side stand-in; the kernel
+  // needs the device address of this device's copy.  The lookup also makes
+  // the device's primary context current if no context was.
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return e;
+  if (!current_ctx_id(&id)) return cudaErrorDeviceUninitialized;
+  g_addr[dev].ctx_id = id;
+  g_addr[dev].ptr = p;
+  *ptr = p;
   return cudaSuccess;
 }
 

@@ -33,7 +33,8 @@ EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_att
            "rf_prepare", "rf_attend", "rf_unpermute", "rf_sparse_attention_host", "rf_read_status",
            "rf_debug_set_wait", "rf_debug_set_path", "rf_debug_set_stage_event", "rf_read_stats",
            "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
-           "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv"]
+           "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv",
+           "rf_read_stats_ex", "rf_debug_exp2_poly"]
 
 
 class RfPlan(ctypes.Structure):
@@ -84,6 +85,9 @@ def _load():
         "rf_debug_set_path": (I, [I, F]),
         "rf_debug_set_stage_event": (I, [P]),
         "rf_read_stats": (I, [P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfStats), P]),
+        "rf_read_stats_ex": (I, [I, P, Z, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan),
+                                 ctypes.POINTER(RfStats), P]),
+        "rf_debug_exp2_poly": (I, [P, P, I, P]),
         "rf_last_error_string": (ctypes.c_char_p, []),
         "rf_plan_kv": (I, [I, I, I, I, I, I, I, I, I, I, F, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan)]),
         "rf_workspace_layout_ex": (I, [I, I, I, I, ctypes.POINTER(RfPlan), ctypes.POINTER(RfPlan),
@@ -116,6 +120,37 @@ def _dims(x, layout: str):
     else:
         raise RfError(1, "input layout must be BSND or BNSD")
     return B, S, N, D
+
+
+def _check_tensors(layout: str, q, k=None, v=None, out=None, same_kv_len: bool = True):
+    """Checks, before any call into the library, what the C ABI cannot see
+    from bare pointers: every tensor is a contiguous torch tensor of bf16 or
+    fp16 (all of one type) on one CUDA device; k and v have one shape, with
+    q's batch, heads and head dim (and q's length unless k and v have a
+    geometry of their own); out has q's shape.  Raises RfError(RF_ERR_ARG)."""
+    dims = _dims(q, layout)
+    tensors = [("q", q), ("k", k), ("v", v), ("out", out)]
+    tensors = [(n, t) for n, t in tensors if t is not None]
+    for name, t in tensors:
+        if t.dim() != 4:
+            raise RfError(2, f"{name} must have 4 dims ({layout}), got {tuple(t.shape)}")
+        if t.dtype != q.dtype:
+            raise RfError(2, f"{name} is {t.dtype}, q is {q.dtype}")
+    _dtype(q)
+    if k is not None and v is not None and k.shape != v.shape:
+        raise RfError(2, f"k {tuple(k.shape)} and v {tuple(v.shape)} differ in shape")
+    if k is not None:
+        kd = _dims(k, layout)
+        if (kd[0], kd[2], kd[3]) != (dims[0], dims[2], dims[3]) or (same_kv_len and kd[1] != dims[1]):
+            raise RfError(2, f"k {tuple(k.shape)} does not match q {tuple(q.shape)} ({layout})")
+    if out is not None and out.shape != q.shape:
+        raise RfError(2, f"out {tuple(out.shape)} must have q's shape {tuple(q.shape)}")
+    for name, t in tensors:
+        if not t.is_contiguous():
+            raise RfError(2, f"{name} must be contiguous")
+    for name, t in tensors:
+        if not t.is_cuda or t.device != q.device:
+            raise RfError(2, f"{name} must be a CUDA tensor on q's device ({q.device}), got {t.device}")
 
 
 def _stream(x, stream):
@@ -206,6 +241,7 @@ def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: fl
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
+    _check_tensors(layout, q, k, v, out, same_kv_len=latent_k is None)
     lay = LAYOUTS.get(layout, -1)
     if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_sparse_attention(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
@@ -223,6 +259,7 @@ def rf_sparse_attention_ws(q, k, v, layout, txt_len, latent, sparsity, workspace
     B, S, N, D = _dims(q, layout)
     if out is None:
         out = torch.empty_like(q)
+    _check_tensors(layout, q, k, v, out, same_kv_len=latent_k is None)
     lay = LAYOUTS.get(layout, -1)
     if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_sparse_attention_ws(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
@@ -239,6 +276,7 @@ def rf_sparse_attention_ws(q, k, v, layout, txt_len, latent, sparsity, workspace
 def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size=128, stream=None,
                precision: str = "native", latent_k=None):
     B, S, N, D = _dims(q, layout)
+    _check_tensors(layout, q, k, v, same_kv_len=latent_k is None)
     lay = LAYOUTS.get(layout, -1)
     if _plain(q, precision) and latent_k is None:
         _check(LIB.rf_prepare(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent, block_size,
@@ -252,6 +290,7 @@ def rf_prepare(q, k, v, layout, txt_len, latent, sparsity, workspace, block_size
 def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, block_size=128, stream=None,
               precision: str = "native", S_kv: int = 0, latent_k=None):
     B, S, N, D = _dims(out, layout)
+    _check_tensors(layout, out)
     lay = LAYOUTS.get(layout, -1)
     kv = (S_kv, *latent_k) if latent_k is not None else (0, 0, 0, 0)
     if _plain(out, precision) and latent_k is None:
@@ -266,6 +305,9 @@ def rf_attend(out, layout, txt_len, latent, sparsity, workspace, scale=None, blo
 
 def rf_unpermute(o_int, out, layout, txt_len, latent, stream=None):
     B, S, N, D = _dims(out, layout)
+    _check_tensors(layout, out)
+    if o_int.dtype != out.dtype or not o_int.is_contiguous() or not o_int.is_cuda:
+        raise RfError(2, "o_int must be a contiguous CUDA tensor of out's type")
     _check(LIB.rf_unpermute(_ptr(o_int), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent, _ptr(out),
                             _stream(out, stream)))
     return out
@@ -287,6 +329,7 @@ def rf_block_mask_noalloc(q, k, layout, txt_len, latent, sparsity, mask, kept, m
                           stream=None):
     """Block mask into caller buffers, with no device allocation (see include/rfsa.h)."""
     B, S, N, D = _dims(q, layout)
+    _check_tensors(layout, q, k)
     _check(LIB.rf_block_mask_noalloc(_ptr(q), _ptr(k), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
                                      block_size, float(sparsity), _ptr(mask), _ptr(kept), _ptr(margin),
                                      _stream(q, stream)))
@@ -322,12 +365,31 @@ def rf_read_status(workspace, B, N, D, plan, stream=None) -> int:
     return st.value
 
 
-def rf_read_stats(workspace, B, N, D, plan, stream=None) -> dict:
+def rf_read_stats(workspace, B, N, D, plan, stream=None, precision: str = "native", plan_kv=None) -> dict:
     """Statistics of the last call on a workspace (see include/rfsa.h)."""
     st = RfStats()
-    _check(LIB.rf_read_stats(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
-                             ctypes.byref(plan), ctypes.byref(st), _stream(workspace, stream)))
+    if precision == "native" and plan_kv is None:
+        _check(LIB.rf_read_stats(_ptr(workspace), workspace.numel() * workspace.element_size(), B, N, D,
+                                 ctypes.byref(plan), ctypes.byref(st), _stream(workspace, stream)))
+    else:
+        _check(LIB.rf_read_stats_ex(_prec(precision), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    B, N, D, ctypes.byref(plan), ctypes.byref(plan_kv) if plan_kv is not None else None,
+                                    ctypes.byref(st), _stream(workspace, stream)))
     return st.as_dict()
+
+
+def rf_debug_exp2_poly(x, y=None, stream=None):
+    """y = 2^x by the attention's FMA-pipe exponential (see include/rfsa.h);
+    x, y: contiguous fp32 CUDA tensors of one size."""
+    import torch
+    if y is None:
+        y = torch.empty_like(x)
+    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel():
+        raise RfError(2, "x and y must be fp32 tensors of one size")
+    if not (x.is_contiguous() and y.is_contiguous() and x.is_cuda and y.is_cuda):
+        raise RfError(2, "x and y must be contiguous CUDA tensors")
+    _check(LIB.rf_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(x, stream)))
+    return y
 
 
 def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native", plan_kv=None):

@@ -8,11 +8,21 @@
  * with the geometry and dense-fallback rules of the vllm-omni user guide
  * page "RainFusion Attention" (intro; "Configuration"; "Geometry handling").
  *
+ * Each declaration below names the passage that defines it: [SA] is
+ * MindSpore Lite "lite_boost.ops.sparse_attention" (its pipeline line, its
+ * parameter list, "Returns" and "Raises"); [RF] is the vllm-omni user guide
+ * page "RainFusion Attention" (intro, "Configuration", "Requirements and
+ * compatibility", "Geometry handling").  Entry points marked "library"
+ * have no counterpart on the pages: they expose the stages, buffers and
+ * test controls of this implementation.
+ *
  * Conventions for every entry point:
  *  - q, k, v, out: DEVICE pointers to bf16 (fp16 through the _ex entry
- *    points with dtype RF_F16), caller-owned, contiguous, in the layout
- *    given (RF_BSND = [B, S, N, D], RF_BNSD = [B, N, S, D]); out has the
- *    shape, layout and element type of q and must not alias q, k or v.
+ *    points with dtype RF_F16), caller-owned, contiguous, 16-byte aligned
+ *    (the kernels move 16-byte vectors; a misaligned pointer is RF_ERR_ARG),
+ *    in the layout given (RF_BSND = [B, S, N, D], RF_BNSD = [B, N, S, D]);
+ *    out has the shape, layout and element type of q and must not alias q,
+ *    k or v.
  *  - D and block_size must be 128.
  *  - S = txt_len + latent_t * latent_h * latent_w.  latent (0, 0, 0) means
  *    "no video geometry": the call is dense softmax attention over S.
@@ -39,13 +49,16 @@
 extern "C" {
 #endif
 
+/* [SA] parameter input_layout: "BSND" or "BNSD". */
 typedef enum { RF_BSND = 0, RF_BNSD = 1 } rf_layout_t;
 
-/* Element type of q, k, v and out (lite_boost.ops.sparse_attention accepts
- * float16 and bfloat16). */
+/* Element type of q, k, v and out.  [SA] intro: input tensors may be
+ * float16 or bfloat16. */
 typedef enum { RF_BF16 = 0, RF_F16 = 1 } rf_dtype_t;
 
-/* Arithmetic of the attention's two products.  RF_PREC_NATIVE: Q K^T and P V
+/* Arithmetic of the attention's two products.  [RF] "Configuration",
+ * precision "bf16" (the default) or "fp8" (the "mix" mode is not offered).
+ * RF_PREC_NATIVE: Q K^T and P V
  * on the tensor cores in the input type (bf16 or fp16) with fp32
  * accumulation.  RF_PREC_FP8: Q, K and V quantised to fp8 e4m3 with one
  * fp32 scale per 128-row block of the internal layout (per tensor and head:
@@ -56,21 +69,31 @@ typedef enum { RF_BF16 = 0, RF_F16 = 1 } rf_dtype_t;
  * both: it is computed from the unquantised inputs. */
 typedef enum { RF_PREC_NATIVE = 0, RF_PREC_FP8 = 1 } rf_precision_t;
 
+/* Return codes.  RF_ERR_LAYOUT is [SA] "Raises" (ValueError on input_layout);
+ * the sparsity range is [SA] parameter sparsity and [RF] "Configuration";
+ * the others are library codes. */
 typedef enum {
   RF_OK = 0,
   RF_ERR_LAYOUT = 1,      /* layout not BSND/BNSD (the page's ValueError on input_layout) */
-  RF_ERR_ARG = 2,         /* bad sizes, sparsity outside [0, 1], S != txt_len + t*h*w, NULL pointer */
+  RF_ERR_ARG = 2,         /* bad sizes, sparsity outside [0, 1], S != txt_len + t*h*w, NULL or misaligned pointer */
   RF_ERR_UNSUPPORTED = 3, /* D != 128, block_size != 128, or more sparse blocks than RF_MAX_BLOCKS */
   RF_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
   RF_ERR_WORKSPACE = 5,   /* workspace too small or misaligned */
   RF_ERR_TIMEOUT = 6      /* a device-side wait ran past its limit (read via rf_read_status) */
 } rf_status_t;
 
+/* [SA] parameter block_size (default 128; the only size supported here) and
+ * the head dim of every workload on the pages (MiniMax-H3: 56 heads x 128). */
 #define RF_HEAD_DIM 128
 #define RF_BLOCK 128
+/* Library limit on sparse blocks per clip (524,288 aligned video tokens). */
 #define RF_MAX_BLOCKS 4096
 
-/* Geometry of one clip, shared by every (batch, head).
+/* Geometry of one clip, shared by every (batch, head).  [RF] "Geometry
+ * handling" (8x8-aligned spatial arrangement, the promoted suffix, the
+ * 62,496 / 2,976 / 465 x 128 worked example) and intro (128-token blocks,
+ * (t, h, w) order, first-frame blocks dense, fewer than 32 blocks dense);
+ * [SA] parameters txt_len and latent_shape_q.
  * Internal row order per (b, head): [prefix: text, promoted video tokens in
  * natural (t, h, w) order, aligned tokens past the last whole block]
  * [zero pad to a multiple of 128] [nb sparse blocks of 128 rows, each two
@@ -91,7 +114,7 @@ typedef struct {
   int mask_words;    /* 32-bit words per mask row = ceil(nb / 32) */
 } rf_plan_t;
 
-/* Byte offsets of the regions of a workspace (all 256-byte aligned).
+/* Library: byte offsets of the regions of a workspace (all 256-byte aligned).
  * q_int/k_int/v_int: 16-bit (input type) [B, N, S_int, 128]; pooled_q/pooled_k: fp32
  * [B, N, nb, 128] (block means); mask: uint32 [B, N, nb, mask_words], bit j
  * of row i set when query block i reads key block j; kept: int32 [B, N, nb]
@@ -115,7 +138,8 @@ typedef struct {
   size_t total;
 } rf_ws_layout_t;
 
-/* Statistics of the last call on a workspace (rf_read_stats). */
+/* Library: statistics of the last call on a workspace (rf_read_stats).  The
+ * near-tie count is the one the mask's bit-exact check excuses. */
 typedef struct {
   long long kept_blocks;   /* key blocks kept over all sparse query blocks (top-k plus forced first-frame columns) */
   long long query_blocks;  /* sparse query blocks that select (B * N * (nb - ff)) */
@@ -127,24 +151,26 @@ typedef struct {
   int status;              /* the workspace status word (not cleared) */
 } rf_stats_t;
 
-/* Host-only: validate a geometry and fill *plan.  No CUDA call. */
+/* Host-only: validate a geometry and fill *plan.  No CUDA call.  [RF]
+ * "Geometry handling" and intro; [SA] parameters txt_len, block_size,
+ * latent_shape_q, sparsity (k = nb - floor(sparsity * nb + 1e-6)). */
 rf_status_t rf_plan(int S, int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
                     rf_plan_t* plan);
 
 /* Host-only: the plans of a call whose keys and values have a geometry of
- * their own (S_kv, kv_t, kv_h, kv_w as in rf_prepare_ex; S_kv <= 0: the
+ * their own ([SA] parameter latent_shape_k, which defaults to latent_shape_q) (S_kv, kv_t, kv_h, kv_w as in rf_prepare_ex; S_kv <= 0: the
  * query's, and *plan_kv = *plan).  If either geometry is dense both plans
  * come back dense (the whole sequence as the prefix, in its own order). */
 rf_status_t rf_plan_kv(int S, int txt_len, int latent_t, int latent_h, int latent_w, int S_kv, int kv_t, int kv_h,
                        int kv_w, int block_size, float sparsity, rf_plan_t* plan, rf_plan_t* plan_kv);
 
-/* Host-only: workspace regions for B x N heads of head dim D under `plan`. */
+/* Library, host-only: workspace regions for B x N heads of head dim D under `plan`. */
 rf_status_t rf_workspace_layout(int B, int N, int D, const rf_plan_t* plan, rf_ws_layout_t* layout);
 
-/* Host-only: bytes of workspace rf_sparse_attention_ws needs (0 on bad arguments). */
+/* Library, host-only: bytes of workspace rf_sparse_attention_ws needs (0 on bad arguments). */
 size_t rf_workspace_size(int B, int S, int N, int D, int txt_len, int latent_t, int latent_h, int latent_w);
 
-/* Host-only: the same for a given precision (RF_PREC_FP8 adds the e4m3
+/* Library, host-only: the same for a given precision (RF_PREC_FP8 adds the e4m3
  * tensors and scales) and a key/value geometry of its own (plan_kv NULL, or
  * S_kv <= 0: the query's; see rf_prepare_ex). */
 rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D, const rf_plan_t* plan,
@@ -152,7 +178,12 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
 size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D, int txt_len, int latent_t,
                             int latent_h, int latent_w, int S_kv, int kv_t, int kv_h, int kv_w);
 
-/* The whole rf_v2 call, with a workspace cached by the library per device
+/* The whole rf_v2 call: [SA] sparse_type "rf_v2" (token reorder -> block
+ * pooling -> top-k sparse mask -> rain_fusion_attention -> inverse
+ * reorder), its parameters scale (NaN or <= 0: head_dim ** -0.5), head_num
+ * (N), input_layout, txt_len, block_size, latent_shape_q, sparsity, and
+ * "Returns" (out shaped like q); the dense fallbacks of [RF] intro.  Here
+ * with a workspace cached by the library per device
  * (grown with cudaMalloc on first use of a larger shape; never shrunk).  The
  * cached buffers are shared by rf_sparse_attention, rf_sparse_attention_ex
  * (NULL workspace) and rf_sparse_attention_host on a device: calls from
@@ -162,7 +193,7 @@ rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_
                                 int D, int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
                                 float sparsity, float scale, void* out, void* stream);
 
-/* The whole call with a caller-owned device workspace of ws_bytes
+/* Library: the whole call (as rf_sparse_attention) with a caller-owned device workspace of ws_bytes
  * (>= rf_workspace_size, 256-byte aligned).  Calls that share a workspace
  * must be ordered on one stream. */
 rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
@@ -170,14 +201,17 @@ rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, 
                                    int block_size, float sparsity, float scale, void* out, void* workspace,
                                    size_t ws_bytes, void* stream);
 
-/* Stage 1 (token reorder + block pooling, then block scores + top-k mask):
+/* Stage 1, [SA] pipeline steps one to three (token reorder + block pooling,
+ * then block scores + top-k mask), with [RF] intro's forced first-frame
+ * blocks:
  * fills q_int/k_int/v_int, pooled_q/pooled_k, mask, kept and margin of the
  * workspace. */
 rf_status_t rf_prepare(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N, int D,
                        int txt_len, int latent_t, int latent_h, int latent_w, int block_size, float sparsity,
                        void* workspace, size_t ws_bytes, void* stream);
 
-/* Stage 2 (rain_fusion_attention + inverse reorder): attention of every
+/* Stage 2, [SA] pipeline steps four and five (rain_fusion_attention +
+ * inverse reorder): attention of every
  * query over its key set as given by the workspace mask, written to out in
  * the caller's token order and layout.  The mask region may be overwritten
  * between the stages (e.g. to run under another mask). */
@@ -185,8 +219,9 @@ rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_le
                       int latent_w, int block_size, float sparsity, float scale, void* out, void* workspace,
                       size_t ws_bytes, void* stream);
 
-/* rf_prepare / rf_attend / rf_sparse_attention_ws for any input type,
- * precision and key/value geometry (the plain entry points are these with
+/* rf_prepare / rf_attend / rf_sparse_attention_ws for any input type ([SA]
+ * intro: float16 and bfloat16), precision ([RF] "Configuration": precision)
+ * and key/value geometry ([SA] latent_shape_k) (the plain entry points are these with
  * RF_BF16, RF_PREC_NATIVE and S_kv = 0).
  * - Key/value geometry (lite_boost.ops.sparse_attention, latent_shape_k):
  *   S_kv <= 0 means k and v have q's length and geometry (kv_* ignored).
@@ -219,12 +254,14 @@ rf_status_t rf_sparse_attention_ex(const void* q, const void* k, const void* v, 
                                    int kv_h, int kv_w, int block_size, float sparsity, float scale, void* out,
                                    void* workspace, size_t ws_bytes, void* stream);
 
-/* Inverse reorder alone: o_int [B, N, S_int, 128] of 16-bit values (internal
+/* [SA] pipeline, last step, alone (the inverse reorder, which the attention
+ * otherwise fuses into its epilogue): o_int [B, N, S_int, 128] of 16-bit values (internal
  * order) -> out in the caller's layout.  Pad rows are skipped. */
 rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, int N, int D, int txt_len,
                          int latent_t, int latent_h, int latent_w, void* out, void* stream);
 
-/* End-to-end through HOST buffers (bf16, caller layout): copies q, k, v to
+/* Library: the whole call (as rf_sparse_attention) end-to-end through HOST
+ * buffers (bf16, caller layout): copies q, k, v to
  * the device, runs the call, copies the result back to out_host and
  * synchronises.  The heads are independent, so the call runs on chunks of
  * heads (about 96 MiB of q, k and v each, and at least two heads in BSND) in
@@ -239,7 +276,7 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
                                      int latent_w, int block_size, float sparsity, float scale, void* out_host,
                                      void* stream);
 
-/* Synchronises `stream`, reads the workspace status word into *status
+/* Library: synchronises `stream`, reads the workspace status word into *status
  * (0 = fine, otherwise an rf_status_t code recorded by a kernel) and clears
  * it.  The status word sits at the same place in every workspace (any
  * precision or key geometry); the plan only validates the arguments.
@@ -247,17 +284,26 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
 rf_status_t rf_read_status(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                            int* status, void* stream);
 
-/* Synchronises `stream` and reads *stats from a workspace after rf_prepare +
+/* Library: synchronises `stream` and reads *stats from a workspace after rf_prepare +
  * rf_attend (or rf_sparse_attention_ws) with keys in the query's geometry
  * and native precision: the kept counts and k-th-score margins of the mask,
  * the redo list and the status word (copied, not cleared).  The debug view of
  * a call: how much of the sequence it kept, how many selections sat on a
- * near-tie (R7), how many tiles took the second pass.
+ * near-tie (k-th and (k+1)-th block scores within 1e-5, relative), how
+ * many tiles took the second pass.
  * Returns RF_OK, RF_ERR_ARG, RF_ERR_WORKSPACE or RF_ERR_CUDA. */
 rf_status_t rf_read_stats(void* workspace, size_t ws_bytes, int B, int N, int D, const rf_plan_t* plan,
                           rf_stats_t* stats, void* stream);
+/* Library: the same after a call of any precision and key/value geometry
+ * (rf_prepare_ex + rf_attend_ex, or rf_sparse_attention_ex with a
+ * workspace): plan and plan_kv as rf_plan_kv gives them (plan_kv NULL: the
+ * query's).  kept_pairs and density then count the key sequence's length:
+ * dense rows read all of S_kv keys, a sparse block's rows the key prefix and
+ * 128 keys per kept key block. */
+rf_status_t rf_read_stats_ex(rf_precision_t precision, void* workspace, size_t ws_bytes, int B, int N, int D,
+                             const rf_plan_t* plan, const rf_plan_t* plan_kv, rf_stats_t* stats, void* stream);
 
-/* Test control of the device-side waits of the attention kernel, process-wide,
+/* Library test control of the device-side waits of the attention kernel, process-wide,
  * read at each launch.  wait_limit_ns: limit of every wait (0 = the default,
  * 2 s).  skip_first_q = 1: every CTA's first query tile never gets its Q
  * copy, so the first wait on it runs out; the kernel then records
@@ -267,7 +313,7 @@ rf_status_t rf_read_stats(void* workspace, size_t ws_bytes, int B, int N, int D,
  * without any fault; call with (0, 0) to restore normal operation. */
 rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q);
 
-/* Test control of the attention path, process-wide, read at each launch.
+/* Library test control of the attention path, process-wide, read at each launch.
  * path 0 (default): the three-chain kernel runs every query tile and hands
  * the tiles whose P left the type's headroom to the two-tile kernel; path 1:
  * the two-tile kernel runs every query tile.  sum_limit > 0 replaces the
@@ -279,7 +325,7 @@ rf_status_t rf_debug_set_wait(long long wait_limit_ns, int skip_first_q);
  * {0, 1} or sum_limit < 0. */
 rf_status_t rf_debug_set_path(int path, float sum_limit);
 
-/* Measurement hook, process-wide: while `event` is not NULL, rf_prepare /
+/* Library measurement hook, process-wide: while `event` is not NULL, rf_prepare /
  * rf_prepare_ex record it (cudaEventRecord) on their stream between the
  * reorder + block-mean kernel (K1) and the kernels after it (block scores +
  * top-k, fp8 quantisation), so a caller's CUDA events around the call can
@@ -295,7 +341,7 @@ rf_status_t rf_debug_set_stage_event(void* event);
 
 /* Block mask without any device allocation.  The pages have no counterpart:
  * this is a library convenience for callers that cannot allocate device
- * memory themselves.  Examples are a plugin in a process whose device memory
+ * memory themselves.  q and k are bf16 (the only input type it takes).  Examples are a plugin in a process whose device memory
  * belongs entirely to one allocator that forbids side allocations, or a
  * latency-critical loop that cannot afford the implicit synchronisation of
  * cudaMalloc/cudaFree.
@@ -312,7 +358,9 @@ rf_status_t rf_debug_set_stage_event(void* event);
  *   RF_ERR_UNSUPPORTED with a message; a dense plan (nb = 0) writes nothing.
  * - The first call on a device looks up the device address of the array
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is kept per device and CUDA
+ *   context: after a device reset (or a new primary context) the next call
+ *   looks it up again, and that call too should come before any capture.
  * - All calls share the array: calls whose work overlaps on the GPU race
  *   and must be ordered by the caller.  Each call rewrites all the scratch
  *   it reads, so nothing needs clearing between calls. */
@@ -320,7 +368,18 @@ rf_status_t rf_block_mask_noalloc(const void* q, const void* k, rf_layout_t layo
                                   int txt_len, int latent_t, int latent_h, int latent_w, int block_size,
                                   float sparsity, uint32_t* mask, int32_t* kept, float* margin, void* stream);
 
-/* Thread-local text of the last error returned on this thread. */
+/* Library debug kernel: y[i] = 2^x[i] for n fp32 values (device pointers,
+ * 4-byte aligned, may be the same array), computed two at a time by the
+ * exponential the attention's softmax runs on the FMA pipe for a share of
+ * its weights: 2^round(x) by the exponent field times a degree-3 polynomial
+ * for 2^f, |f| <= 1/2 (relative error below 7.5e-5).  x is clamped to
+ * [-125, 128] first, so x < -125 gives about 2^-125, x >= 127.5 at least
+ * 2^127.5 (never a small or negative number: a softmax sum that overflows
+ * stays visible as one), and NaN gives about 2^-125.  Asynchronous on
+ * `stream`.  Returns RF_ERR_ARG for n < 0, NULL or misaligned pointers. */
+rf_status_t rf_debug_exp2_poly(const float* x, float* y, int n, void* stream);
+
+/* Library: thread-local text of the last error returned on this thread. */
 const char* rf_last_error_string(void);
 
 #ifdef __cplusplus

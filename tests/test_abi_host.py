@@ -24,7 +24,7 @@ def rfsa():
 
 def test_exports_match_header(rfsa):
     hdr = open(os.path.join(ROOT, "include", "rfsa.h")).read()
-    declared = set(re.findall(r"^\S[^\n(]*?\b(rf_[a-z_]+)\s*\(", hdr, flags=re.M))
+    declared = set(re.findall(r"^\S[^\n(]*?\b(rf_[a-z0-9_]+)\s*\(", hdr, flags=re.M))
     assert declared == set(rfsa.EXPORTS)
     lib = ctypes.CDLL(rfsa.LIB_PATH)
     for name in declared:
@@ -234,3 +234,70 @@ def test_empty_or_negative_sizes_are_argument_errors(rfsa, B, S, N):
     st = L.rf_sparse_attention(fake, fake, fake, 0, B, S, N, 128, 0, 4, 32, 32, 128, 0.5, 0.0, P(0x2000), None)
     assert st == 2, st
     assert L.rf_last_error_string()
+
+
+def test_misaligned_tensors_are_argument_errors_before_any_cuda_call(rfsa):
+    # the kernels move 16-byte vectors of each 256-byte row: a tensor that
+    # does not start on a 16-byte boundary is refused up front (RF_ERR_ARG),
+    # never launched on
+    L = rfsa.LIB
+    P = ctypes.c_void_p
+    ok, odd = P(0x1000), P(0x1008)
+    geo = (0, 1, 4096, 2, 128, 0, 4, 32, 32, 128, 0.5, 0.0)
+    for args in ((odd, ok, ok, P(0x2000)), (ok, odd, ok, P(0x2000)), (ok, ok, odd, P(0x2000)), (ok, ok, ok, odd)):
+        assert L.rf_sparse_attention(*args[:3], *geo, args[3], None) == 2
+        assert b"16-byte" in L.rf_last_error_string()
+    assert L.rf_prepare(ok, odd, ok, *geo[:-1], P(0x10000), 1 << 40, None) == 2
+    assert L.rf_attend(*geo, odd, P(0x10000), 1 << 40, None) == 2
+    assert L.rf_unpermute(odd, 0, 1, 4096, 2, 128, 0, 4, 32, 32, P(0x2000), None) == 2
+    assert L.rf_block_mask_noalloc(odd, ok, *geo[:-1], ok, ok, ok, None) == 2
+    assert L.rf_block_mask_noalloc(ok, ok, *geo[:-1], P(0x3002), ok, ok, None) == 2     # mask not 4-byte aligned
+    ex = (0, 0, 0, 1, 4096, 2, 128, 0, 4, 32, 32, 0, 0, 0, 0, 128, 0.5, 0.0)
+    assert L.rf_sparse_attention_ex(ok, ok, ok, *ex, odd, None, 0, None) == 2
+
+
+def test_debug_exp2_validates_before_any_cuda_call(rfsa):
+    L = rfsa.LIB
+    P = ctypes.c_void_p
+    assert L.rf_debug_exp2_poly(P(0x1000), P(0x2000), -1, None) == 2
+    assert L.rf_debug_exp2_poly(None, P(0x2000), 4, None) == 2
+    assert L.rf_debug_exp2_poly(P(0x1002), P(0x2000), 4, None) == 2
+
+
+def test_read_stats_ex_validates_before_any_cuda_call(rfsa):
+    L = rfsa.LIB
+    P = ctypes.c_void_p
+    p = rfsa.rf_plan(4096, 0, (4, 32, 32), 0.5)
+    st = rfsa.RfStats()
+    assert L.rf_read_stats_ex(5, P(0x1000), 1 << 30, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 2
+    assert L.rf_read_stats_ex(1, P(0x1000), 16, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 5
+    assert L.rf_read_stats_ex(1, P(0x1000), 1 << 30, 1, 2, 128, None, None, ctypes.byref(st), None) == 2
+    # the fp8 workspace is larger than the native one: a native-sized buffer is too small for it
+    nat = rfsa.rf_workspace_size(1, 4096, 2, 128, 0, (4, 32, 32))
+    assert L.rf_read_stats_ex(1, P(0x1000), nat, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 5
+
+
+def test_binding_checks_tensors_before_the_library(rfsa):
+    # what bare pointers cannot tell the C ABI -- type, shape, contiguity,
+    # device -- is refused by the binding before any call into the library
+    import torch
+    q = torch.zeros(1, 4096, 2, 128, dtype=torch.bfloat16)
+    cases = [
+        (q, q.clone(), q.clone().float()),                           # v of another type
+        (q, q[:, :4000].clone(), q.clone()),                         # k shorter than q
+        (q, q.clone(), q.clone()[:, :, :1]),                         # k and v shapes differ
+        (q, q.transpose(1, 2).contiguous().transpose(1, 2), q.clone()),   # k not contiguous
+        (q.float(), q.float(), q.float()),                           # fp32 is not an input type
+        (q, q.clone(), q.clone()),                                   # all fine but on the CPU
+    ]
+    for qq, kk, vv in cases:
+        with pytest.raises(rfsa.RfError) as e:
+            rfsa.rf_sparse_attention(qq, kk, vv, "BSND", 0, (4, 32, 32), 0.5, out=torch.empty_like(qq))
+        assert e.value.code == 2
+    with pytest.raises(rfsa.RfError) as e:
+        rfsa.rf_sparse_attention(q, q, q, "BSND", 0, (4, 32, 32), 0.5, out=torch.empty(1, 4096, 2, 64,
+                                                                                      dtype=torch.bfloat16))
+    assert e.value.code == 2 and "out" in str(e.value)
+    with pytest.raises(rfsa.RfError) as e:
+        rfsa.rf_sparse_attention(q, q, q, "BSND", 0, (4, 32, 32), 0.5, out=torch.empty_like(q))
+    assert "CUDA" in str(e.value)

@@ -17,6 +17,11 @@ import torch
 CASES = [
     ("minimax", {"N": 3, "latent": (12, 24, 42)}),
     ("tiny", {"txt_len": 37, "latent": (8, 21, 43), "sparsity": 0.7, "seed": 11, "N": 2}),
+    # BNSD, and two batch entries (BSND and BNSD): the kernel's own token
+    # offsets for each layout and batch index
+    ("tiny", {"txt_len": 19, "latent": (5, 24, 40), "sparsity": 0.6, "layout": "BNSD", "seed": 12, "N": 2}),
+    ("tiny", {"B": 2, "N": 2, "txt_len": 37, "latent": (6, 24, 40), "sparsity": 0.6, "seed": 41}),
+    ("tiny", {"B": 2, "N": 3, "txt_len": 5, "latent": (6, 24, 40), "sparsity": 0.5, "layout": "BNSD", "seed": 42}),
     ("minimax", {"N": 3, "latent": (12, 24, 42)}),
 ]
 
