@@ -1,7 +1,7 @@
 """Benchmark of the rf_v2 block-sparse attention call on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload minimax] [--impl reference]
-                    [--sparsity S] [--dtype bf16|f16] [--precision native|fp8]
+                    [--sparsity S] [--dtype bf16|f16] [--precision native|fp8] [--mode replicas|ulysses]
 
 One step = one full call (token reorder + pooling, block scores + top-k mask,
 block-sparse attention with the inverse reorder fused) on one batch of seeded
@@ -12,6 +12,15 @@ all S keys), divided by the device time of the step.  Under torchrun each rank
 runs its own replica (the call shards by independent problems; no collective
 on the data path), so the aggregate is the sum over ranks divided by the
 slowest rank's time.
+
+``--mode ulysses`` runs the call sequence-parallel instead (vllm-omni
+"RainFusion Attention", "Requirements and compatibility"): each rank holds a
+sequence shard [B, S/P, N, D] of q, k and v; one all-to-all turns them into
+head shards [B, S, N/P, D], the library's call runs on the local heads, and a
+second all-to-all returns the output's sequence shard.  The exchanges are
+NCCL collectives (a process group of one rank without torchrun); the work of
+the whole problem is fixed as P grows ("scaling": "strong"), and the line
+reports the two exchanges and the call separately.
 
 ``--impl reference`` times the plain CPU oracle on the host cores instead, on
 a bounded sample of the same workload.
@@ -96,6 +105,43 @@ def _kv_stream(flops, prec, ms_attention, sm_mhz, sms):
 
 # The attention kernels' sources, hashed together to tie a traffic capture to the code it measured.
 K3_SOURCES = ("rf_attn_common.cuh", "rf_attn_chain.cu", "rf_attn.cu")
+
+
+# Nominal dense tensor peaks of B200 (TFLOP/s), for context beside the measured ones.
+NOMINAL_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0}
+
+
+def _roofline(k3_tflops: float, prec: str, dtype: str, peaks: dict, src: str, traffic):
+    """K3 against the measured sustained matmul peak (the kernel runs back to
+    back for the whole timed region, under the power cap), with the measured
+    burst and the nominal dense peaks beside it.  fp8 takes twice the bf16
+    figures (the nominal fp8 / bf16 ratio)."""
+    mult = 2.0 if prec == "fp8" else 1.0
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * mult
+    burst = peaks["bf16_tflops"] * mult
+    nominal = NOMINAL_TFLOPS["fp8" if prec == "fp8" else "bf16"]
+    note = f"{src} bf16_tflops_sustained"
+    if prec == "fp8":
+        note += " x 2 (nominal fp8 / bf16 ratio)"
+    elif dtype == "f16":
+        note += " (fp16 and bf16 have the same nominal peak)"
+    return {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": sustained,
+            "unit": "TFLOP/s", "frac": k3_tflops / sustained, "traffic": traffic, "peak_source": note,
+            "frac_of_measured_burst": k3_tflops / burst, "measured_burst_peak": burst,
+            "frac_of_nominal": k3_tflops / nominal, "nominal_peak": nominal}
+
+
+def _mask_stats(stats: dict, plan) -> dict:
+    """The mask of the timed call, from the library's statistics: kept key
+    blocks, the realised density of (query, key) pairs, and the selections
+    that sat on a near-tie (k-th and (k+1)-th block scores within 1e-5,
+    relative), which the bit-exact mask check excuses."""
+    return {"k": plan.k, "nb": plan.nb, "ff": plan.ff, "kept_blocks": stats["kept_blocks"],
+            "query_blocks": stats["query_blocks"],
+            "kept_per_query_block": stats["kept_blocks"] / max(stats["query_blocks"], 1),
+            "density": stats["density"], "near_ties": stats["near_ties"],
+            "near_tie_rule": "k-th and (k+1)-th block scores within 1e-5 (relative)",
+            "second_pass_tiles": stats["redo_tiles"]}
 
 
 def _k3_traffic(heads: int):
@@ -304,6 +350,174 @@ def run_reference(args, w):
     return 0
 
 
+# ---------------------------------------------------------------- sequence-parallel arm
+def shard_rows(x, rank: int, world: int):
+    """This rank's sequence shard of a BSND tensor: tokens [r S/P, (r + 1) S/P)."""
+    S = x.shape[1]
+    if S % world:
+        raise ValueError(f"sequence length {S} is not a multiple of the {world} ranks")
+    Sl = S // world
+    return x[:, rank * Sl:(rank + 1) * Sl].contiguous()
+
+
+def _free_port() -> int:
+    import socket
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return port
+
+
+def run_ulysses(args, w):
+    """--mode ulysses: the call on sequence shards, Ulysses all-to-all to head
+    shards and back around the library's call on N / P heads (see the module
+    docstring).  Timed per step with CUDA events: the first exchange, the
+    call (and its attention stage alone), the second exchange; the slowest
+    rank decides each."""
+    import datetime
+    import torch.distributed as dist
+    from block_sparse_video_rf_b200 import rfsa, synth, ulysses
+    if w.layout != "BSND":
+        raise SystemExit("--mode ulysses takes BSND workloads")
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    os.environ.setdefault("RANK", "0")
+    os.environ.setdefault("WORLD_SIZE", "1")
+    os.environ.setdefault("LOCAL_RANK", "0")
+    if "MASTER_PORT" not in os.environ:
+        os.environ["MASTER_PORT"] = str(_free_port())
+    world, rank, local = int(os.environ["WORLD_SIZE"]), int(os.environ["RANK"]), int(os.environ["LOCAL_RANK"])
+    if w.S % world or w.N % world:
+        raise SystemExit(f"S = {w.S} and N = {w.N} must be multiples of the {world} ranks")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    try:
+        return _ulysses_timed(args, w, dist, rfsa, synth, ulysses, world, rank, local, dev)
+    finally:
+        dist.destroy_process_group()
+
+
+def _ulysses_timed(args, w, dist, rfsa, synth, ulysses, world, rank, local, dev):
+    prec = args.precision
+    tdtype = torch.float16 if args.dtype == "f16" else torch.bfloat16
+    sp = np.float32(w.sparsity)
+    Nl = w.N // world
+    # every rank draws the whole seeded problem and keeps its sequence shard
+    q, k, v = synth.make_inputs(w, device=dev, dtype=tdtype)
+    q_sh, k_sh, v_sh = (shard_rows(t, rank, world) for t in (q, k, v))
+    del q, k, v
+    torch.cuda.empty_cache()
+    ws = rfsa.alloc_workspace(w.B, w.S, Nl, w.D, w.txt_len, w.latent, device=dev, precision=prec)
+    plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, sp)
+    views = rfsa.workspace_views(ws, w.B, Nl, plan, dtype=tdtype, precision=prec)
+    out_h = torch.empty((w.B, w.S, Nl, w.D), dtype=tdtype, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cur = {"ev": None}
+
+    def attend(qh, kh, vh):
+        rfsa.rf_prepare(qh, kh, vh, "BSND", w.txt_len, w.latent, sp, ws, precision=prec)
+        if cur["ev"] is not None:
+            cur["ev"][4].record(stream)            # the attention stage starts
+        rfsa.rf_attend(out_h, "BSND", w.txt_len, w.latent, sp, ws, precision=prec)
+        return out_h
+
+    def step(ev=None):
+        cur["ev"] = ev
+        marks = (lambda i: ev[i].record(stream)) if ev is not None else None
+        return ulysses.rf_sparse_attention_ulysses(q_sh, k_sh, v_sh, w.txt_len, w.latent, sp, attend=attend,
+                                                   marks=marks)
+
+    for _ in range(max(args.warmup, 1)):
+        step()
+    torch.cuda.synchronize(dev)
+    if rfsa.rf_read_status(ws, w.B, Nl, w.D, plan) != 0:
+        raise RuntimeError("device status after warm-up")
+    flops_local = rfsa.kept_block_flops(plan, views["kept"], w.B, Nl, w.D)
+    stats = rfsa.rf_read_stats(ws, w.B, Nl, w.D, plan, precision=prec)
+    tot = torch.tensor([flops_local, float(stats["near_ties"]), float(stats["kept_blocks"]),
+                        float(stats["query_blocks"])], dtype=torch.float64, device=dev)
+    dist.all_reduce(tot)
+    flops, near, kept_blocks, query_blocks = tot.tolist()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clocks:
+        t0.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+    a2a_in = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    call = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    k3 = statistics.mean(e[4].elapsed_time(e[2]) for e in evs)
+    a2a_out = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    # end to end: this rank's shards from pinned host memory, the output shard back
+    e2e_steps = args.e2e_steps if args.e2e_steps is not None else min(args.steps, 10)
+    hq, hk, hv = (t.cpu().pin_memory() for t in (q_sh, k_sh, v_sh))
+    ho = torch.empty(q_sh.shape, dtype=tdtype, pin_memory=True)
+
+    def e2e_call():
+        dq, dk, dv = (t.to(dev, non_blocking=True) for t in (hq, hk, hv))
+        o = ulysses.rf_sparse_attention_ulysses(dq, dk, dv, w.txt_len, w.latent, sp, attend=attend)
+        ho.copy_(o, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+
+    e2e_call()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / max(e2e_steps, 1)
+    ms_total, e2e_ms, a2a_in, call, k3, a2a_out = reduce_max([ms_total, e2e_ms, a2a_in, call, k3, a2a_out], dist, dev)
+    ms_step = ms_total / args.steps
+    if rank == 0:
+        peaks, src = _peaks()
+        k3_tflops_rank = flops / world / (k3 * 1e-3) / 1e12          # the slowest rank's K3 over its share
+        shard_bytes = q_sh.numel() * q_sh.element_size()
+        line = {
+            "metric": METRIC, "value": flops / (ms_step * 1e-3) / 1e12, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None,
+            "dtype": args.dtype if prec == "native" else f"e4m3 ({args.dtype} in/out)", "data": "synthetic",
+            "config": {"workload": _describe(w, args.dtype, prec), "mode": "ulysses",
+                       "parallelism": f"ulysses sequence parallel over {world} rank(s): [B, S/{world}, {w.N}, D] "
+                                      f"-> [B, S, {Nl}, D] -> [B, S/{world}, {w.N}, D]",
+                       "l2": "inputs larger than L2 (no flush)", "kept_block_tflop_per_call": flops / 1e12},
+            "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": 3 * shard_bytes, "d2h_bytes_per_step": shard_bytes, "per": "rank"},
+            "roofline": _roofline(k3_tflops_rank, prec, args.dtype, peaks, src, None),
+            "mask_stats": {"k": plan.k, "nb": plan.nb, "kept_blocks": int(kept_blocks),
+                           "query_blocks": int(query_blocks), "near_ties": int(near),
+                           "near_tie_rule": "k-th and (k+1)-th block scores within 1e-5 (relative)"},
+            # per rank and step: K1, K2, K3 and its second pass (the exchanges are NCCL's kernels)
+            "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
+            "stages": {"all_to_all_in": {"ms": a2a_in, "bytes_per_rank": 3 * shard_bytes * (world - 1) / world},
+                       "call": {"ms": call, "heads_per_rank": Nl},
+                       "attention": {"kernels": "K3", "ms": k3, "tflops_per_rank": k3_tflops_rank},
+                       "all_to_all_out": {"ms": a2a_out, "bytes_per_rank": shard_bytes * (world - 1) / world}},
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            from block_sparse_video_rf_b200 import synth as _s
+            qc, kc, vc = _s.make_inputs(_s.workload(w.name, N=1, seed=w.seed), device="cpu")
+            val, threads, desc = oracle_sample(qc, kc, vc, _s.workload(w.name, N=1, sparsity=w.sparsity),
+                                               heads_total=w.N)
+            line["cpu_baseline"] = {"value": val, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": desc}
+        print(json.dumps(line), flush=True)
+    dist.barrier()
+    return 0
+
+
 # ---------------------------------------------------------------- CUDA arm
 def main():
     ap = argparse.ArgumentParser()
@@ -319,6 +533,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f16"])
     ap.add_argument("--precision", default="native", choices=["native", "fp8"])
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "ulysses"],
+                    help="replicas: every rank runs the whole call; ulysses: sequence-parallel over the ranks")
     args = ap.parse_args()
 
     from block_sparse_video_rf_b200 import synth
@@ -328,6 +544,8 @@ def main():
     w = synth.workload(args.workload, **over)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.mode == "ulysses":
+        return run_ulysses(args, w)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -370,6 +588,7 @@ def main():
     if status != 0:
         raise RuntimeError(f"device status {status} after warm-up")
     flops = rfsa.kept_block_flops(plan, views["kept"], w.B, w.N, w.D)
+    stats = rfsa.rf_read_stats(ws, w.B, w.N, w.D, plan, precision=prec)
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     for e in evs:
@@ -429,13 +648,6 @@ def main():
 
     if rank == 0:
         peaks, src = _peaks()
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        peak_note = f"{src} bf16_tflops_sustained"
-        if prec == "fp8":
-            peak *= 2.0           # nominal dense fp8 / bf16 ratio: 4.5 / 2.25 PFLOP/s
-            peak_note += " x 2 (nominal fp8 / bf16 ratio)"
-        elif args.dtype == "f16":
-            peak_note += " (fp16 and bf16 have the same nominal peak)"
         k3_tflops = flops / (k3_ms * 1e-3) / 1e12
         tensor_bytes = q.numel() * q.element_size()
         line = {
@@ -448,9 +660,8 @@ def main():
                        "P": plan.P, "ms_prepare": statistics.mean(k1k2), "ms_attention": k3_ms},
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
-            "roofline": {"kernel": "rf attention (K3)", "bound": "tensor", "achieved": k3_tflops, "peak": peak,
-                         "unit": "TFLOP/s", "frac": k3_tflops / peak,
-                         "traffic": _k3_traffic(w.N) if default_mode else None, "peak_source": peak_note},
+            "roofline": _roofline(k3_tflops, prec, args.dtype, peaks, src, _k3_traffic(w.N) if default_mode else None),
+            "mask_stats": _mask_stats(stats, plan),
             # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
             # handed to it); fp8 adds the quantisation pass
             "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,

@@ -49,13 +49,15 @@ def heads_to_seq(y: torch.Tensor, group=None) -> torch.Tensor:
 
 
 def rf_sparse_attention_ulysses(q, k, v, txt_len: int, latent, sparsity: float, group=None, scale=None,
-                                precision: str = "native", attend=None):
+                                precision: str = "native", attend=None, marks=None):
     """The rf_v2 call on sequence-sharded BSND q, k, v (see the module
     docstring); returns this rank's sequence shard of the output.
 
     ``attend`` is the call on whole-sequence head shards; it defaults to the
     library's ``rf_sparse_attention`` (tests pass a CPU stand-in to check the
-    exchanges without a GPU)."""
+    exchanges without a GPU).  ``marks``, if given, is called with 0 before
+    the first exchange, 1 after it, 2 after the call and 3 after the second
+    exchange (a benchmark records CUDA events there)."""
     if attend is None:
         from . import rfsa
 
@@ -63,5 +65,12 @@ def rf_sparse_attention_ulysses(q, k, v, txt_len: int, latent, sparsity: float, 
             return rfsa.rf_sparse_attention(qh, kh, vh, "BSND", txt_len, latent, sparsity, scale=scale,
                                             precision=precision)
 
+    mark = marks if marks is not None else (lambda i: None)
+    mark(0)
     qh, kh, vh = (seq_to_heads(t.contiguous(), group) for t in (q, k, v))
-    return heads_to_seq(attend(qh, kh, vh), group)
+    mark(1)
+    oh = attend(qh, kh, vh)
+    mark(2)
+    o = heads_to_seq(oh, group)
+    mark(3)
+    return o

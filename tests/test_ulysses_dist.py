@@ -52,9 +52,15 @@ def _worker(rank, world, port, out):
         heads_ok = torch.equal(qh, q[:, :, rank * Nl:(rank + 1) * Nl])
         # and back
         back_ok = torch.equal(ulysses.heads_to_seq(qh), q[:, mine])
-        # the composed call against the oracle on the whole problem
-        got = ulysses.rf_sparse_attention_ulysses(q[:, mine], k[:, mine], v[:, mine], w.txt_len, w.latent,
-                                                  np.float32(w.sparsity), attend=_oracle_attend(w))
+        # the composed call against the oracle on the whole problem, on the
+        # shards bench.py's sequence-parallel arm takes, with its stage marks
+        import bench
+        marks = []
+        qs, ks, vs = (bench.shard_rows(t, rank, world) for t in (q, k, v))
+        shard_ok = torch.equal(qs, q[:, mine])
+        got = ulysses.rf_sparse_attention_ulysses(qs, ks, vs, w.txt_len, w.latent, np.float32(w.sparsity),
+                                                  attend=_oracle_attend(w), marks=marks.append)
+        heads_ok = heads_ok and shard_ok and marks == [0, 1, 2, 3]
         try:
             ulysses.seq_to_heads(torch.zeros(1, 4, 3, 8))       # 3 heads over 2 ranks
             reject_ok = False
