@@ -144,9 +144,10 @@ def _mask_stats(stats: dict, plan) -> dict:
             "second_pass_tiles": stats["redo_tiles"]}
 
 
-def _k3_traffic(heads: int):
-    """DRAM bytes per attention launch from the committed ncu summary, scaled to
-    ``heads``; None when the kernel source changed since the capture."""
+def _k3_traffic(heads: int, label: str = "k3"):
+    """DRAM bytes per attention launch from the committed ncu summary (label
+    k3: 16-bit operands, k3_fp8: e4m3 operands), scaled to ``heads``; None
+    when the kernel source changed since the capture."""
     import hashlib
     csrc = os.path.join(ROOT, "block_sparse_video_rf_b200", "csrc")
     path = os.path.join(ROOT, "profiles", "k3_traffic.txt")
@@ -158,7 +159,7 @@ def _k3_traffic(heads: int):
     digest = h.hexdigest()[:16]
     for line in open(path):
         parts = line.split()
-        if len(parts) >= 3 and not line.startswith("#") and parts[0] == "k3" and parts[1] == digest:
+        if len(parts) >= 3 and not line.startswith("#") and parts[0] == label and parts[1] == digest:
             return int(parts[2]) * heads / 56.0
     return None
 
@@ -660,7 +661,10 @@ def main():
                        "P": plan.P, "ms_prepare": statistics.mean(k1k2), "ms_attention": k3_ms},
             "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_step": e2e_ms,
                     "h2d_bytes_per_step": 3 * tensor_bytes, "d2h_bytes_per_step": tensor_bytes},
-            "roofline": _roofline(k3_tflops, prec, args.dtype, peaks, src, _k3_traffic(w.N) if default_mode else None),
+            # the committed capture is of the MiniMax-H3 shape: other workloads' traffic is not a multiple of it
+            "roofline": _roofline(k3_tflops, prec, args.dtype, peaks, src,
+                                  _k3_traffic(w.N, "k3_fp8" if prec == "fp8" else "k3")
+                                  if args.dtype == "bf16" and w.name == "minimax" else None),
             "mask_stats": _mask_stats(stats, plan),
             # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
             # handed to it); fp8 adds the quantisation pass
