@@ -128,3 +128,40 @@ def test_text_prefixed_clip_all_heads():
     if not torch.cuda.is_available():
         pytest.skip("needs a GPU")
     _whole_heads("text", tuple(range(12)))
+
+
+def test_half_head_minimax_fp8():
+    # fp8 e4m3 at MiniMax-H3: every second row of one head (31,376 rows: text,
+    # promoted, first-frame and sparse rows alike) against the oracle over the
+    # dequantised operands, under the error model of P's e4m3 rounding
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    w, q, k, v, out, plan, views = _run("minimax", precision="fp8")
+    g = oracle.geometry(w.S, w.txt_len, *w.latent)
+    words = views["mask"].cpu().numpy().view(np.uint32)
+    n = 31
+    rows = np.arange(0, w.S, 2)
+    qh, kh, vh = _head(q, n), _head(k, n), _head(v, n)
+    ref, bound, sigma = fp8_reference(qh, kh, vh, g, unpack_mask(words[0, n], g.nb), w.D ** -0.5, rows=rows)
+    got = out[0, torch.from_numpy(rows).cuda(), n].float().cpu().numpy()
+    mx, mean, ratio = assert_close_fp8(got, ref, bound, sigma, f"minimax fp8 head {n}, every second row")
+    print(f"minimax fp8 head {n}: {len(rows)} rows, max-abs {mx:.2e} mean-abs {mean:.2e} (err/sigma)^2 {ratio:.3f}")
+
+
+def test_full_size_bnsd_sampled():
+    # the caller's BNSD layout at the full MiniMax-H3 shape (the bench runs BSND)
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    w, q, k, v, out, plan, views = _run("minimax", layout="BNSD")
+    g = oracle.geometry(w.S, w.txt_len, *w.latent)
+    words = views["mask"].cpu().numpy().view(np.uint32)
+    rng = np.random.default_rng(321)
+    for n in (2, 44):
+        qh, kh, vh = (x[0, n].float().cpu().numpy() for x in (q, k, v))     # BNSD -> [S, D]
+        mask, margin = oracle.build_mask(qh[None, None], kh[None, None], g, float(np.float32(w.sparsity)))
+        bad, excused, near = mask_mismatch(words[0, n][None, None], mask, margin)
+        assert bad == 0, f"head {n}: {bad} mask rows differ outside near-ties"
+        rows = _sample_rows(g, rng)
+        got = out[0, n, torch.from_numpy(rows).cuda()].float().cpu().numpy()
+        ref = oracle.attention_rows(qh, kh, vh, g, unpack_mask(words[0, n], g.nb), w.D ** -0.5, rows=rows)
+        assert_close(got, ref, f"minimax BNSD head {n}")
