@@ -301,3 +301,21 @@ def test_binding_checks_tensors_before_the_library(rfsa):
     with pytest.raises(rfsa.RfError) as e:
         rfsa.rf_sparse_attention(q, q, q, "BSND", 0, (4, 32, 32), 0.5, out=torch.empty_like(q))
     assert "CUDA" in str(e.value)
+
+
+def test_plain_c_caller(rfsa, tmp_path):
+    # the header compiles as C11 and a C program links the library and runs
+    # its host-only entry points (tests/c/abi_host.c)
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    exe = tmp_path / "abi_host"
+    lib_dir = os.path.dirname(rfsa.LIB_PATH)
+    subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_host.c"), "-L", lib_dir, "-lrfsa",
+                    "-Wl,-rpath," + lib_dir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "FAIL" not in r.stdout and r.stdout.count("ok") >= 11
