@@ -94,7 +94,7 @@ def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs, ms_k1=N
 def _kv_stream(flops, prec, ms_attention, sm_mhz, sms):
     """K and V brought from L2 into the SMs by K3: each (query row, kept key) pair costs 4 bytes (a 128 x 128
     tile pair of 64 KB serves 128 x 128 pairs; e4m3: 2 bytes) and 4 D = 512 FLOPs.  Per SM cycle at the median
-    SM clock sampled in the timed region, against the ~50 bytes per SM cycle a streaming probe reached."""
+    SM clock sampled in the timed region (two TMA threads per SM stream about 74 bytes per SM cycle from L2)."""
     pairs = flops / (4 * 128)
     nbytes = pairs * (2 if prec == "fp8" else 4)
     out = {"bytes": nbytes, "tbs": nbytes / (ms_attention * 1e-3) / 1e12}
