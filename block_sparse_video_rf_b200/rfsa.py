@@ -335,6 +335,49 @@ def rf_block_mask_noalloc(q, k, layout, txt_len, latent, sparsity, mask, kept, m
                                      _stream(q, stream)))
 
 
+def sparse_attention(q, k, v, attn_mask=None, scale=None, is_causal=False, head_num=1, input_layout="BNSD",
+                     inner_precise=0, sparse_type=None, txt_len=0, block_size=128, latent_shape_q=None,
+                     latent_shape_k=None, keep_sink=True, keep_recent=True, cdf_threshold=1.0, sparsity=0.0,
+                     **_kwargs):
+    """The operation under the parameter list of MindSpore Lite's
+    ``lite_boost.ops.sparse_attention`` (argument checks and marshalling
+    only; the call is ``rf_sparse_attention``).
+
+    - ``sparse_type=None``: dense softmax attention over the whole sequence;
+      ``"rf_v2"``: block-sparse (token reorder, block pooling, top-k mask,
+      attention, inverse reorder) with ``latent_shape_q`` (required) and
+      ``latent_shape_k`` (default: the query's).  Any other value raises
+      ValueError, as does an ``input_layout`` other than "BSND" / "BNSD"
+      (the page's "Raises").
+    - ``head_num`` must equal the tensors' head dimension.
+    - ``scale`` None means head_dim ** -0.5.  ``sparsity`` in [0, 1].
+    - ``attn_mask`` is reserved on the page and unused by rf_v2; ``keep_sink``,
+      ``keep_recent`` and ``cdf_threshold`` belong to another mode and are
+      not read; ``inner_precise`` selects nothing here (the arithmetic is
+      the precision the inputs give).  A causal mask (``is_causal=True``) is
+      not implemented and raises NotImplementedError.
+    Returns the output, shaped like q."""
+    if input_layout not in LAYOUTS:
+        raise ValueError(f'input_layout must be "BSND" or "BNSD" (got {input_layout!r})')
+    if sparse_type not in (None, "rf_v2"):
+        raise ValueError(f'sparse_type must be None or "rf_v2" (got {sparse_type!r})')
+    if is_causal:
+        raise NotImplementedError("causal attention is not implemented")
+    B, S, N, D = _dims(q, input_layout)
+    if head_num != N:
+        raise ValueError(f"head_num {head_num} does not match the tensors' {N} heads")
+    if sparse_type is None:
+        return rf_sparse_attention(q, k, v, input_layout, 0, (0, 0, 0), 0.0, scale=scale, block_size=block_size)
+    if latent_shape_q is None:
+        raise ValueError("the rf_v2 path needs latent_shape_q (t, h, w)")
+    latent = tuple(int(x) for x in latent_shape_q)
+    latent_k = None if latent_shape_k is None else tuple(int(x) for x in latent_shape_k)
+    if latent_k == latent:
+        latent_k = None
+    return rf_sparse_attention(q, k, v, input_layout, int(txt_len), latent, float(sparsity), scale=scale,
+                               block_size=int(block_size), latent_k=latent_k)
+
+
 def rf_debug_set_wait(wait_limit_ns: int = 0, skip_first_q: int = 0):
     """Test control of the attention kernel's bounded waits (see include/rfsa.h)."""
     _check(LIB.rf_debug_set_wait(int(wait_limit_ns), int(skip_first_q)))

@@ -319,3 +319,25 @@ def test_plain_c_caller(rfsa, tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "FAIL" not in r.stdout and r.stdout.count("ok") >= 11
+
+
+def test_page_signature_checks(rfsa):
+    # rfsa.sparse_attention takes lite_boost.ops.sparse_attention's parameter
+    # list; the page's ValueErrors come before anything reaches the library
+    import torch
+    q = torch.zeros(1, 4096, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        rfsa.sparse_attention(q, q, q, head_num=2, input_layout="SBND", sparse_type="rf_v2", latent_shape_q=(4, 32, 32))
+    with pytest.raises(ValueError):
+        rfsa.sparse_attention(q, q, q, head_num=2, input_layout="BSND", sparse_type="rf_v3", latent_shape_q=(4, 32, 32))
+    with pytest.raises(ValueError):
+        rfsa.sparse_attention(q, q, q, head_num=3, input_layout="BSND", sparse_type="rf_v2", latent_shape_q=(4, 32, 32))
+    with pytest.raises(ValueError):
+        rfsa.sparse_attention(q, q, q, head_num=2, input_layout="BSND", sparse_type="rf_v2")
+    with pytest.raises(NotImplementedError):
+        rfsa.sparse_attention(q, q, q, head_num=2, input_layout="BSND", is_causal=True)
+    # accepted arguments reach the tensor checks (these are CPU tensors)
+    with pytest.raises(rfsa.RfError) as e:
+        rfsa.sparse_attention(q, q, q, head_num=2, input_layout="BSND", sparse_type="rf_v2", latent_shape_q=(4, 32, 32),
+                              sparsity=0.5, keep_sink=False, cdf_threshold=0.5)
+    assert "CUDA" in str(e.value)

@@ -263,3 +263,21 @@ def test_tiny_sequences_without_video_geometry(rfsa, S):
     qb, kb, vb = (to_bnsd_np(t, "BSND") for t in (q, k, v))
     for n in range(3):
         assert_close(to_bnsd_np(out, "BSND")[0, n], oracle.dense_attention(qb[0, n], kb[0, n], vb[0, n], 128 ** -0.5))
+
+
+@pytest.mark.parametrize("layout", ["BSND", "BNSD"])
+def test_page_signature_call(rfsa, layout):
+    # rfsa.sparse_attention, the page's parameter list: rf_v2 gives the direct
+    # call's output bit for bit; sparse_type None is dense attention
+    w, q, k, v = _inputs("tiny", txt_len=37, latent=(8, 21, 43), sparsity=0.7, layout=layout, seed=71)
+    sp = np.float32(w.sparsity)
+    a = rfsa.sparse_attention(q, k, v, head_num=w.N, input_layout=layout, sparse_type="rf_v2", txt_len=w.txt_len,
+                              latent_shape_q=list(w.latent), sparsity=sp)
+    b = rfsa.rf_sparse_attention(q, k, v, layout, w.txt_len, w.latent, sp)
+    d = rfsa.sparse_attention(q, k, v, head_num=w.N, input_layout=layout)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+    qb, kb, vb = (to_bnsd_np(t, layout) for t in (q, k, v))
+    got = to_bnsd_np(d, layout)
+    for n in range(w.N):
+        assert_close(got[0, n], oracle.dense_attention(qb[0, n], kb[0, n], vb[0, n], w.D ** -0.5), f"dense n{n}")
