@@ -308,6 +308,9 @@ def rf_unpermute(o_int, out, layout, txt_len, latent, stream=None):
     _check_tensors(layout, out)
     if o_int.dtype != out.dtype or not o_int.is_contiguous() or not o_int.is_cuda:
         raise RfError(2, "o_int must be a contiguous CUDA tensor of out's type")
+    plan = rf_plan(S, txt_len, latent, 0.0)
+    if o_int.numel() < B * N * plan.S_int * D:
+        raise RfError(2, f"o_int holds {o_int.numel()} values, the internal layout needs {B * N * plan.S_int * D}")
     _check(LIB.rf_unpermute(_ptr(o_int), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent, _ptr(out),
                             _stream(out, stream)))
     return out
@@ -318,6 +321,9 @@ def rf_sparse_attention_host(q, k, v, layout, txt_len, latent, sparsity, out, sc
     """q, k, v, out: CPU (ideally pinned) bf16 tensors; copies happen inside the library."""
     import torch
     B, S, N, D = _dims(q, layout)
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
+            raise RfError(2, f"{name} must be a contiguous CPU bf16 tensor shaped like q {tuple(q.shape)}")
     st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
     _check(LIB.rf_sparse_attention_host(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
                                         *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
@@ -327,9 +333,20 @@ def rf_sparse_attention_host(q, k, v, layout, txt_len, latent, sparsity, out, sc
 
 def rf_block_mask_noalloc(q, k, layout, txt_len, latent, sparsity, mask, kept, margin, block_size=128,
                           stream=None):
-    """Block mask into caller buffers, with no device allocation (see include/rfsa.h)."""
+    """Block mask into caller buffers, with no device allocation (see include/rfsa.h).
+
+    mask: int32 or uint32 [B, N, nb, ceil(nb / 32)], kept: int32 [B, N, nb],
+    margin: float32 [B, N, nb], contiguous CUDA tensors (checked here: the
+    library sees only their addresses)."""
+    import torch
     B, S, N, D = _dims(q, layout)
     _check_tensors(layout, q, k)
+    plan = rf_plan(S, txt_len, latent, float(sparsity), block_size)
+    rows = B * N * plan.nb
+    for name, t, n, types in (("mask", mask, rows * plan.mask_words, (torch.int32, torch.uint32)),
+                              ("kept", kept, rows, (torch.int32,)), ("margin", margin, rows, (torch.float32,))):
+        if t.dtype not in types or not t.is_contiguous() or not t.is_cuda or t.numel() < n:
+            raise RfError(2, f"{name} must be a contiguous CUDA {types[0]} tensor of at least {n} values")
     _check(LIB.rf_block_mask_noalloc(_ptr(q), _ptr(k), LAYOUTS.get(layout, -1), B, S, N, D, txt_len, *latent,
                                      block_size, float(sparsity), _ptr(mask), _ptr(kept), _ptr(margin),
                                      _stream(q, stream)))

@@ -341,3 +341,20 @@ def test_page_signature_checks(rfsa):
         rfsa.sparse_attention(q, q, q, head_num=2, input_layout="BSND", sparse_type="rf_v2", latent_shape_q=(4, 32, 32),
                               sparsity=0.5, keep_sink=False, cdf_threshold=0.5)
     assert "CUDA" in str(e.value)
+
+
+def test_binding_checks_buffer_sizes_and_kinds(rfsa):
+    # the host-buffer call takes CPU bf16 tensors shaped like q; the
+    # allocation-free mask takes output tensors of at least the mask's size:
+    # both are refused in the binding, before the library sees bare pointers
+    import torch
+    q = torch.zeros(1, 4096, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_sparse_attention_host(q, q, q.float(), "BSND", 0, (4, 32, 32), 0.5, torch.empty_like(q))
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_sparse_attention_host(q, q[:, :2048].contiguous(), q, "BSND", 0, (4, 32, 32), 0.5, torch.empty_like(q))
+    with pytest.raises(rfsa.RfError) as e:
+        # CPU q and k: refused by the tensor checks (a GPU run would reach the size checks below)
+        rfsa.rf_block_mask_noalloc(q, q, "BSND", 0, (4, 32, 32), 0.5, torch.zeros(1, dtype=torch.int32),
+                                   torch.zeros(1, dtype=torch.int32), torch.zeros(1))
+    assert e.value.code == 2

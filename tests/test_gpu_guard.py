@@ -92,3 +92,24 @@ def test_guard_bytes_key_geometry(rfsa):
     rfsa.rf_sparse_attention_ws(q, kk, vv, w.layout, w.txt_len, w.latent, sp, ws, out=out, latent_k=kv_latent)
     torch.cuda.synchronize()
     assert _intact(ws_buf, n_ws) and _intact(out_buf, n_out)
+
+
+def test_undersized_caller_buffers_are_refused():
+    # buffers the library would write through bare pointers are checked for
+    # size in the binding: an output one element short is an argument error
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    from block_sparse_video_rf_b200 import rfsa, synth
+    w = synth.workload("tiny", N=2)
+    q, k, v = synth.make_inputs(w, device="cuda")
+    sp = np.float32(w.sparsity)
+    plan = rfsa.rf_plan(w.S, w.txt_len, w.latent, sp)
+    rows = w.B * w.N * plan.nb
+    mask = torch.zeros(rows * plan.mask_words - 1, dtype=torch.int32, device="cuda")
+    kept = torch.zeros(rows, dtype=torch.int32, device="cuda")
+    margin = torch.zeros(rows, dtype=torch.float32, device="cuda")
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_block_mask_noalloc(q, k, w.layout, w.txt_len, w.latent, sp, mask, kept, margin)
+    o_int = torch.zeros(w.B * w.N * plan.S_int * 128 - 1, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rfsa.RfError):
+        rfsa.rf_unpermute(o_int, torch.empty_like(q), w.layout, w.txt_len, w.latent)
