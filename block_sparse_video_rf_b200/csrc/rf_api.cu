@@ -468,43 +468,51 @@ rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, in
   return ok();
 }
 
-rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void* vh, rf_layout_t layout, int B, int S,
-                                     int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
-                                     float scale, void* out_h, void* stream) {
+rf_status_t rf_sparse_attention_host_ex(const void* qh, const void* kh, const void* vh, rf_dtype_t dtype,
+                                        rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                                        int txt_len, int T, int H, int W, int S_kv, int kv_t, int kv_h, int kv_w,
+                                        int block_size, float sparsity, float scale, void* out_h, void* stream) {
   rf_status_t st = check_common(layout, B, S, N, D);
   if (st != RF_OK) return st;
+  if ((st = check_types(dtype, precision)) != RF_OK) return st;
   if (!qh || !kh || !vh || !out_h) return fail(RF_ERR_ARG, "host buffers must not be NULL");
-  rf_plan_t g;
-  if ((st = rf_plan(S, txt_len, T, H, W, block_size, sparsity, &g)) != RF_OK) return st;
-  // Heads are independent: the call runs on chunks of c heads of one batch
-  // entry, each a [1, S, c, D] (BSND) or [1, c, S, D] (BNSD) problem, in two
-  // device slots.  While chunk i computes on the caller's stream, chunk i + 1
-  // is copied in on one stream and chunk i - 1 copied out on another.
-  // About 96 MiB of q, k and v per chunk (2 heads at MiniMax-H3): a shorter
-  // pipeline tail than 192 MiB (52.3 vs 53.4 ms per call there).  At least 2
-  // heads when BSND: a chunk of 1 head copies 256-byte rows, and the strided
-  // copy then runs far below the link's rate (81.6 ms).
-  const size_t head_bytes = (size_t)S * D * 2;
-  int c = std::max(1, std::min(N, (int)(((size_t)96 << 20) / (3 * head_bytes))));
+  rf_plan_t g, gk;
+  if ((st = make_plans(S, txt_len, T, H, W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, &g, &gk)) != RF_OK)
+    return st;
+  // Heads are independent in every precision (the fp8 scales belong to one
+  // head's tiles, vmax to one head), so the call runs on chunks of c heads
+  // of one batch entry, each a [1, S, c, D] (BSND) or [1, c, S, D] (BNSD)
+  // problem, in two device slots.  While chunk i computes on the caller's
+  // stream, chunk i + 1 is copied in on one stream and chunk i - 1 copied
+  // out on another.  About 96 MiB of q, k and v per chunk (2 heads at
+  // MiniMax-H3): a shorter pipeline tail than 192 MiB (52.3 vs 53.4 ms per
+  // call there).  At least 2 heads when BSND: a chunk of 1 head copies
+  // 256-byte rows, and the strided copy then runs far below the link's rate
+  // (81.6 ms).
+  const int S_k = S_kv > 0 ? S_kv : S;
+  const size_t head_q = (size_t)S * D * 2, head_k = (size_t)S_k * D * 2;
+  int c = std::max(1, std::min(N, (int)(((size_t)96 << 20) / (head_q + 2 * head_k))));
   if (layout == RF_BSND && c < 2) c = std::min(N, 2);
-  const size_t chunk = align256((size_t)c * head_bytes);
+  const size_t chunk_q = align256((size_t)c * head_q), chunk_k = align256((size_t)c * head_k);
+  const size_t slot = 2 * chunk_q + 2 * chunk_k;   // q, k, v, out
   rf_ws_layout_t L;
-  if ((st = rf_workspace_layout(1, c, D, &g, &L)) != RF_OK) return st;
+  if ((st = rf_workspace_layout_ex(precision, 1, c, D, &g, &gk, &L)) != RF_OK) return st;
   const size_t ws_slot = align256(L.total);
   void* io = nullptr;
   void* ws = nullptr;
-  if ((st = cached_buffer(g_io, 2 * 4 * chunk, &io)) != RF_OK) return st;
+  if ((st = cached_buffer(g_io, 2 * slot, &io)) != RF_OK) return st;
   if ((st = cached_buffer(g_ws, 2 * ws_slot, &ws)) != RF_OK) return st;
   HostPipe* hp = nullptr;
   if ((st = host_pipe(&hp)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == RF_BSND;
   const size_t row = (size_t)N * D * 2;   // BSND: one token's heads
-  auto copy = [&](void* dst, const void* src, int heads, cudaMemcpyKind kind, bool to_dev, cudaStream_t cs) {
-    if (!bsnd) return cudaMemcpyAsync(dst, src, (size_t)heads * head_bytes, kind, cs);
+  // `heads` heads of a tensor of `len` tokens; BSND copies `len` strided rows
+  auto copy = [&](void* dst, const void* src, int heads, int len, cudaMemcpyKind kind, bool to_dev, cudaStream_t cs) {
+    if (!bsnd) return cudaMemcpyAsync(dst, src, (size_t)heads * len * D * 2, kind, cs);
     const size_t w = (size_t)heads * D * 2;
-    return to_dev ? cudaMemcpy2DAsync(dst, w, src, row, w, S, kind, cs)
-                  : cudaMemcpy2DAsync(dst, row, src, w, w, S, kind, cs);
+    return to_dev ? cudaMemcpy2DAsync(dst, w, src, row, w, len, kind, cs)
+                  : cudaMemcpy2DAsync(dst, row, src, w, w, len, kind, cs);
   };
   const char* srcs[3] = {static_cast<const char*>(qh), static_cast<const char*>(kh), static_cast<const char*>(vh)};
   char* outh = static_cast<char*>(out_h);
@@ -514,20 +522,25 @@ rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void*
     for (int n0 = 0; n0 < N; n0 += c, ++i) {
       const int heads = std::min(c, N - n0);
       const int z = i & 1;
-      char* d = static_cast<char*>(io) + (size_t)z * 4 * chunk;
-      // host offset of the chunk's first element
-      const size_t off = bsnd ? ((size_t)b * S * N + n0) * D * 2 : ((size_t)b * N + n0) * head_bytes;
+      char* d = static_cast<char*>(io) + (size_t)z * slot;
+      char* dev[4] = {d, d + chunk_q, d + chunk_q + chunk_k, d + chunk_q + 2 * chunk_k};   // q, k, v, out
+      // host offset of the chunk's first element in a tensor of `len` tokens
+      auto off = [&](int len) {
+        return bsnd ? ((size_t)b * len * N + n0) * D * 2 : ((size_t)b * N + n0) * len * D * 2;
+      };
       // copy in once the slot's previous chunk has been computed
       if (i >= 2 && (e = cudaStreamWaitEvent(hp->in, hp->comp[z], 0)) != cudaSuccess) break;
-      for (int t = 0; t < 3 && e == cudaSuccess; ++t)
-        e = copy(d + t * chunk, srcs[t] + off, heads, cudaMemcpyHostToDevice, true, hp->in);
+      for (int t = 0; t < 3 && e == cudaSuccess; ++t) {
+        const int len = t == 0 ? S : S_k;
+        e = copy(dev[t], srcs[t] + off(len), heads, len, cudaMemcpyHostToDevice, true, hp->in);
+      }
       if (e != cudaSuccess || (e = cudaEventRecord(hp->loaded[z], hp->in)) != cudaSuccess) break;
       // compute once it is in and the slot's previous output has left
       if ((e = cudaStreamWaitEvent(s, hp->loaded[z], 0)) != cudaSuccess) break;
       if (i >= 2 && (e = cudaStreamWaitEvent(s, hp->stored[z], 0)) != cudaSuccess) break;
-      st = rf_sparse_attention_ws(d, d + chunk, d + 2 * chunk, layout, 1, S, heads, D, txt_len, T, H, W, block_size,
-                                  sparsity, scale, d + 3 * chunk, static_cast<char*>(ws) + (size_t)z * ws_slot,
-                                  ws_slot, stream);
+      st = rf_sparse_attention_ex(dev[0], dev[1], dev[2], dtype, precision, layout, 1, S, heads, D, txt_len, T, H,
+                                  W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, scale, dev[3],
+                                  static_cast<char*>(ws) + (size_t)z * ws_slot, ws_slot, stream);
       if (st != RF_OK) {
         // no copy of the caller's buffers may still run when this returns
         cudaStreamSynchronize(hp->in);
@@ -538,7 +551,7 @@ rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void*
       if ((e = cudaEventRecord(hp->comp[z], s)) != cudaSuccess) break;
       // copy out
       if ((e = cudaStreamWaitEvent(hp->out, hp->comp[z], 0)) != cudaSuccess) break;
-      if ((e = copy(outh + off, d + 3 * chunk, heads, cudaMemcpyDeviceToHost, false, hp->out)) != cudaSuccess) break;
+      if ((e = copy(outh + off(S), dev[3], heads, S, cudaMemcpyDeviceToHost, false, hp->out)) != cudaSuccess) break;
       if ((e = cudaEventRecord(hp->stored[z], hp->out)) != cudaSuccess) break;
     }
     if (e != cudaSuccess) break;
@@ -549,6 +562,13 @@ rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void*
   if (e == cudaSuccess) e = e_in != cudaSuccess ? e_in : e_out != cudaSuccess ? e_out : e_s;
   if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline (copies, events or synchronisation)");
   return ok();
+}
+
+rf_status_t rf_sparse_attention_host(const void* qh, const void* kh, const void* vh, rf_layout_t layout, int B, int S,
+                                     int N, int D, int txt_len, int T, int H, int W, int block_size, float sparsity,
+                                     float scale, void* out_h, void* stream) {
+  return rf_sparse_attention_host_ex(qh, kh, vh, RF_BF16, RF_PREC_NATIVE, layout, B, S, N, D, txt_len, T, H, W, 0, 0,
+                                     0, 0, block_size, sparsity, scale, out_h, stream);
 }
 
 rf_status_t rf_read_status(void* ws, size_t ws_bytes, int B, int N, int D, const rf_plan_t* g, int* status,

@@ -34,7 +34,7 @@ EXPORTS = ["rf_plan", "rf_workspace_layout", "rf_workspace_size", "rf_sparse_att
            "rf_debug_set_wait", "rf_debug_set_path", "rf_debug_set_stage_event", "rf_read_stats",
            "rf_block_mask_noalloc", "rf_last_error_string", "rf_workspace_layout_ex",
            "rf_workspace_size_ex", "rf_prepare_ex", "rf_attend_ex", "rf_sparse_attention_ex", "rf_plan_kv",
-           "rf_read_stats_ex", "rf_debug_exp2_poly"]
+           "rf_read_stats_ex", "rf_debug_exp2_poly", "rf_sparse_attention_host_ex"]
 
 
 class RfPlan(ctypes.Structure):
@@ -96,6 +96,7 @@ def _load():
         "rf_prepare_ex": (I, [P, P, P, I, I] + geo + [I, I, I, I, I, I, F, P, Z, P]),
         "rf_attend_ex": (I, [I, I] + geo + [I, I, I, I, I, I, F, F, P, P, Z, P]),
         "rf_sparse_attention_ex": (I, [P, P, P, I, I] + geo + [I, I, I, I, I, I, F, F, P, P, Z, P]),
+        "rf_sparse_attention_host_ex": (I, [P, P, P, I, I] + geo + [I, I, I, I, I, I, F, F, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -122,12 +123,13 @@ def _dims(x, layout: str):
     return B, S, N, D
 
 
-def _check_tensors(layout: str, q, k=None, v=None, out=None, same_kv_len: bool = True):
+def _check_tensors(layout: str, q, k=None, v=None, out=None, same_kv_len: bool = True, host: bool = False):
     """Checks, before any call into the library, what the C ABI cannot see
     from bare pointers: every tensor is a contiguous torch tensor of bf16 or
-    fp16 (all of one type) on one CUDA device; k and v have one shape, with
-    q's batch, heads and head dim (and q's length unless k and v have a
-    geometry of their own); out has q's shape.  Raises RfError(RF_ERR_ARG)."""
+    fp16 (all of one type) on one CUDA device (host: in CPU memory); k and v
+    have one shape, with q's batch, heads and head dim (and q's length unless
+    k and v have a geometry of their own); out has q's shape.  Raises
+    RfError(RF_ERR_ARG)."""
     dims = _dims(q, layout)
     tensors = [("q", q), ("k", k), ("v", v), ("out", out)]
     tensors = [(n, t) for n, t in tensors if t is not None]
@@ -149,7 +151,9 @@ def _check_tensors(layout: str, q, k=None, v=None, out=None, same_kv_len: bool =
         if not t.is_contiguous():
             raise RfError(2, f"{name} must be contiguous")
     for name, t in tensors:
-        if not t.is_cuda or t.device != q.device:
+        if host and t.device.type != "cpu":
+            raise RfError(2, f"{name} must be a CPU tensor, got {t.device}")
+        if not host and (not t.is_cuda or t.device != q.device):
             raise RfError(2, f"{name} must be a CUDA tensor on q's device ({q.device}), got {t.device}")
 
 
@@ -317,17 +321,24 @@ def rf_unpermute(o_int, out, layout, txt_len, latent, stream=None):
 
 
 def rf_sparse_attention_host(q, k, v, layout, txt_len, latent, sparsity, out, scale=None, block_size=128,
-                             stream=None):
-    """q, k, v, out: CPU (ideally pinned) bf16 tensors; copies happen inside the library."""
+                             stream=None, precision: str = "native", latent_k=None):
+    """The whole call through host buffers: q, k, v, out are contiguous CPU
+    (ideally pinned) tensors of one 16-bit type, out shaped like q; the
+    copies to and from the device happen inside the library."""
     import torch
     B, S, N, D = _dims(q, layout)
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
-        if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != q.shape:
-            raise RfError(2, f"{name} must be a contiguous CPU bf16 tensor shaped like q {tuple(q.shape)}")
-    st = stream if stream is not None else torch.cuda.current_stream().cuda_stream
-    _check(LIB.rf_sparse_attention_host(_ptr(q), _ptr(k), _ptr(v), LAYOUTS.get(layout, -1), B, S, N, D, txt_len,
-                                        *latent, block_size, float(sparsity), _scale(scale), _ptr(out),
-                                        ctypes.c_void_p(st)))
+    if out is None:
+        raise RfError(2, "out must be a CPU tensor shaped like q")
+    _check_tensors(layout, q, k, v, out, same_kv_len=latent_k is None, host=True)
+    st = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    lay = LAYOUTS.get(layout, -1)
+    if _plain(q, precision) and latent_k is None:
+        _check(LIB.rf_sparse_attention_host(_ptr(q), _ptr(k), _ptr(v), lay, B, S, N, D, txt_len, *latent,
+                                            block_size, float(sparsity), _scale(scale), _ptr(out), st))
+    else:
+        _check(LIB.rf_sparse_attention_host_ex(_ptr(q), _ptr(k), _ptr(v), _dtype(q), _prec(precision), lay, B, S, N,
+                                               D, txt_len, *latent, *_kv(k, layout, latent_k), block_size,
+                                               float(sparsity), _scale(scale), _ptr(out), st))
     return out
 
 

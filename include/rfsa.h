@@ -31,8 +31,9 @@
  *  - scale <= 0 or NaN selects head_dim ** -0.5.
  *  - Argument errors are returned before anything is enqueued.  Work is
  *    enqueued on `stream` (NULL = legacy default stream) and is asynchronous;
- *    launch failures return RF_ERR_CUDA.  Nothing here synchronises the
- *    device except rf_read_status and rf_sparse_attention_host.
+ *    launch failures return RF_ERR_CUDA.  Nothing here synchronises except
+ *    rf_read_status and rf_read_stats(_ex) (the stream given) and
+ *    rf_sparse_attention_host(_ex) (its streams).
  *  - A device-side wait that runs past its time limit makes the kernel
  *    record RF_ERR_TIMEOUT in the workspace status word and return early;
  *    rf_read_status reports it.
@@ -186,7 +187,7 @@ size_t rf_workspace_size_ex(rf_precision_t precision, int B, int S, int N, int D
  * with a workspace cached by the library per device
  * (grown with cudaMalloc on first use of a larger shape; never shrunk).  The
  * cached buffers are shared by rf_sparse_attention, rf_sparse_attention_ex
- * (NULL workspace) and rf_sparse_attention_host on a device: calls from
+ * (NULL workspace) and rf_sparse_attention_host(_ex) on a device: calls from
  * several host threads to the same device must be serialised by the caller,
  * and device calls must be ordered on one stream. */
 rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S, int N,
@@ -275,6 +276,19 @@ rf_status_t rf_sparse_attention_host(const void* q_host, const void* k_host, con
                                      int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
                                      int latent_w, int block_size, float sparsity, float scale, void* out_host,
                                      void* stream);
+/* Library: rf_sparse_attention_host for any input type, precision and
+ * key/value geometry, with the arguments and rules of rf_sparse_attention_ex
+ * (host buffers of 16-bit values in the caller's layout; k_host and v_host
+ * hold S_kv tokens when S_kv > 0).  The same chunked pipeline: the heads
+ * are independent in every precision (an fp8 block scale belongs to one
+ * head's tile, vmax to one head), so the result equals the device call on
+ * the whole tensors bit for bit.  rf_sparse_attention_host is this with
+ * RF_BF16, RF_PREC_NATIVE and S_kv = 0. */
+rf_status_t rf_sparse_attention_host_ex(const void* q_host, const void* k_host, const void* v_host, rf_dtype_t dtype,
+                                        rf_precision_t precision, rf_layout_t layout, int B, int S, int N, int D,
+                                        int txt_len, int latent_t, int latent_h, int latent_w, int S_kv, int kv_t,
+                                        int kv_h, int kv_w, int block_size, float sparsity, float scale,
+                                        void* out_host, void* stream);
 
 /* Library: synchronises `stream`, reads the workspace status word into *status
  * (0 = fine, otherwise an rf_status_t code recorded by a kernel) and clears

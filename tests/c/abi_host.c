@@ -45,5 +45,18 @@ int main(void) {
   st = rf_sparse_attention((const void*)0x1008, (const void*)0x1000, (const void*)0x1000, RF_BSND, 1, 4096, 2, 128,
                            0, 4, 32, 32, 128, 0.5f, 0.f, (void*)0x2000, NULL);
   check(st == RF_ERR_ARG, "a q pointer off a 16-byte boundary is RF_ERR_ARG");
+
+  /* the host-buffer call of any type, precision and key geometry refuses its
+   * arguments before it copies anything */
+  static char hbuf[64];
+  st = rf_sparse_attention_host_ex(hbuf, hbuf, hbuf, (rf_dtype_t)5, RF_PREC_NATIVE, RF_BSND, 1, 4096, 2, 128, 0, 4,
+                                   32, 32, 0, 0, 0, 0, 128, 0.5f, 0.f, hbuf, NULL);
+  check(st == RF_ERR_ARG, "host call: an unknown input type is RF_ERR_ARG");
+  st = rf_sparse_attention_host_ex(hbuf, NULL, hbuf, RF_F16, RF_PREC_FP8, RF_BSND, 1, 4096, 2, 128, 0, 4, 32, 32, 0,
+                                   0, 0, 0, 128, 0.5f, 0.f, hbuf, NULL);
+  check(st == RF_ERR_ARG, "host call: a NULL host buffer is RF_ERR_ARG");
+  st = rf_sparse_attention_host_ex(hbuf, hbuf, hbuf, RF_BF16, RF_PREC_NATIVE, RF_BNSD, 1, 4096, 2, 128, 0, 4, 32, 32,
+                                   5000, 5, 32, 32, 128, 0.5f, 0.f, hbuf, NULL);
+  check(st == RF_ERR_ARG, "host call: S_kv other than txt_len + t h w is RF_ERR_ARG");
   return fails ? 1 : 0;
 }
