@@ -24,6 +24,9 @@ CUDA library takes the same one; the two share no code):
       output element a worst-case bound and an error scale, both computed
       from the oracle's own weights (see there for the derivation).
 
+Parity unpinned: R14's choice of block and of rounding (a reading; the
+e4m3 format itself is pinned against torch's cast).
+
 The e4m3 format (OCP 8-bit floating point, E4M3): 1 sign bit, 4 exponent
 bits with bias 7, 3 mantissa bits; exponent field 0 holds subnormals
 m * 2^-9; no infinities; exponent 15 with mantissa 7 is NaN, so the largest
@@ -109,7 +112,7 @@ def internal_tiles(g: rf_v2.Geometry, dense: bool | None = None) -> list[np.ndar
     """Token indices of each 128-row block of the internal layout, -1 for the
     zero pad rows: the prefix in order (the whole sequence when dense),
     padded to a multiple of 128, then the sparse blocks.  ``dense``
-    overrides g.dense (a call is dense when either geometry is, R9)."""
+    overrides g.dense (a call is dense when either geometry is, R10)."""
     dense = g.dense if dense is None else dense
     pre = np.arange(g.S) if dense else np.asarray(g.prefix, dtype=np.int64)
     pad = (-len(pre)) % rf_v2.BLOCK

@@ -23,25 +23,41 @@ is the same one the CUDA library implements (the two share no code):
      partial block; its tokens join the always-kept prefix (the "suffix").
   R3 first-frame blocks (blocks holding any token of frame 0) are both
      dense query blocks and key blocks that every query block keeps.
-  R4 pooling is the mean over the block's 128 tokens; prefix rows are not
+  R4 when frame 0 is not a whole number of blocks, every block holding one
+     of its tokens counts: ceil(Ha * Wa / 128) first-frame blocks.
+  R5 pooling is the mean over the block's 128 tokens; prefix rows are not
      pooled.  The score is the plain dot product of pooled vectors.
-  R5 kept count k = nb - floor(sparsity * nb + 1e-6), i.e. the dropped
+  R6 kept count k = nb - floor(sparsity * nb + 1e-6), i.e. the dropped
      count rounds down; sparsity 0 keeps every block.
-  R6 equal scores are ranked by the lower block index.
-  R7 prefix rows (text, promoted, partial-block suffix) attend to every
+  R7 equal scores are ranked by the lower block index.
+  R8 sparsity 1 is accepted: k = 0 leaves the prefix and the first-frame
+     blocks.
+  R9 prefix rows (text, promoted, partial-block suffix) attend to every
      key; every query attends to every prefix key.
-  R8 fewer than 32 sparse blocks, or no geometry, means dense attention
+  R10 fewer than 32 sparse blocks, or no geometry, means dense attention
      over the whole sequence.
-  R9 a key/value geometry of its own ([SA] ``latent_shape_k``, which
+  R11 the top-k is decided on fp32 scores: pooled means summed in fp64 and
+     rounded to fp32, dot products in fp64 rounded to fp32.
+  R13 every (batch, head) has its own mask; the permutation is shared.
+  R17 a key/value geometry of its own ([SA] ``latent_shape_k``, which
      defaults to the query's): queries are reordered, pooled and blocked by
      the query geometry, keys and values by theirs, and both share txt_len.
-     Block scores are nb_q x nb_k; k counts key blocks (R5 over nb_k); the
+     Block scores are nb_q x nb_k; k counts key blocks (R6 over nb_k); the
      forced columns are the key geometry's first-frame blocks and the dense
      rows the query geometry's; every query attends to the key prefix.  If
-     either side is dense (R8), the call is dense attention.
+     either side is dense (R10), the call is dense attention.
+
+(R12, the output's rounding, is the kernel's; R14 and R15, the fp8
+quantisation and the rounding of its softmax weights, are in ``fp8.py``;
+R16, fp16 inputs, takes this same path.)
 
 Parity status of each function is stated in its docstring; the pins live in
-``tests/test_oracle_*.py``.
+``tests/test_oracle_*.py``.  Parity unpinned: R1, R2, R4 beyond the
+MiniMax-H3 count, R6 beyond sparsity 0 and 0.5 with an even block count,
+R7, the key-column half of R3 and the pairing rules of R17 (its sparsity-0
+and dense cases are pinned to rectangular softmax attention).  These are
+readings, not facts the pages fix: the oracle states each once and the CUDA
+path follows it.
 """
 
 from __future__ import annotations
@@ -68,7 +84,7 @@ class Geometry:
     T: int
     H: int
     W: int
-    dense: bool            # R8 fallback: every row attends to every key
+    dense: bool            # R10 fallback: every row attends to every key
     prefix: np.ndarray     # token indices of the always-kept prefix, in order
     blocks: np.ndarray     # [nb, 128] token indices of each sparse block
     first_frame: np.ndarray  # [nb] bool: block holds a token of frame 0
@@ -99,7 +115,7 @@ def geometry(S: int, txt_len: int, T: int, H: int, W: int) -> Geometry:
     """
     n_video = T * H * W
     if n_video == 0:
-        # No geometry: everything is prefix and dense (R8).
+        # No geometry: everything is prefix and dense (R10).
         return Geometry(S, txt_len, T, H, W, True, np.arange(S), np.zeros((0, BLOCK), np.int64),
                         np.zeros(0, bool), np.zeros(0, np.int64), np.zeros(0, np.int64))
     assert S == txt_len + n_video, "sequence length must be txt_len + t*h*w"
@@ -124,12 +140,12 @@ def geometry(S: int, txt_len: int, T: int, H: int, W: int) -> Geometry:
     first_frame = (t_pi[: nb * BLOCK].reshape(nb, BLOCK) == 0).any(axis=1)   # R3
 
     prefix = np.concatenate([np.arange(txt_len), promoted, tail]).astype(np.int64)
-    dense = nb < MIN_SPARSE_BLOCKS                      # R8: the partition is kept, every row is dense
+    dense = nb < MIN_SPARSE_BLOCKS                      # R10: the partition is kept, every row is dense
     return Geometry(S, txt_len, T, H, W, dense, prefix, blocks, first_frame, promoted, tail)
 
 
 def kept_count(nb: int, sparsity: float) -> int:
-    """R5: number of top-scoring key blocks each sparse query block keeps.
+    """R6: number of top-scoring key blocks each sparse query block keeps.
 
     [RF] "Configuration": sparsity is the nominal dropped fraction of key
     blocks, 0 disables sparsity.  [SA] ``sparsity``: 0.5 prunes half the KV
@@ -147,7 +163,7 @@ def kept_count(nb: int, sparsity: float) -> int:
 # ---------------------------------------------------------------------------
 
 def pool_blocks(x: np.ndarray, blocks: np.ndarray) -> np.ndarray:
-    """R4: mean of each block's rows.  ``x`` is [S, D] for one (b, head).
+    """R5: mean of each block's rows.  ``x`` is [S, D] for one (b, head).
 
     [RF] intro: key blocks of 128 tokens are pooled; [SA] pipeline: block
     pooling.  Sum in fp64, divide by the block size, round to fp32 (the
@@ -158,7 +174,7 @@ def pool_blocks(x: np.ndarray, blocks: np.ndarray) -> np.ndarray:
 
 
 def block_scores(qbar: np.ndarray, kbar: np.ndarray) -> np.ndarray:
-    """R4: s_ij = qbar_i . kbar_j, fp64 sum over fp32 inputs, rounded to fp32.
+    """R5: s_ij = qbar_i . kbar_j, fp64 sum over fp32 inputs, rounded to fp32.
 
     [RF] intro: pooled key blocks are ranked per query block.  The softmax
     scale is positive and left out: it does not change the ranking.
@@ -172,11 +188,11 @@ def topk_mask(scores: np.ndarray, k: int, first_frame: np.ndarray, first_frame_c
     [SA] pipeline: top-k sparse mask generation; [RF] intro: attend to the
     highest-scoring blocks; first-frame blocks stay dense (R3).  Row i keeps
     the first k blocks of j = 0..nb-1 ordered by (score descending, j
-    ascending) (R6), plus every first-frame block; a first-frame query row
+    ascending) (R7), plus every first-frame block; a first-frame query row
     keeps all blocks.  ``margin[i]`` = (s_(k) - s_(k+1)) / max(|s_(k)|, 1e-30)
     over the sorted row (inf when k is 0 or nb, or for first-frame rows).
 
-    With a key geometry of its own (R9) the matrix is nb_q x nb_k:
+    With a key geometry of its own (R17) the matrix is nb_q x nb_k:
     ``first_frame`` marks the dense rows, ``first_frame_cols`` (default:
     the same) the forced columns.
 
@@ -202,14 +218,14 @@ def topk_mask(scores: np.ndarray, k: int, first_frame: np.ndarray, first_frame_c
 
 
 def is_dense(g: Geometry, gk: Geometry | None = None) -> bool:
-    """R8, R9: dense attention when either side is."""
+    """R10, R17: dense attention when either side is."""
     return g.dense or (gk is not None and gk.dense)
 
 
 def build_mask(q_bnsd: np.ndarray, k_bnsd: np.ndarray, g: Geometry, sparsity: float, gk: Geometry | None = None):
     """Block mask for every (b, head): [B, N, nb_q, nb_k] bool and margins [B, N, nb_q].
 
-    ``gk`` is the key geometry (R9); None means the query's."""
+    ``gk`` is the key geometry (R17); None means the query's."""
     B, N = q_bnsd.shape[:2]
     gk = g if gk is None else gk
     mask = np.ones((B, N, g.nb, gk.nb), dtype=bool)
@@ -234,8 +250,8 @@ def key_set(g: Geometry, mask_bn: np.ndarray, row_block: int | None, gk: Geometr
     """Token indices (of the key sequence) a query attends to.
 
     ``row_block`` is the query geometry's sparse block holding the query, or
-    None for a prefix (dense) query; ``gk`` the key geometry (R9, default
-    the query's).  R7: prefix queries and first-frame blocks see every key;
+    None for a prefix (dense) query; ``gk`` the key geometry (R17, default
+    the query's).  R9: prefix queries and first-frame blocks see every key;
     a sparse query block sees the key prefix plus its kept key blocks.
     """
     gk = g if gk is None else gk
@@ -261,7 +277,7 @@ def attention_rows(qh, kh, vh, g: Geometry, mask_bn, scale: float, rows=None, ch
     caller's token order, so the inverse reorder ([SA] pipeline, last step)
     is implicit: row r of the result is token r.  ``rows`` restricts the
     output to the given token indices (all when None).  ``gk`` is the key
-    geometry (R9; None: the query's); kh and vh then have its length.
+    geometry (R17; None: the query's); kh and vh then have its length.
 
     Parity: the dense case is pinned against torch's scaled-dot-product
     attention; masked cases against the same routine given an explicit
@@ -323,7 +339,7 @@ def rf_sparse_attention(q, k, v, layout: str, txt_len: int, latent, sparsity: fl
 
     ``q, k, v`` are float arrays (bf16 values widened) in BSND or BNSD.
     [SA] ``scale`` defaults to head_dim ** -0.5; [SG] and [RF] bound
-    sparsity to [0, 1].  ``latent_k`` ([SA] ``latent_shape_k``, R9) gives k
+    sparsity to [0, 1].  ``latent_k`` ([SA] ``latent_shape_k``, R17) gives k
     and v a geometry of their own; the returned geometry is then the pair
     (query, key).
     """

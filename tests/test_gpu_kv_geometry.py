@@ -1,5 +1,5 @@
 """Parity of calls whose keys and values have a geometry of their own
-(lite_boost.ops.sparse_attention, latent_shape_k; oracle reading R9) with the
+(lite_boost.ops.sparse_attention, latent_shape_k; oracle reading R17) with the
 CPU oracle: the rectangular block mask bit for bit (near-ties excused), the
 output within max-abs 2e-2 / mean-abs 2e-3 (bf16, fp16) or the fp8 bounds,
 the fp8 codes and scales of each side bit for bit."""

@@ -359,7 +359,7 @@ def test_sparsity_range_is_checked():
         oracle.to_bnsd(q, "SBND")
 
 
-# ---------------------------------------------------------------- a key geometry of its own (R9)
+# ---------------------------------------------------------------- a key geometry of its own (R17)
 
 def test_key_geometry_equal_to_query_changes_nothing():
     txt, T, H, W, D = 16, 4, 32, 40, 128
