@@ -63,30 +63,29 @@ def _peaks():
 
 def _stages(w, plan, prec, ms_prepare, ms_attention, k3_tflops, hbm_gbs, ms_k1=None):
     """Per-stage times with the HBM-bound stages' algorithmic bytes: K1 reads q, k, v in the caller's layout and
-    writes the internal copies plus the fp32 block means of q and k, K2 reads the block means and writes the
-    mask, kept counts and margins; fp8 adds the quantisation pass (reads the internal copies, writes e4m3 codes
-    and one fp32 scale per 128-row block).  ``ms_k1`` (K1 alone, from the library's stage event) splits the
-    prepare stage into K1 and the kernels after it."""
+    writes the internal copies (fp8: e4m3 codes and one fp32 scale per 128-row tile) plus the fp32 block means
+    of q and k, K2 reads the block means and writes the mask, kept counts and margins.  ``ms_k1`` (K1 alone,
+    from the library's stage event) splits the prepare stage into K1 and the kernel after it."""
     heads = w.B * w.N
     row = 128 * 2                                          # one token's head vector, bytes
     pooled = 2 * plan.nb * 128 * 4                         # q and k block means, bytes per head
     words = (plan.nb + 31) // 32
-    k1 = heads * (3 * w.S * row + 3 * plan.S_int * row + pooled)
+    written = 3 * plan.S_int * 128 + 3 * plan.n_tiles * 4 if prec == "fp8" else 3 * plan.S_int * row
+    k1 = heads * (3 * w.S * row + written + pooled)
     k2 = heads * (pooled + plan.nb * (words * 4 + 8))
-    kq = heads * (3 * plan.S_int * row + 3 * plan.S_int * 128 + 3 * plan.n_tiles * 4) if prec == "fp8" else 0
-    moved = k1 + k2 + kq
+    moved = k1 + k2
     gbs = moved / (ms_prepare * 1e-3) / 1e9
-    out = {"prepare": {"kernels": "K1 reorder + block means, K2 block scores + top-k" +
-                       (", Kq e4m3 quantisation" if prec == "fp8" else ""),
+    k1_name = "K1 reorder + block means" + (" + e4m3 codes" if prec == "fp8" else "")
+    out = {"prepare": {"kernels": k1_name + ", K2 block scores + top-k",
                        "ms": ms_prepare, "algorithmic_bytes": moved, "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs}}
     if ms_k1 is not None and 0 < ms_k1 < ms_prepare:
         g1 = k1 / (ms_k1 * 1e-3) / 1e9
         rest = ms_prepare - ms_k1
-        g2 = (k2 + kq) / (rest * 1e-3) / 1e9
-        out["permute_pool"] = {"kernels": "K1 reorder + block means", "ms": ms_k1, "algorithmic_bytes": k1,
+        g2 = k2 / (rest * 1e-3) / 1e9
+        out["permute_pool"] = {"kernels": k1_name, "ms": ms_k1, "algorithmic_bytes": k1,
                                "gbs": g1, "frac_of_hbm": g1 / hbm_gbs}
-        out["after_permute_pool"] = {"kernels": "K2" + (" + Kq" if prec == "fp8" else ""), "ms": rest,
-                                     "algorithmic_bytes": k2 + kq, "gbs": g2, "frac_of_hbm": g2 / hbm_gbs}
+        out["after_permute_pool"] = {"kernels": "K2", "ms": rest,
+                                     "algorithmic_bytes": k2, "gbs": g2, "frac_of_hbm": g2 / hbm_gbs}
     out["attention"] = {"kernels": "K3", "ms": ms_attention, "tflops": k3_tflops}
     return out
 
@@ -501,7 +500,7 @@ def _ulysses_timed(args, w, dist, rfsa, synth, ulysses, world, rank, local, dev)
                            "query_blocks": int(query_blocks), "near_ties": int(near),
                            "near_tie_rule": "k-th and (k+1)-th block scores within 1e-5 (relative)"},
             # per rank and step: K1, K2, K3 and its second pass (the exchanges are NCCL's kernels)
-            "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
+            "gpu_launches": 4 * args.steps,
             "stages": {"all_to_all_in": {"ms": a2a_in, "bytes_per_rank": 3 * shard_bytes * (world - 1) / world},
                        "call": {"ms": call, "heads_per_rank": Nl},
                        "attention": {"kernels": "K3", "ms": k3, "tflops_per_rank": k3_tflops_rank},
@@ -660,8 +659,8 @@ def main():
                                   if args.dtype == "bf16" and w.name == "minimax" else None),
             "mask_stats": _mask_stats(stats, plan),
             # K1, K2 and K3 (the chain kernel and its second pass, which returns at once when no unit was
-            # handed to it); fp8 adds the quantisation pass
-            "gpu_launches": (5 if prec == "fp8" else 4) * args.steps,
+            # handed to it)
+            "gpu_launches": 4 * args.steps,
             "stages": _stages(w, plan, prec, statistics.mean(k1k2), k3_ms, k3_tflops, peaks["hbm_gbs"],
                               statistics.mean(k1)),
             "clocks": clocks.summary(),

@@ -288,15 +288,16 @@ rf_status_t rf_workspace_layout_ex(rf_precision_t precision, int B, int N, int D
   // the work counter and the status word first: their places depend on nothing
   L.counter = take(4);
   L.status = take(4);
-  L.q_int = take(rows_q * RF_HEAD_DIM * 2);
-  L.k_int = take(rows_k * RF_HEAD_DIM * 2);
-  L.v_int = take(rows_k * RF_HEAD_DIM * 2);
+  // the 16-bit internal copies: native precision only (fp8 stage 1 writes e4m3 codes instead)
+  const bool fp8 = precision == RF_PREC_FP8;
+  L.q_int = take(fp8 ? 0 : rows_q * RF_HEAD_DIM * 2);
+  L.k_int = take(fp8 ? 0 : rows_k * RF_HEAD_DIM * 2);
+  L.v_int = take(fp8 ? 0 : rows_k * RF_HEAD_DIM * 2);
   L.pooled_q = take(heads * g->nb * RF_HEAD_DIM * 4);
   L.pooled_k = take(heads * gk->nb * RF_HEAD_DIM * 4);
   L.mask = take(heads * g->nb * gk->mask_words * 4);
   L.kept = take(heads * g->nb * 4);
   L.margin = take(heads * g->nb * 4);
-  const bool fp8 = precision == RF_PREC_FP8;
   L.q8 = take(fp8 ? rows_q * RF_HEAD_DIM : 0);
   L.k8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
   L.v8 = take(fp8 ? rows_k * RF_HEAD_DIM : 0);
@@ -344,9 +345,14 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
   if ((st = check_ws(ws, ws_bytes, L)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   NvtxRange range("rf prepare: K1 reorder + block means, K2 scores + top-k");
-  cudaError_t e = rf::launch_permute_pool(q, k, v, dtype, layout, B, S, gk.S, N, g, gk, at<void>(ws, L.q_int),
-                                          at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
-                                          at<float>(ws, L.pooled_k), s);
+  cudaError_t e =
+      precision == RF_PREC_FP8
+          ? rf::launch_permute_pool_fp8(q, k, v, dtype, layout, B, S, gk.S, N, g, gk, at<uint8_t>(ws, L.q8),
+                                        at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8), at<float>(ws, L.scales),
+                                        at<float>(ws, L.vmax), at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), s)
+          : rf::launch_permute_pool(q, k, v, dtype, layout, B, S, gk.S, N, g, gk, at<void>(ws, L.q_int),
+                                    at<void>(ws, L.k_int), at<void>(ws, L.v_int), at<float>(ws, L.pooled_q),
+                                    at<float>(ws, L.pooled_k), s);
   if (e != cudaSuccess) return cuda_fail(e, "permute/pool launch");
   cudaEvent_t stage_event;
   {
@@ -357,12 +363,6 @@ rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_
   e = rf::launch_mask(at<float>(ws, L.pooled_q), at<float>(ws, L.pooled_k), B * N, g, gk, at<uint32_t>(ws, L.mask),
                       at<int>(ws, L.kept), at<float>(ws, L.margin), s);
   if (e != cudaSuccess) return cuda_fail(e, "mask launch");
-  if (precision == RF_PREC_FP8) {
-    e = rf::launch_quantize_fp8(at<void>(ws, L.q_int), at<void>(ws, L.k_int), at<void>(ws, L.v_int), dtype, B * N, g,
-                                gk, at<uint8_t>(ws, L.q8), at<uint8_t>(ws, L.k8), at<uint8_t>(ws, L.v8),
-                                at<float>(ws, L.scales), at<float>(ws, L.vmax), s);
-    if (e != cudaSuccess) return cuda_fail(e, "fp8 quantisation launch");
-  }
   return ok();
 }
 

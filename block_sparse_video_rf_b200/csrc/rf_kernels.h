@@ -16,6 +16,17 @@ cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int
                                 int Sk, int N, const rf_plan_t& g, const rf_plan_t& gk, void* q_int, void* k_int,
                                 void* v_int, float* pooled_q, float* pooled_k, cudaStream_t stream);
 
+// K1 at the fp8 precision (RF_PREC_FP8): the same reorder and block means,
+// with the reordered tiles written as e4m3 codes instead of 16-bit rows: per
+// (tensor, head, 128-row tile) scale = amax / 448 and codes of x * 448 / amax;
+// V's tiles stored transposed; scales = q [BN, g.n_tiles], then k and v
+// [BN, gk.n_tiles]; vmax[bn] = the largest V tile scale of head bn (zeroed
+// here first).
+cudaError_t launch_permute_pool_fp8(const void* q, const void* k, const void* v, int dtype, int layout, int B, int S,
+                                    int Sk, int N, const rf_plan_t& g, const rf_plan_t& gk, uint8_t* q8, uint8_t* k8,
+                                    uint8_t* v8, float* scales, float* vmax, float* pooled_q, float* pooled_k,
+                                    cudaStream_t stream);
+
 // K4: inverse reorder of an internal-order tensor into the caller's layout.
 cudaError_t launch_unpermute(const void* o_int, int layout, int B, int S, int N, const rf_plan_t& g, void* out,
                              cudaStream_t stream);
@@ -52,15 +63,7 @@ cudaError_t launch_attention_slots(const void* q_int, const void* k_int, const v
                                    const rf_plan_t& gk, float scale, void* out, int* counter, int* status, int* redo,
                                    int list_mode, const AttnDebug& dbg, cudaStream_t stream);
 
-// fp8 quantisation of the reordered q (plan g), k and v (plan gk)
-// (RF_PREC_FP8): per (tensor, head, 128-row block) scale = amax / 448 and
-// e4m3 codes; V's blocks stored transposed; scales = q [BN, g.n_tiles], k and
-// v [BN, gk.n_tiles]; vmax[bn] = the largest V block scale of head bn.
-cudaError_t launch_quantize_fp8(const void* q_int, const void* k_int, const void* v_int, int dtype, int BN,
-                                const rf_plan_t& g, const rf_plan_t& gk, uint8_t* q8, uint8_t* k8, uint8_t* v8,
-                                float* scales, float* vmax, cudaStream_t stream);
-
-// K3 on the e4m3 tensors of launch_quantize_fp8; output in dtype.  As
+// K3 on the e4m3 tensors of launch_permute_pool_fp8; output in dtype.  As
 // launch_attention: chain_kernel, then attn_kernel over the units it lists
 // (P above e4m3's 448).
 cudaError_t launch_attention_fp8(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, const float* scales,

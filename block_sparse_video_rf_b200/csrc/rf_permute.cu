@@ -5,6 +5,16 @@
 // pooling; inverse reorder at the end.  vllm-omni "RainFusion Attention":
 // 128-token key blocks are pooled (intro); the reorder groups video tokens
 // into 8x8 tiles and promotes the non-aligned rest ("Geometry handling").
+//
+// At the fp8 precision (lite_boost.ops.sparse_attention lists one; the pages
+// fix no scaling rule) K1 writes the reordered tiles as e4m3 codes instead
+// of 16-bit copies.  The reading taken: one fp32 scale per 128-row tile of
+// the internal layout, per tensor and head (the attention's own tile),
+// scale = amax(|x|) / 448 with 448 the largest finite e4m3 value, code =
+// e4m3 round-to-nearest-even, saturating, of x * (448 / amax) in fp32; an
+// all-zero tile has scale 0 and codes 0.  V's tiles are stored transposed
+// (channel-major) so that the P V product reads them K-major, and vmax[head]
+// is the largest V tile scale of the head.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -12,6 +22,7 @@
 #include "rf_dtype.h"
 #include "rf_geometry.h"
 #include "rf_kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace rf {
 
@@ -89,6 +100,148 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(PermArgs a, 
   a.pooled[t][((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c] = s * (1.0f / RF_BLOCK);
 }
 
+// fp8 form: e4m3 codes and tile scales in place of the 16-bit copies.
+constexpr int kVtStride = RF_BLOCK + 4;   // bytes per transposed row in shared memory
+
+struct PermArgs8 {
+  const uint16_t* src[3];
+  uint8_t* dst[3];    // e4m3 codes, internal layout (the v_index tensor's tiles transposed)
+  float* scales[3];   // [BN, n_tiles] tile scales of each tensor
+  float* pooled[2];   // block means of tensors 0 and 1 (nullptr: not pooled)
+  int count;          // tensors in use
+  int v_index;        // the transposed tensor, whose largest tile scale goes to vmax (-1: none)
+  float* vmax;        // [BN], zero before the launch
+};
+
+// One CTA = one 128-row internal tile of one (b, head), for each tensor in
+// turn: its rows gathered (8 16-byte loads in flight per thread), the tile's
+// amax behind one barrier, then its codes.  Few registers, so that several
+// CTAs share an SM and hide the barriers.  Block means as permute_pool_kernel,
+// summed in the same order.
+template <bool kF16>
+__global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermArgs8 a, int layout, int B, int S,
+                                                                           int N, rf_plan_t g) {
+  __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
+  __shared__ float red_max[3][kPermThreads / 32];
+  __shared__ __align__(16) uint8_t vt[RF_HEAD_DIM][kVtStride];
+  const int tile = blockIdx.x;
+  const int bn = blockIdx.y;
+  const int b = bn / N, n = bn - b * N;
+  const int chunk = threadIdx.x & 15;     // 16-byte column chunk
+  const int rsub = threadIdx.x >> 4;      // row within the pass
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool sparse = (tile * RF_BLOCK >= g.P_pad) && !g.dense;
+  int src[kPasses];   // token of each of the thread's rows (-1: pad row)
+#pragma unroll
+  for (int p = 0; p < kPasses; ++p) src[p] = rf_src_of_row(g, tile * RF_BLOCK + p * kRowsPerPass + rsub);
+  const int64_t code_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM;
+  // every tensor's rows requested into L2 at once (one request per 128-byte
+  // line, no registers held), so that the tile's DRAM reads overlap the
+  // tensor-by-tensor work below
+  if ((chunk & 7) == 0) {
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      if (t >= a.count) break;
+      const uint16_t* in = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
+#pragma unroll
+      for (int p = 0; p < kPasses; ++p)
+        if (src[p] >= 0) prefetch_l2(in + rf_token_offset(layout, B, S, N, b, n, src[p]) + chunk * 8);
+    }
+  }
+
+#pragma unroll 1
+  for (int t = 0; t < a.count; ++t) {
+    // the tensor's pointers, chosen with constant indices (a runtime index
+    // into the parameter arrays would copy them to local memory)
+    const uint16_t* in = t == 0 ? a.src[0] : t == 1 ? a.src[1] : a.src[2];
+    uint8_t* codes = t == 0 ? a.dst[0] : t == 1 ? a.dst[1] : a.dst[2];
+    float* scales = t == 0 ? a.scales[0] : t == 1 ? a.scales[1] : a.scales[2];
+    float* pooled = t == 0 ? a.pooled[0] : t == 1 ? a.pooled[1] : nullptr;
+    uint4 buf[kPasses];
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p)
+      buf[p] = src[p] < 0 ? make_uint4(0, 0, 0, 0)
+                          : __ldcs(reinterpret_cast<const uint4*>(
+                                in + rf_token_offset(layout, B, S, N, b, n, src[p]) + chunk * 8));
+    // amax on the packed values: for finite bf16 and fp16 alike, |x| orders
+    // like the integer bits & 0x7FFF, so a per-half unsigned max finds it
+    // exactly (nothing unpacked stays live across the barrier)
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p)
+      m2 = __vmaxu2(__vmaxu2(m2, buf[p].x & 0x7FFF7FFFu), __vmaxu2(buf[p].y & 0x7FFF7FFFu, 0u)),
+      m2 = __vmaxu2(m2, __vmaxu2(buf[p].z & 0x7FFF7FFFu, buf[p].w & 0x7FFF7FFFu));
+    const uint32_t mbits = max(m2 & 0xFFFFu, m2 >> 16);
+    float amax;
+    if (kF16)
+      amax = __half2float(__ushort_as_half((unsigned short)mbits));
+    else
+      amax = __uint_as_float(mbits << 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    if (lane == 0) red_max[t][warp] = amax;
+    __syncthreads();
+    amax = red_max[t][0];
+#pragma unroll
+    for (int i = 1; i < kPermThreads / 32; ++i) amax = fmaxf(amax, red_max[t][i]);
+    const float inv = amax > 0.f ? __fdiv_rn(448.f, amax) : 0.f;
+    const float scale = __fdiv_rn(amax, 448.f);
+    const bool transposed = t == a.v_index;
+    const bool pool = sparse && pooled;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // the block means' partial sums
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) {
+      if (pool) acc_half8<kF16>(acc, buf[p]);
+      float f[8];
+      unpack_half8<kF16>(buf[p], f);
+      const int r = p * kRowsPerPass + rsub;
+      const uint32_t lo = pack_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
+                                      __fmul_rn(f[3], inv));
+      const uint32_t hi = pack_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
+                                      __fmul_rn(f[7], inv));
+      if (!transposed) {
+        *reinterpret_cast<uint2*>(codes + code_base + (int64_t)r * RF_HEAD_DIM + chunk * 8) = make_uint2(lo, hi);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          vt[chunk * 8 + i][r] = (uint8_t)(lo >> (8 * i));
+          vt[chunk * 8 + 4 + i][r] = (uint8_t)(hi >> (8 * i));
+        }
+      }
+    }
+    if (pool) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) red[t][rsub][chunk * 8 + i] = acc[i];
+    }
+    if (threadIdx.x == 0) {
+      scales[(int64_t)bn * g.n_tiles + tile] = scale;
+      // non-negative floats order like their bit patterns
+      if (transposed) atomicMax(reinterpret_cast<int*>(a.vmax) + bn, __float_as_int(scale));
+    }
+  }
+  __syncthreads();   // the transposed V tile and the block means' partial sums are in place
+  if (a.v_index >= 0) {
+    // the transposed V tile: 128 channel rows of 128 bytes, one word per thread and step
+    uint8_t* codes = a.v_index == 1 ? a.dst[1] : a.dst[2];
+#pragma unroll
+    for (int i = 0; i < RF_HEAD_DIM * RF_BLOCK / 4 / kPermThreads; ++i) {
+      const int idx = threadIdx.x + i * kPermThreads;
+      const int row = idx >> 5, word = idx & 31;
+      *reinterpret_cast<uint32_t*>(codes + code_base + (int64_t)row * RF_BLOCK + word * 4) =
+          *reinterpret_cast<const uint32_t*>(&vt[row][word * 4]);
+    }
+  }
+  if (!sparse) return;
+  const int t = threadIdx.x >> 7, c = threadIdx.x & 127;
+  float* pooled = t == 0 ? a.pooled[0] : a.pooled[1];
+  if (t >= a.count || !pooled) return;
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRowsPerPass; ++i) s += red[t][i][c];
+  const int blk = tile - g.P_pad / RF_BLOCK;
+  pooled[((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c] = s * (1.0f / RF_BLOCK);
+}
+
 __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const uint16_t* __restrict__ o_int, int layout, int B,
                                                                  int S, int N, rf_plan_t g,
                                                                  uint16_t* __restrict__ out) {
@@ -129,6 +282,33 @@ cudaError_t launch_permute_pool(const void* q, const void* k, const void* v, int
   if (e != cudaSuccess) return e;
   a = PermArgs{{s16(k), s16(v), nullptr}, {d16(k_int), d16(v_int), nullptr}, {pooled_k, nullptr}, 2};
   kern<<<dim3(gk.n_tiles, B * N), kPermThreads, 0, stream>>>(a, layout, B, Sk, N, gk);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_pool_fp8(const void* q, const void* k, const void* v, int dtype, int layout, int B, int S,
+                                    int Sk, int N, const rf_plan_t& g, const rf_plan_t& gk, uint8_t* q8, uint8_t* k8,
+                                    uint8_t* v8, float* scales, float* vmax, float* pooled_q, float* pooled_k,
+                                    cudaStream_t stream) {
+  const int BN = B * N;
+  cudaError_t e = cudaMemsetAsync(vmax, 0, sizeof(float) * BN, stream);
+  if (e != cudaSuccess) return e;
+  auto kern = dtype == RF_F16 ? permute_pool_fp8_kernel<true> : permute_pool_fp8_kernel<false>;
+  auto s16 = [](const void* x) { return static_cast<const uint16_t*>(x); };
+  float* sq = scales;
+  float* sk = sq + (size_t)BN * g.n_tiles;
+  float* sv = sk + (size_t)BN * gk.n_tiles;
+  if (S == Sk && std::memcmp(&g, &gk, sizeof(rf_plan_t)) == 0) {   // one geometry: one pass over q, k, v
+    const PermArgs8 a{{s16(q), s16(k), s16(v)}, {q8, k8, v8}, {sq, sk, sv}, {pooled_q, pooled_k}, 3, 2, vmax};
+    kern<<<dim3(g.n_tiles, BN), kPermThreads, 0, stream>>>(a, layout, B, S, N, g);
+    return cudaGetLastError();
+  }
+  const PermArgs8 aq{{s16(q), nullptr, nullptr}, {q8, nullptr, nullptr}, {sq, nullptr, nullptr},
+                     {pooled_q, nullptr}, 1, -1, vmax};
+  kern<<<dim3(g.n_tiles, BN), kPermThreads, 0, stream>>>(aq, layout, B, S, N, g);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const PermArgs8 akv{{s16(k), s16(v), nullptr}, {k8, v8, nullptr}, {sk, sv, nullptr}, {pooled_k, nullptr}, 2, 1,
+                      vmax};
+  kern<<<dim3(gk.n_tiles, BN), kPermThreads, 0, stream>>>(akv, layout, B, Sk, N, gk);
   return cudaGetLastError();
 }
 

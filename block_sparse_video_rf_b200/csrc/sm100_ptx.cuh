@@ -90,6 +90,11 @@ __device__ __forceinline__ bool rf_wait_time(uint64_t* bar, uint32_t parity, uin
 }
 
 // ---------------------------------------------------------------- TMA
+// Requests the line holding `p` into L2 (a hint: no register waits on it).
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(p)));
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

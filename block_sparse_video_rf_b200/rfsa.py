@@ -480,10 +480,9 @@ def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"
         return raw[off:off + nbytes].view(dtype).view(shape)
 
     nb, nbk, words = plan.nb, pk.nb, pk.mask_words
-    fp8 = {}
     if precision == "fp8":
         nq, nk = plan.n_tiles, pk.n_tiles
-        fp8 = {
+        copies = {
             "q8": view(lay.q8, heads * plan.S_int * 128, torch.uint8, (B, N, plan.S_int, 128)),
             "k8": view(lay.k8, heads * pk.S_int * 128, torch.uint8, (B, N, pk.S_int, 128)),
             "v8": view(lay.v8, heads * pk.S_int * 128, torch.uint8, (B, N, nk, 128, 128)),
@@ -492,10 +491,13 @@ def workspace_views(workspace, B, N, plan, dtype=None, precision: str = "native"
             "v_scales": view(lay.scales + 4 * heads * (nq + nk), heads * nk, torch.float32, (B, N, nk)),
             "vmax": view(lay.vmax, heads, torch.float32, (B, N)),
         }
-    return fp8 | {
-        "q_int": view(lay.q_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
-        "k_int": view(lay.k_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
-        "v_int": view(lay.v_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
+    else:   # the 16-bit internal copies exist at native precision only
+        copies = {
+            "q_int": view(lay.q_int, heads * plan.S_int * 128, dtype, (B, N, plan.S_int, 128)),
+            "k_int": view(lay.k_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
+            "v_int": view(lay.v_int, heads * pk.S_int * 128, dtype, (B, N, pk.S_int, 128)),
+        }
+    return copies | {
         "pooled_q": view(lay.pooled_q, heads * nb * 128, torch.float32, (B, N, nb, 128)),
         "pooled_k": view(lay.pooled_k, heads * nbk * 128, torch.float32, (B, N, nbk, 128)),
         "mask": view(lay.mask, heads * nb * words, torch.int32, (B, N, nb, words)),

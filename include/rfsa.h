@@ -116,7 +116,8 @@ typedef struct {
 } rf_plan_t;
 
 /* Library: byte offsets of the regions of a workspace (all 256-byte aligned).
- * q_int/k_int/v_int: 16-bit (input type) [B, N, S_int, 128]; pooled_q/pooled_k: fp32
+ * q_int/k_int/v_int: 16-bit (input type) [B, N, S_int, 128], native
+ * precision only (zero-sized with RF_PREC_FP8); pooled_q/pooled_k: fp32
  * [B, N, nb, 128] (block means); mask: uint32 [B, N, nb, mask_words], bit j
  * of row i set when query block i reads key block j; kept: int32 [B, N, nb]
  * (bits set per row); margin: fp32 [B, N, nb] (relative gap between the
@@ -239,8 +240,9 @@ rf_status_t rf_attend(rf_layout_t layout, int B, int S, int N, int D, int txt_le
  *   precision and geometries; rf_sparse_attention_ex takes workspace = NULL
  *   (ws_bytes ignored) to use the library's cached workspace.
  * - Invalid dtype or precision: RF_ERR_ARG.
- * - RF_PREC_FP8 stage 1 also quantises the reordered q, k, v (q8/k8/v8,
- *   scales, vmax); its stage 2 reads only those. */
+ * - RF_PREC_FP8 stage 1 writes the reordered q, k, v as e4m3 codes with
+ *   their tile scales (q8/k8/v8, scales, vmax) instead of 16-bit copies;
+ *   its stage 2 reads only those. */
 rf_status_t rf_prepare_ex(const void* q, const void* k, const void* v, rf_dtype_t dtype, rf_precision_t precision,
                           rf_layout_t layout, int B, int S, int N, int D, int txt_len, int latent_t, int latent_h,
                           int latent_w, int S_kv, int kv_t, int kv_h, int kv_w, int block_size, float sparsity,

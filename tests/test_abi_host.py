@@ -159,12 +159,17 @@ def test_fp8_workspace_layout(rfsa):
     offs = [getattr(lay, f) for f in rfsa.WS_FIELDS]
     assert all(o % 256 == 0 for o in offs)
     codes = 56 * 62848 * 128
-    assert _regions_disjoint(lay, {"q_int": 2 * codes, "v_int": 2 * codes, "q8": codes, "k8": codes, "v8": codes,
+    rows = 56 * p.nb
+    assert _regions_disjoint(lay, {"pooled_q": rows * 512, "pooled_k": rows * 512, "mask": rows * p.mask_words * 4,
+                                   "kept": rows * 4, "margin": rows * 4, "q8": codes, "k8": codes, "v8": codes,
                                    "scales": 3 * 56 * p.n_tiles * 4, "vmax": 56 * 4})
-    # the native layout is the same up to the fp8 regions, which it leaves empty; both end with the
-    # attention's redo list (two counters and one id per query tile)
-    assert [getattr(nat, f) for f in rfsa.WS_FIELDS[:10]] == offs[:10]
+    # fp8 keeps no 16-bit internal copies (zero-sized regions) and the native layout no fp8 regions; both
+    # start with the work counter and the status word and end with the attention's redo list (two counters
+    # and one id per query tile)
+    assert lay.q_int == lay.k_int == lay.v_int == lay.pooled_q
     assert nat.q8 == nat.k8 == nat.v8 == nat.scales == nat.vmax == nat.redo
+    assert (lay.counter, lay.status) == (nat.counter, nat.status)
+    assert lay.total < nat.total - 2 * codes
     for L in (nat, lay):
         assert L.total - L.redo >= (2 + 56 * p.n_tiles) * 4
     assert rfsa.rf_workspace_size(1, 62752, 56, 128, 256, (62, 24, 42), precision="fp8") == lay.total
@@ -272,9 +277,9 @@ def test_read_stats_ex_validates_before_any_cuda_call(rfsa):
     assert L.rf_read_stats_ex(5, P(0x1000), 1 << 30, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 2
     assert L.rf_read_stats_ex(1, P(0x1000), 16, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 5
     assert L.rf_read_stats_ex(1, P(0x1000), 1 << 30, 1, 2, 128, None, None, ctypes.byref(st), None) == 2
-    # the fp8 workspace is larger than the native one: a native-sized buffer is too small for it
-    nat = rfsa.rf_workspace_size(1, 4096, 2, 128, 0, (4, 32, 32))
-    assert L.rf_read_stats_ex(1, P(0x1000), nat, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 5
+    # a buffer one byte short of the fp8 workspace is refused
+    n8 = rfsa.rf_workspace_size(1, 4096, 2, 128, 0, (4, 32, 32), precision="fp8")
+    assert L.rf_read_stats_ex(1, P(0x1000), n8 - 1, 1, 2, 128, ctypes.byref(p), None, ctypes.byref(st), None) == 5
 
 
 def test_binding_checks_tensors_before_the_library(rfsa):
