@@ -197,7 +197,12 @@ rf_status_t rf_sparse_attention(const void* q, const void* k, const void* v, rf_
 
 /* Library: the whole call (as rf_sparse_attention) with a caller-owned device workspace of ws_bytes
  * (>= rf_workspace_size, 256-byte aligned).  Calls that share a workspace
- * must be ordered on one stream. */
+ * must be ordered on one stream.  With a caller-owned workspace a call (this
+ * one, rf_sparse_attention_ex, or rf_prepare(_ex) + rf_attend(_ex)) only
+ * enqueues kernels and memsets on `stream`, so it can be captured in a CUDA
+ * graph and replayed; the graph holds the buffers' addresses.  The cached
+ * workspace of rf_sparse_attention may be allocated on first use and is not
+ * for capture. */
 rf_status_t rf_sparse_attention_ws(const void* q, const void* k, const void* v, rf_layout_t layout, int B, int S,
                                    int N, int D, int txt_len, int latent_t, int latent_h, int latent_w,
                                    int block_size, float sparsity, float scale, void* out, void* workspace,
