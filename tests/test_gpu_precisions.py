@@ -151,6 +151,32 @@ def test_fp8_quantisation_is_bit_exact(rfsa, case, dtype):
     np.testing.assert_array_equal(views["vmax"].cpu().numpy(), views["v_scales"].cpu().numpy().max(axis=-1))
 
 
+CASES["ragged_b2"] = ("tiny", {"B": 2, "N": 2, "txt_len": 37, "latent": (8, 21, 43), "sparsity": 0.7, "seed": 13})
+CASES["oddtiles_bnsd_b2"] = ("tiny", {"B": 2, "txt_len": 19, "latent": (5, 24, 40), "sparsity": 0.6,
+                                      "layout": "BNSD", "seed": 14})
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("case", ["ragged_b2", "oddtiles_bnsd_b2"])
+def test_fp8_quantisation_is_bit_exact_two_batches(rfsa, case, dtype):
+    test_fp8_quantisation_is_bit_exact(rfsa, case, dtype)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+@pytest.mark.parametrize("case", ["ragged", "ragged_b2", "oddtiles_bnsd_b2", "rope_small"])
+def test_fp8_prepare_gives_the_native_mask(rfsa, case, dtype):
+    # K1's fp8 form sums the block means in the 16-bit form's order, so the
+    # means, and with them the mask, its kept counts and margins, are the
+    # native precision's bit for bit
+    name, over = CASES[case]
+    w, q, k, v = _inputs(name, dtype, **over)
+    _, _, nat = _prepare(rfsa, w, q, k, v, "native")
+    _, _, f8 = _prepare(rfsa, w, q, k, v, "fp8")
+    torch.cuda.synchronize()
+    for key in ("pooled_q", "pooled_k", "mask", "kept", "margin"):
+        assert torch.equal(nat[key].view(torch.int32), f8[key].view(torch.int32)), key
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("case", ["tiny", "text2", "ragged", "oddtiles_bnsd", "rope_small", "dense_fallback"])
 def test_fp8_attention(rfsa, case, dtype):
