@@ -40,6 +40,35 @@ RF_HD int rf_src_of_aligned(const rf_plan_t& g, int s) {
   return g.txt_len + (t * g.H + y) * g.W + x;
 }
 
+// A sparse block is two consecutive 8x8 tiles of the aligned order (tiles
+// 2 blk and 2 blk + 1): their frames and top-left corners, with two
+// divisions for the block instead of two per row.
+struct RfBlockTiles {
+  int t[2], y[2], x[2];
+};
+RF_HD RfBlockTiles rf_block_tiles(const rf_plan_t& g, int blk) {
+  const int tiles_x = g.Wa >> 3, tiles_y = g.Ha >> 3;
+  const int tiles_per_frame = tiles_y * tiles_x;
+  const int tile = 2 * blk;
+  int t = tile / tiles_per_frame;
+  const int tf = tile - t * tiles_per_frame;
+  int ty = tf / tiles_x, tx = tf - ty * tiles_x;
+  RfBlockTiles b;
+  b.t[0] = t, b.y[0] = ty << 3, b.x[0] = tx << 3;
+  if (++tx == tiles_x) {   // the next tile: the next column, row or frame
+    tx = 0;
+    if (++ty == tiles_y) ty = 0, ++t;
+  }
+  b.t[1] = t, b.y[1] = ty << 3, b.x[1] = tx << 3;
+  return b;
+}
+// Sequence index of row r (0 <= r < 128) of that block: the same as
+// rf_src_of_aligned(g, 128 blk + r).
+RF_HD int rf_src_in_block(const rf_plan_t& g, const RfBlockTiles& b, int r) {
+  const int h = r >> 6, in_tile = r & 63;
+  return g.txt_len + (b.t[h] * g.H + b.y[h] + (in_tile >> 3)) * g.W + b.x[h] + (in_tile & 7);
+}
+
 // Internal row r -> sequence index of its token, or -1 for a pad row.
 RF_HD int rf_src_of_row(const rf_plan_t& g, int r) {
   if (r < g.P) {

@@ -52,12 +52,13 @@ __global__ void __launch_bounds__(kThreads) pool_blocks_kernel(const uint16_t* _
   const int chunk = threadIdx.x & 15;
   const int rsub = threadIdx.x >> 4;
   const uint16_t* srcs[2] = {q, k};
+  const RfBlockTiles bt = rf_block_tiles(g, blk);   // the block's two 8x8 tiles
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
-      const int s = rf_src_of_row(g, g.P_pad + blk * RF_BLOCK + p * kRowsPerPass + rsub);
+      const int s = rf_src_in_block(g, bt, p * kRowsPerPass + rsub);
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(srcs[t] + rf_token_offset(layout, B, S, N, b, n, s) +
                                                            chunk * 8));
       acc_half8<kF16>(acc, u);

@@ -32,6 +32,21 @@ constexpr int kPermThreads = 256;   // 16 rows x 16 chunks of 16 bytes per pass
 constexpr int kRowsPerPass = kPermThreads / 16;
 constexpr int kPasses = RF_BLOCK / kRowsPerPass;
 
+// Token (sequence index) of each of a thread's rows of internal tile `tile`
+// (row p * kRowsPerPass + rsub; -1 for a pad row): a sparse block's rows
+// from its two 8x8 tiles (two divisions for the block), prefix rows one by
+// one.
+__device__ __forceinline__ void tile_sources(const rf_plan_t& g, int tile, int rsub, int (&src)[kPasses]) {
+  if (!g.dense && tile * RF_BLOCK >= g.P_pad) {
+    const RfBlockTiles bt = rf_block_tiles(g, tile - g.P_pad / RF_BLOCK);
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) src[p] = rf_src_in_block(g, bt, p * kRowsPerPass + rsub);
+  } else {
+#pragma unroll
+    for (int p = 0; p < kPasses; ++p) src[p] = rf_src_of_row(g, tile * RF_BLOCK + p * kRowsPerPass + rsub);
+  }
+}
+
 // Up to three tensors of one geometry (plan g, S rows in the caller's layout).
 struct PermArgs {
   const uint16_t* src[3];
@@ -57,13 +72,12 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(PermArgs a, 
   const int rsub = threadIdx.x >> 4;      // row within the pass
   const bool sparse = (tile * RF_BLOCK >= g.P_pad) && !g.dense;
 
+  int tok[kPasses];
+  tile_sources(g, tile, rsub, tok);
   int64_t src_off[kPasses];
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p) {
-    const int r = tile * RF_BLOCK + p * kRowsPerPass + rsub;
-    const int s = rf_src_of_row(g, r);
-    src_off[p] = s < 0 ? -1 : rf_token_offset(layout, B, S, N, b, n, s) + chunk * 8;
-  }
+  for (int p = 0; p < kPasses; ++p)
+    src_off[p] = tok[p] < 0 ? -1 : rf_token_offset(layout, B, S, N, b, n, tok[p]) + chunk * 8;
   const int64_t dst_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM + chunk * 8;
 
 #pragma unroll
@@ -92,12 +106,13 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(PermArgs a, 
   __syncthreads();
   // 256 threads: 2 tensors x 128 columns.
   const int t = threadIdx.x >> 7, c = threadIdx.x & 127;
-  if (!a.pooled[t]) return;
+  float* pooled = t == 0 ? a.pooled[0] : a.pooled[1];   // constant indices: no local copy of the arguments
+  if (!pooled) return;
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < kRowsPerPass; ++i) s += red[t][i][c];
   const int blk = tile - g.P_pad / RF_BLOCK;
-  a.pooled[t][((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c] = s * (1.0f / RF_BLOCK);
+  pooled[((int64_t)bn * g.nb + blk) * RF_HEAD_DIM + c] = s * (1.0f / RF_BLOCK);
 }
 
 // fp8 form: e4m3 codes and tile scales in place of the 16-bit copies.
@@ -132,8 +147,7 @@ __global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermA
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool sparse = (tile * RF_BLOCK >= g.P_pad) && !g.dense;
   int src[kPasses];   // token of each of the thread's rows (-1: pad row)
-#pragma unroll
-  for (int p = 0; p < kPasses; ++p) src[p] = rf_src_of_row(g, tile * RF_BLOCK + p * kRowsPerPass + rsub);
+  tile_sources(g, tile, rsub, src);
   const int64_t code_base = ((int64_t)bn * g.S_int + (int64_t)tile * RF_BLOCK) * RF_HEAD_DIM;
   // every tensor's rows requested into L2 at once (one request per 128-byte
   // line, no registers held), so that the tile's DRAM reads overlap the
@@ -255,11 +269,11 @@ __global__ void __launch_bounds__(kPermThreads) unpermute_kernel(const uint16_t*
 #pragma unroll
   for (int p = 0; p < kPasses; ++p)
     buf[p] = __ldcs(reinterpret_cast<const uint4*>(o_int + src_base + (int64_t)(p * kRowsPerPass + rsub) * RF_HEAD_DIM));
+  int src[kPasses];
+  tile_sources(g, tile, rsub, src);
 #pragma unroll
-  for (int p = 0; p < kPasses; ++p) {
-    const int s = rf_src_of_row(g, tile * RF_BLOCK + p * kRowsPerPass + rsub);
-    if (s >= 0) *reinterpret_cast<uint4*>(out + rf_token_offset(layout, B, S, N, b, n, s) + chunk * 8) = buf[p];
-  }
+  for (int p = 0; p < kPasses; ++p)
+    if (src[p] >= 0) *reinterpret_cast<uint4*>(out + rf_token_offset(layout, B, S, N, b, n, src[p]) + chunk * 8) = buf[p];
 }
 
 }  // namespace

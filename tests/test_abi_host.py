@@ -326,6 +326,25 @@ def test_plain_c_caller(rfsa, tmp_path):
     assert "FAIL" not in r.stdout and r.stdout.count("ok") >= 11
 
 
+def test_block_fast_path_of_the_reorder_geometry(rfsa, tmp_path):
+    # K1 maps a sparse block's rows to tokens from the block's two 8x8 tiles
+    # (two divisions per block); a C++ program checks it against the
+    # row-by-row mapping for every sparse row of 14 plans (tests/c/geometry_host.cpp)
+    import shutil
+    import subprocess
+    gxx = shutil.which("g++")
+    if gxx is None:
+        pytest.skip("no C++ compiler")
+    exe = tmp_path / "geometry_host"
+    lib_dir = os.path.dirname(rfsa.LIB_PATH)
+    subprocess.run([gxx, "-std=c++17", "-O1", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(lib_dir, "csrc"), os.path.join(ROOT, "tests", "c", "geometry_host.cpp"),
+                    "-L", lib_dir, "-lrfsa", "-Wl,-rpath," + lib_dir, "-o", str(exe)], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert int(r.stdout.split()[0]) > 500_000
+
+
 def test_page_signature_checks(rfsa):
     # rfsa.sparse_attention takes lite_boost.ops.sparse_attention's parameter
     # list; the page's ValueErrors come before anything reaches the library
