@@ -116,7 +116,6 @@ __global__ void __launch_bounds__(kPermThreads) permute_pool_kernel(PermArgs a, 
 }
 
 // fp8 form: e4m3 codes and tile scales in place of the 16-bit copies.
-constexpr int kVtStride = RF_BLOCK + 4;   // bytes per transposed row in shared memory
 
 struct PermArgs8 {
   const uint16_t* src[3];
@@ -138,7 +137,7 @@ __global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermA
                                                                            int N, rf_plan_t g) {
   __shared__ float red[2][kRowsPerPass][RF_HEAD_DIM];
   __shared__ float red_max[3][kPermThreads / 32];
-  __shared__ __align__(16) uint8_t vt[RF_HEAD_DIM][kVtStride];
+  __shared__ __align__(16) uint32_t vr[RF_BLOCK][RF_HEAD_DIM / 4];   // V's codes, row-major, words swizzled
   const int tile = blockIdx.x;
   const int bn = blockIdx.y;
   const int b = bn / N, n = bn - b * N;
@@ -203,24 +202,25 @@ __global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermA
     const bool transposed = t == a.v_index;
     const bool pool = sparse && pooled;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // the block means' partial sums
+    const uint64_t inv2 = f2_pack(inv, inv);
 #pragma unroll
     for (int p = 0; p < kPasses; ++p) {
       if (pool) acc_half8<kF16>(acc, buf[p]);
       float f[8];
       unpack_half8<kF16>(buf[p], f);
       const int r = p * kRowsPerPass + rsub;
-      const uint32_t lo = pack_e4m3x4(__fmul_rn(f[0], inv), __fmul_rn(f[1], inv), __fmul_rn(f[2], inv),
-                                      __fmul_rn(f[3], inv));
-      const uint32_t hi = pack_e4m3x4(__fmul_rn(f[4], inv), __fmul_rn(f[5], inv), __fmul_rn(f[6], inv),
-                                      __fmul_rn(f[7], inv));
+      float y[8];
+#pragma unroll
+      for (int i = 0; i < 8; i += 2) f2_unpack(f2_mul(f2_pack(f[i], f[i + 1]), inv2), y[i], y[i + 1]);
+      const uint32_t lo = pack_e4m3x4(y[0], y[1], y[2], y[3]);
+      const uint32_t hi = pack_e4m3x4(y[4], y[5], y[6], y[7]);
       if (!transposed) {
         *reinterpret_cast<uint2*>(codes + code_base + (int64_t)r * RF_HEAD_DIM + chunk * 8) = make_uint2(lo, hi);
       } else {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          vt[chunk * 8 + i][r] = (uint8_t)(lo >> (8 * i));
-          vt[chunk * 8 + 4 + i][r] = (uint8_t)(hi >> (8 * i));
-        }
+        // row r's 8 codes at logical words 2 chunk, 2 chunk + 1, the pair
+        // moved by an even swizzle of its row group (conflict-free here,
+        // 2-way in the transposing read below)
+        *reinterpret_cast<uint2*>(&vr[r][(2 * chunk) ^ (2 * ((r >> 2) & 15))]) = make_uint2(lo, hi);
       }
     }
     if (pool) {
@@ -235,14 +235,25 @@ __global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermA
   }
   __syncthreads();   // the transposed V tile and the block means' partial sums are in place
   if (a.v_index >= 0) {
-    // the transposed V tile: 128 channel rows of 128 bytes, one word per thread and step
+    // the transposed V tile, 128 channel rows of 128 bytes: a thread takes
+    // rows 4 l .. 4 l + 3 (l its lane) of channel quads warp + 8 k, and
+    // transposes each 4 x 4 block of bytes in registers; a warp then writes
+    // 128 contiguous bytes of one channel per store
     uint8_t* codes = a.v_index == 1 ? a.dst[1] : a.dst[2];
+    const int sw = 2 * (lane & 15);
 #pragma unroll
-    for (int i = 0; i < RF_HEAD_DIM * RF_BLOCK / 4 / kPermThreads; ++i) {
-      const int idx = threadIdx.x + i * kPermThreads;
-      const int row = idx >> 5, word = idx & 31;
-      *reinterpret_cast<uint32_t*>(codes + code_base + (int64_t)row * RF_BLOCK + word * 4) =
-          *reinterpret_cast<const uint32_t*>(&vt[row][word * 4]);
+    for (int kk = 0; kk < RF_HEAD_DIM / 4 / (kPermThreads / 32); ++kk) {
+      const int cq = warp + (kPermThreads / 32) * kk;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) w[j] = vr[4 * lane + j][cq ^ sw];
+      const uint32_t t0 = __byte_perm(w[0], w[1], 0x5140), t1 = __byte_perm(w[0], w[1], 0x7362);
+      const uint32_t t2 = __byte_perm(w[2], w[3], 0x5140), t3 = __byte_perm(w[2], w[3], 0x7362);
+      const uint32_t o[4] = {__byte_perm(t0, t2, 0x5410), __byte_perm(t0, t2, 0x7632), __byte_perm(t1, t3, 0x5410),
+                             __byte_perm(t1, t3, 0x7632)};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint32_t*>(codes + code_base + (int64_t)(4 * cq + i) * RF_BLOCK + 4 * lane) = o[i];
     }
   }
   if (!sparse) return;
