@@ -59,6 +59,7 @@ def _sample_rows(g, rng, per_kind=6):
     ("minimax", {"precision": "fp8"}, (5, 50)),
     # the largest block count the library takes: 4096 sparse blocks (524,288 video tokens), one head
     ("tiny", {"N": 1, "latent": (128, 64, 64), "txt_len": 0, "sparsity": 0.5, "seed": 43}, (0,)),
+    ("tiny", {"N": 1, "latent": (128, 64, 64), "txt_len": 0, "sparsity": 0.5, "seed": 44, "precision": "fp8"}, (0,)),
 ])
 def test_full_size_sampled(name, over, heads):
     if not torch.cuda.is_available():
