@@ -1,5 +1,6 @@
 // Token reorder with block pooling fused in (K1), and the inverse reorder
-// (K4).  Both are HBM-bound row gathers/scatters of 256-byte rows.
+// (K4): row gathers/scatters of 256-byte rows, bound by HBM (K1's fp8 form,
+// which also converts every value, by its instruction issue).
 //
 // lite_boost.ops.sparse_attention, rf_v2 pipeline: token reorder, then block
 // pooling; inverse reorder at the end.  vllm-omni "RainFusion Attention":
