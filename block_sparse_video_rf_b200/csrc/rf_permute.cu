@@ -182,9 +182,10 @@ __global__ void __launch_bounds__(kPermThreads, 3) permute_pool_fp8_kernel(PermA
     // exactly (nothing unpacked stays live across the barrier)
     uint32_t m2 = 0;
 #pragma unroll
-    for (int p = 0; p < kPasses; ++p)
-      m2 = __vmaxu2(__vmaxu2(m2, buf[p].x & 0x7FFF7FFFu), __vmaxu2(buf[p].y & 0x7FFF7FFFu, 0u)),
+    for (int p = 0; p < kPasses; ++p) {
+      m2 = __vmaxu2(m2, __vmaxu2(buf[p].x & 0x7FFF7FFFu, buf[p].y & 0x7FFF7FFFu));
       m2 = __vmaxu2(m2, __vmaxu2(buf[p].z & 0x7FFF7FFFu, buf[p].w & 0x7FFF7FFFu));
+    }
     const uint32_t mbits = max(m2 & 0xFFFFu, m2 >> 16);
     float amax;
     if (kF16)
