@@ -162,6 +162,19 @@ def test_kept_count_fixed_points():
     assert all(a >= b for a, b in zip(ks, ks[1:]))
 
 
+def test_block_means_of_constant_and_index_rows():
+    # the mean of a block's 128 rows: rows all equal to c give c; rows equal
+    # to their token index give the mean of the block's token indices
+    txt, T, H, W = 16, 4, 32, 40
+    S = txt + T * H * W
+    g = oracle.geometry(S, txt, T, H, W)
+    c = np.linspace(-3, 3, 128).astype(np.float32)
+    np.testing.assert_array_equal(oracle.pool_blocks(np.tile(c, (S, 1)), g.blocks), np.tile(c, (g.nb, 1)))
+    idx = np.tile(np.arange(S, dtype=np.float32)[:, None], (1, 128))
+    want = np.array([sum(int(t) for t in blk) / 128.0 for blk in g.blocks], dtype=np.float32)
+    np.testing.assert_array_equal(oracle.pool_blocks(idx, g.blocks), np.tile(want[:, None], (1, 128)))
+
+
 # ---------------------------------------------------------------- top-k
 
 def _brute_topk(row, k):
