@@ -7,7 +7,10 @@ that should catch it: at least one must fail.  This shows that the pins fix
 the oracle's results rather than merely agreeing with them.
 """
 
+import dataclasses
+import json
 import math
+import os
 
 import numpy as np
 import pytest
@@ -16,8 +19,37 @@ import oracle
 import test_oracle_pins as pins
 from oracle import rf_v2
 
-ORIG = {n: getattr(rf_v2, n) for n in ("block_scores", "topk_mask", "kept_count", "key_set", "pool_blocks",
-                                      "_softmax_attend")}
+ORIG = {n: getattr(rf_v2, n) for n in ("geometry", "block_scores", "topk_mask", "kept_count", "key_set",
+                                      "pool_blocks", "_softmax_attend")}
+with open(os.path.join(os.path.dirname(__file__), "golden", "geometry_worked_examples.json")) as _f:
+    GOLDEN = json.load(_f)
+
+
+def _raster_transposed_in_tiles(S, txt_len, T, H, W):
+    # R1 read as column-major inside each 8x8 tile
+    g = ORIG["geometry"](S, txt_len, T, H, W)
+    if g.nb == 0:
+        return g
+    tiles = g.blocks.reshape(g.nb, 2, 8, 8).transpose(0, 1, 3, 2).reshape(g.nb, 128)
+    return dataclasses.replace(g, blocks=np.ascontiguousarray(tiles))
+
+
+def _first_frame_only_whole_blocks(S, txt_len, T, H, W):
+    # R3 read as "every token in frame 0" instead of "any token"
+    g = ORIG["geometry"](S, txt_len, T, H, W)
+    if g.nb == 0:
+        return g
+    frame = (g.blocks - txt_len) // (H * W)
+    return dataclasses.replace(g, first_frame=(frame == 0).all(axis=1))
+
+
+def _tail_dropped(S, txt_len, T, H, W):
+    # R2 read as "the aligned tokens past the last whole block are dropped"
+    g = ORIG["geometry"](S, txt_len, T, H, W)
+    if len(g.tail) == 0:
+        return g
+    keep = ~np.isin(g.prefix, g.tail)
+    return dataclasses.replace(g, prefix=g.prefix[keep], tail=g.tail[:0])
 
 
 def _ties_to_the_higher_index(scores, k, first_frame, first_frame_cols=None):
@@ -35,6 +67,9 @@ def _prefix_keys_left_out(g, mask_bn, row_block, gk=None):
 
 
 MISTAKES = {
+    "raster_transposed_in_tiles": ("geometry", _raster_transposed_in_tiles),
+    "first_frame_only_whole_blocks": ("geometry", _first_frame_only_whole_blocks),
+    "tail_dropped_not_promoted": ("geometry", _tail_dropped),
     "scores_transposed": ("block_scores", lambda qbar, kbar: ORIG["block_scores"](kbar, qbar)),
     "ties_to_the_higher_index": ("topk_mask", _ties_to_the_higher_index),
     "first_frame_columns_not_forced": (
@@ -50,6 +85,11 @@ MISTAKES = {
 
 # the pins run against each mistake (pins with parameters: a few of their cases)
 PINS = [
+    (pins.test_worked_geometry_minimax, (GOLDEN,)),
+    *[(pins.test_partition_is_a_bijection, args) for args in [(0, 4, 32, 32), (5, 5, 24, 40)]],
+    (pins.test_tile_order_by_enumeration, ()),
+    (pins.test_odd_tile_count_promotes_last_half_block, ()),
+    (pins.test_minimax_first_frame_is_eight, ()),
     (pins.test_kept_count_fixed_points, ()),
     (pins.test_block_means_of_constant_and_index_rows, ()),
     *[(pins.test_topk_matches_exhaustive_search, (seed,)) for seed in range(4)],
