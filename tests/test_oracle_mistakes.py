@@ -16,8 +16,9 @@ import numpy as np
 import pytest
 
 import oracle
+import test_oracle_fp8 as fp8_pins
 import test_oracle_pins as pins
-from oracle import rf_v2
+from oracle import fp8, rf_v2
 
 ORIG = {n: getattr(rf_v2, n) for n in ("geometry", "block_scores", "topk_mask", "kept_count", "key_set",
                                       "pool_blocks", "_softmax_attend")}
@@ -122,3 +123,79 @@ def test_a_planted_mistake_fails_a_pin(mistake, monkeypatch):
         monkeypatch.setattr(oracle, name, wrong)
     failed = _failures()
     assert failed, f"no pin caught {mistake}"
+
+
+# ---------------------------------------------------------------- e4m3 quantisation (R14)
+
+ORIG8 = {n: getattr(fp8, n) for n in ("e4m3_round", "quantize_block")}
+_POS = fp8.e4m3_values()[:0x7F]          # codes 0x00 .. 0x7E: the finite non-negative values, ascending
+
+
+def _codes_from_magnitude_index(idx, x):
+    x = np.asarray(x, dtype=np.float64)
+    return (np.asarray(idx, dtype=np.int64) | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def _toward_zero(x):
+    a = np.minimum(np.abs(np.asarray(x, dtype=np.float64)), _POS[-1])
+    return _codes_from_magnitude_index(np.searchsorted(_POS, a, side="right") - 1, x)
+
+
+def _ties_away_from_zero(x):
+    a = np.minimum(np.abs(np.asarray(x, dtype=np.float64)), _POS[-1])
+    lo = np.searchsorted(_POS, a, side="right") - 1
+    hi = np.minimum(lo + 1, len(_POS) - 1)
+    up = (_POS[hi] - a) <= (a - _POS[lo])
+    return _codes_from_magnitude_index(np.where(up, hi, lo), x)
+
+
+def _no_saturation(x):
+    codes = ORIG8["e4m3_round"](x)
+    over = np.abs(np.asarray(x, dtype=np.float64)) > fp8.E4M3_MAX
+    return np.where(over, codes | 0x7F, codes).astype(np.uint8)
+
+
+def _scale_of_127(x):
+    xf = np.asarray(x, dtype=np.float32)
+    amax = np.float32(np.max(np.abs(xf))) if xf.size else np.float32(0.0)
+    if amax == 0:
+        return np.zeros(xf.shape, dtype=np.uint8), np.float32(0.0)
+    return fp8.e4m3_round((xf * np.float32(np.float32(127.0) / amax)).astype(np.float32)), np.float32(amax / 127.0)
+
+
+MISTAKES8 = {
+    "rounding_toward_zero": ("e4m3_round", _toward_zero),
+    "ties_away_from_zero": ("e4m3_round", _ties_away_from_zero),
+    "no_saturation_above_448": ("e4m3_round", _no_saturation),
+    "scale_of_127": ("quantize_block", _scale_of_127),
+}
+PINS8 = [
+    (fp8_pins.test_rounding_matches_torch_in_range, ()),
+    (fp8_pins.test_midpoints_round_to_even_mantissa, ()),
+    (fp8_pins.test_rounding_is_nearest_by_brute_force, ()),
+    (fp8_pins.test_saturation_above_448, ()),
+    (fp8_pins.test_block_amax_maps_to_448_and_error_is_half_a_step, ()),
+    (fp8_pins.test_zero_block_has_zero_scale, ()),
+    (fp8_pins.test_scale_invariance_of_codes, ()),
+]
+
+
+def _failures8():
+    names = []
+    for pin, args in PINS8:
+        try:
+            pin(*args)
+        except Exception:
+            names.append(pin.__name__)
+    return names
+
+
+def test_the_fp8_pins_pass_on_the_oracle_as_it_stands():
+    assert _failures8() == []
+
+
+@pytest.mark.parametrize("mistake", sorted(MISTAKES8))
+def test_a_planted_fp8_mistake_fails_a_pin(mistake, monkeypatch):
+    name, wrong = MISTAKES8[mistake]
+    monkeypatch.setattr(fp8, name, wrong)
+    assert _failures8(), f"no pin caught {mistake}"
