@@ -139,12 +139,15 @@ rf_status_t cached_buffer(WsCache& c, size_t need, void** out) {
   return RF_OK;
 }
 
-// Copy streams and events of rf_sparse_attention_host, one set per device,
+// Streams and events of rf_sparse_attention_host, one set per device,
 // created on first use (non-blocking streams, so a caller on the legacy
-// default stream still overlaps with them).
+// default stream still overlaps with them): one stream for the copies in,
+// one for the copies out, and one compute stream per device slot, so that
+// a chunk's kernels can fill the SMs that the previous chunk's last units
+// (or its second pass) leave idle.
 struct HostPipe {
-  cudaStream_t in = nullptr, out = nullptr;
-  cudaEvent_t loaded[2] = {}, comp[2] = {}, stored[2] = {};
+  cudaStream_t in = nullptr, out = nullptr, comp_s[2] = {};
+  cudaEvent_t loaded[2] = {}, comp[2] = {}, stored[2] = {}, entry = nullptr;
 };
 std::mutex g_pipe_mu;
 HostPipe g_pipe[64];
@@ -160,7 +163,10 @@ rf_status_t host_pipe(HostPipe** out) {
   if (!g_pipe_ready[dev]) {
     e = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.entry, cudaEventDisableTiming);
     for (int z = 0; z < 2 && e == cudaSuccess; ++z) {
+      e = cudaStreamCreateWithFlags(&p.comp_s[z], cudaStreamNonBlocking);
+      if (e != cudaSuccess) break;
       e = cudaEventCreateWithFlags(&p.loaded[z], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.comp[z], cudaEventDisableTiming);
       if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.stored[z], cudaEventDisableTiming);
@@ -482,9 +488,10 @@ rf_status_t rf_sparse_attention_host_ex(const void* qh, const void* kh, const vo
   // Heads are independent in every precision (the fp8 scales belong to one
   // head's tiles, vmax to one head), so the call runs on chunks of c heads
   // of one batch entry, each a [1, S, c, D] (BSND) or [1, c, S, D] (BNSD)
-  // problem, in two device slots.  While chunk i computes on the caller's
-  // stream, chunk i + 1 is copied in on one stream and chunk i - 1 copied
-  // out on another.  About 96 MiB of q, k and v per chunk (2 heads at
+  // problem, in two device slots.  While chunk i computes on its slot's
+  // stream (after the work already queued on the caller's stream), chunk
+  // i + 1 is copied in on one stream and chunk i - 1 copied out on another;
+  // chunk i + 1 may start computing before chunk i's last units are done.  About 96 MiB of q, k and v per chunk (2 heads at
   // MiniMax-H3): a shorter pipeline tail than 192 MiB (52.3 vs 53.4 ms per
   // call there).  At least 2 heads when BSND: a chunk of 1 head copies
   // 256-byte rows, and the strided copy then runs far below the link's rate
@@ -505,6 +512,21 @@ rf_status_t rf_sparse_attention_host_ex(const void* qh, const void* kh, const vo
   HostPipe* hp = nullptr;
   if ((st = host_pipe(&hp)) != RF_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  {
+    cudaError_t e0 = cudaEventRecord(hp->entry, s);
+    for (int z = 0; z < 2 && e0 == cudaSuccess; ++z) e0 = cudaStreamWaitEvent(hp->comp_s[z], hp->entry, 0);
+    if (e0 != cudaSuccess) return cuda_fail(e0, "ordering the host-buffer pipeline after the caller's stream");
+  }
+  // every stream the call used has drained (also on an error: no copy of the
+  // caller's buffers may still run when this returns)
+  auto drain = [&]() {
+    cudaError_t r = cudaSuccess;
+    for (cudaStream_t x : {hp->in, hp->out, hp->comp_s[0], hp->comp_s[1], s}) {
+      const cudaError_t ex = cudaStreamSynchronize(x);
+      if (r == cudaSuccess) r = ex;
+    }
+    return r;
+  };
   const bool bsnd = layout == RF_BSND;
   const size_t row = (size_t)N * D * 2;   // BSND: one token's heads
   // `heads` heads of a tensor of `len` tokens; BSND copies `len` strided rows
@@ -536,19 +558,17 @@ rf_status_t rf_sparse_attention_host_ex(const void* qh, const void* kh, const vo
       }
       if (e != cudaSuccess || (e = cudaEventRecord(hp->loaded[z], hp->in)) != cudaSuccess) break;
       // compute once it is in and the slot's previous output has left
-      if ((e = cudaStreamWaitEvent(s, hp->loaded[z], 0)) != cudaSuccess) break;
-      if (i >= 2 && (e = cudaStreamWaitEvent(s, hp->stored[z], 0)) != cudaSuccess) break;
+      cudaStream_t cs = hp->comp_s[z];
+      if ((e = cudaStreamWaitEvent(cs, hp->loaded[z], 0)) != cudaSuccess) break;
+      if (i >= 2 && (e = cudaStreamWaitEvent(cs, hp->stored[z], 0)) != cudaSuccess) break;
       st = rf_sparse_attention_ex(dev[0], dev[1], dev[2], dtype, precision, layout, 1, S, heads, D, txt_len, T, H,
                                   W, S_kv, kv_t, kv_h, kv_w, block_size, sparsity, scale, dev[3],
-                                  static_cast<char*>(ws) + (size_t)z * ws_slot, ws_slot, stream);
+                                  static_cast<char*>(ws) + (size_t)z * ws_slot, ws_slot, cs);
       if (st != RF_OK) {
-        // no copy of the caller's buffers may still run when this returns
-        cudaStreamSynchronize(hp->in);
-        cudaStreamSynchronize(hp->out);
-        cudaStreamSynchronize(s);
+        drain();
         return st;
       }
-      if ((e = cudaEventRecord(hp->comp[z], s)) != cudaSuccess) break;
+      if ((e = cudaEventRecord(hp->comp[z], cs)) != cudaSuccess) break;
       // copy out
       if ((e = cudaStreamWaitEvent(hp->out, hp->comp[z], 0)) != cudaSuccess) break;
       if ((e = copy(outh + off(S), dev[3], heads, S, cudaMemcpyDeviceToHost, false, hp->out)) != cudaSuccess) break;
@@ -556,10 +576,8 @@ rf_status_t rf_sparse_attention_host_ex(const void* qh, const void* kh, const vo
     }
     if (e != cudaSuccess) break;
   }
-  const cudaError_t e_in = cudaStreamSynchronize(hp->in);
-  const cudaError_t e_out = cudaStreamSynchronize(hp->out);
-  const cudaError_t e_s = cudaStreamSynchronize(s);
-  if (e == cudaSuccess) e = e_in != cudaSuccess ? e_in : e_out != cudaSuccess ? e_out : e_s;
+  const cudaError_t e_drain = drain();
+  if (e == cudaSuccess) e = e_drain;
   if (e != cudaSuccess) return cuda_fail(e, "host-buffer pipeline (copies, events or synchronisation)");
   return ok();
 }

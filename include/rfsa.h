@@ -275,7 +275,9 @@ rf_status_t rf_unpermute(const void* o_int, rf_layout_t layout, int B, int S, in
  * heads (about 96 MiB of q, k and v each, and at least two heads in BSND) in
  * two device slots: chunk i + 1
  * is copied in and chunk i - 1 copied out, on two library-owned streams,
- * while chunk i computes on `stream`.  Buffers are cached by the library per
+ * while chunk i computes on its slot's library-owned stream, after the work
+ * already queued on `stream` (so that a chunk's kernels can start while the
+ * previous chunk's last units still run).  Buffers are cached by the library per
  * device.  Host buffers should be pinned: pageable ones still give the right
  * result, with the copies no longer overlapping the compute.  On return no
  * copy of the caller's buffers is in flight, also after an error. */
